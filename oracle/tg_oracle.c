@@ -1,0 +1,309 @@
+/*
+ * tg_oracle.c -- plain fp64 CPU oracle for the TokenGate prefill hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY (see tg_oracle.h): loaded by the tests, the smoke
+ * check and the CPU-baseline leg of the benchmark, never by the product path.
+ * Shares nothing with the CUDA sources.
+ *
+ * Each function follows one step of the method as the TokenGate pages state
+ * it, with the specification's formulas where the pages only name the
+ * ingredients.  No blocking, fusion or reordering: loops run in the order of
+ * the definition so that a reader can check them by eye.
+ */
+#include "tg_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+int64_t tgo_kept_count(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_doc)
+{
+    if (N < 0 || doc_begin < 0 || doc_end < doc_begin || doc_end > N || k_doc < 0)
+        return -1;
+    int64_t n_doc = doc_end - doc_begin;
+    int64_t keep_doc = k_doc < n_doc ? k_doc : n_doc;
+    return keep_doc + (N - n_doc);
+}
+
+float tgo_round_bf16(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) {
+        u |= 0x00400000u; /* quiet NaN, keep it NaN after truncation */
+        u &= 0xffff0000u;
+    } else {
+        /* round to nearest, ties to even, on the upper 16 bits */
+        uint32_t lsb = (u >> 16) & 1u;
+        u += 0x7fffu + lsb;
+        u &= 0xffff0000u;
+    }
+    float y;
+    memcpy(&y, &u, 4);
+    return y;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Gate score.  The pages: a small MLP scores each token from its
+ * post-attention residual at the gate layer (aiproducthub.cn "事件详情";
+ * chathome.org "ゲートモジュール").  The MLP shape is the specification's:
+ * RMSNorm -> Linear(d -> d_g) -> SiLU -> Linear(d_g -> 1). */
+int tgo_gate_score(const float* h, int64_t N, int d, int64_t ld_h,
+                   const float* gamma, int fold_gamma_bf16, double eps,
+                   const float* W1, const float* b1, const float* w2, double b2,
+                   int d_g, double* s)
+{
+    if (!h || !W1 || !w2 || !s || N < 0 || d <= 0 || d_g <= 0 || ld_h < d)
+        return -1;
+
+    /* Effective first-layer weight: gamma folded in (RMSNorm weight times W1). */
+    double* W = (double*)malloc(sizeof(double) * (size_t)d_g * (size_t)d);
+    if (!W)
+        return -1;
+    for (int j = 0; j < d_g; ++j) {
+        for (int c = 0; c < d; ++c) {
+            double w = W1[(size_t)j * d + c];
+            if (gamma) {
+                if (fold_gamma_bf16)
+                    w = tgo_round_bf16((float)(gamma[c] * W1[(size_t)j * d + c]));
+                else
+                    w = (double)gamma[c] * (double)W1[(size_t)j * d + c];
+            }
+            W[(size_t)j * d + c] = w;
+        }
+    }
+
+    for (int64_t i = 0; i < N; ++i) {
+        const float* hi = h + i * ld_h;
+        /* RMSNorm: r_i = 1 / sqrt(mean_c h_ic^2 + eps) */
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c)
+            ss += (double)hi[c] * (double)hi[c];
+        double r = 1.0 / sqrt(ss / (double)d + eps);
+
+        double si = b2;
+        for (int j = 0; j < d_g; ++j) {
+            /* u_ij = r_i * sum_c h_ic * W_jc + b1_j */
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += (double)hi[c] * W[(size_t)j * d + c];
+            double u = r * acc + (b1 ? (double)b1[j] : 0.0);
+            /* SiLU(u) = u * sigmoid(u) */
+            double a = u / (1.0 + exp(-u));
+            si += a * (double)w2[j];
+        }
+        s[i] = si;
+    }
+    free(W);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Top-K over the document span; the question (and anything else outside the
+ * span) is always kept (aiproducthub.cn "问题部分永远不会被剪掉"; chathome.org
+ * "質問は決してプルーニングされない").  Tie rule and ascending output order
+ * are the specification's. */
+static const float* g_sort_scores; /* qsort has no context argument */
+
+/* Negative when token a ranks before token b. */
+static int rank_cmp(const void* pa, const void* pb)
+{
+    int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+    float sa = g_sort_scores[a], sb = g_sort_scores[b];
+    int na = isnan(sa), nb = isnan(sb);
+    if (na != nb)
+        return na ? 1 : -1;          /* every number ranks above NaN */
+    if (!na && sa != sb)             /* C comparison: -0 == +0 */
+        return sa > sb ? -1 : 1;     /* larger score first */
+    return (a > b) - (a < b);        /* lower index first */
+}
+
+static int64_t sort_doc(const float* scores, int64_t doc_begin, int64_t doc_end, int32_t** out)
+{
+    int64_t n_doc = doc_end - doc_begin;
+    int32_t* order = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n_doc > 0 ? n_doc : 1));
+    if (!order)
+        return -1;
+    for (int64_t i = 0; i < n_doc; ++i)
+        order[i] = (int32_t)(doc_begin + i);
+    g_sort_scores = scores;
+    qsort(order, (size_t)n_doc, sizeof(int32_t), rank_cmp);
+    *out = order;
+    return n_doc;
+}
+
+int64_t tgo_topk_select(const float* scores, int64_t N, int64_t doc_begin,
+                        int64_t doc_end, int64_t k_doc, int32_t* kept)
+{
+    int64_t K = tgo_kept_count(N, doc_begin, doc_end, k_doc);
+    if (K < 0 || !kept || (N > 0 && !scores) || N > 2147483647)
+        return -1;
+    int32_t* order = NULL;
+    int64_t n_doc = sort_doc(scores, doc_begin, doc_end, &order);
+    if (n_doc < 0)
+        return -1;
+    int64_t keep_doc = k_doc < n_doc ? k_doc : n_doc;
+
+    unsigned char* keep = (unsigned char*)calloc((size_t)(N > 0 ? N : 1), 1);
+    if (!keep) {
+        free(order);
+        return -1;
+    }
+    for (int64_t i = 0; i < N; ++i)
+        if (i < doc_begin || i >= doc_end)
+            keep[i] = 1;
+    for (int64_t r = 0; r < keep_doc; ++r)
+        keep[order[r]] = 1;
+
+    int64_t n = 0;
+    for (int64_t i = 0; i < N; ++i)
+        if (keep[i])
+            kept[n++] = (int32_t)i;
+    free(keep);
+    free(order);
+    return n;
+}
+
+double tgo_topk_threshold(const float* scores, int64_t N, int64_t doc_begin,
+                          int64_t doc_end, int64_t k_doc)
+{
+    if (tgo_kept_count(N, doc_begin, doc_end, k_doc) < 0)
+        return NAN;
+    int32_t* order = NULL;
+    int64_t n_doc = sort_doc(scores, doc_begin, doc_end, &order);
+    if (n_doc <= 0 || k_doc == 0) {
+        free(order);
+        return NAN;
+    }
+    int64_t keep_doc = k_doc < n_doc ? k_doc : n_doc;
+    double t = scores[order[keep_doc - 1]];
+    free(order);
+    return t;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Compaction: the layers above the gate see only the kept rows, and pruned
+ * tokens get no KV entries (aiproducthub.cn "被剪掉的 token 不会再生成对应的
+ * KV 缓存条目"; chathome.org "プルーニング後の順伝播").  Original positions
+ * travel with the rows so that RoPE stays correct (specification). */
+int tgo_gather_compact(const uint16_t* h, int64_t N, int d, int64_t ld_h,
+                       const int32_t* idx, int64_t K, const int32_t* pos_in,
+                       const float* scores, uint16_t* h_out, int32_t* pos_out,
+                       float* s_out)
+{
+    if (!h || !idx || !h_out || !pos_out || d <= 0 || ld_h < d || K < 0)
+        return -1;
+    for (int64_t r = 0; r < K; ++r) {
+        int64_t i = idx[r];
+        if (i < 0 || i >= N)
+            return -1;
+        memcpy(h_out + r * (int64_t)d, h + i * ld_h, sizeof(uint16_t) * (size_t)d);
+        pos_out[r] = pos_in ? pos_in[i] : (int32_t)i;
+        if (scores && s_out)
+            s_out[r] = scores[i];
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Rotary embedding at original positions (rotate-half pairing, the Qwen3
+ * convention; the pages are silent on positions, the specification keeps
+ * the original position ids through compaction). */
+int tgo_rope(const float* x, int64_t K, int H, int d_h, const int32_t* pos,
+             double base, double* out)
+{
+    if (!x || !pos || !out || K < 0 || H <= 0 || d_h <= 0 || (d_h & 1))
+        return -1;
+    int half = d_h / 2;
+    for (int64_t r = 0; r < K; ++r) {
+        for (int hh = 0; hh < H; ++hh) {
+            const float* xr = x + (r * H + hh) * (int64_t)d_h;
+            double* o = out + (r * H + hh) * (int64_t)d_h;
+            for (int t = 0; t < half; ++t) {
+                double inv_freq = pow(base, -2.0 * (double)t / (double)d_h);
+                double ang = (double)pos[r] * inv_freq;
+                double c = cos(ang), s = sin(ang);
+                double x1 = xr[t], x2 = xr[t + half];
+                o[t] = x1 * c - x2 * s;
+                o[t + half] = x2 * c + x1 * s;
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Token-gated attention (aiproducthub.cn "token 门控注意力": the kept token's
+ * score becomes a bias on the attention logits, plus a learned per-head gain
+ * and a learned temperature; aisight.pl "Główny problem"; chathome.org
+ * "トークンゲート付きアテンションとは").  Formula from the specification:
+ *   l_{r,c} = tau * (q_r . k_c) / sqrt(d_h) + g_h * s_c   for visible c,
+ *   O_r = sum_c softmax_c(l_{r,.}) v_c. */
+int tgo_gated_attention(const float* q, const float* k, const float* v,
+                        int64_t K, int Hq, int Hkv, int d_h,
+                        const int32_t* pos, const float* s, const float* g,
+                        double tau, const int64_t* rows, int64_t n_rows,
+                        double* out, double* lse)
+{
+    if (!q || !k || !v || !out || K < 0 || Hq <= 0 || Hkv <= 0 || d_h <= 0 || (Hq % Hkv))
+        return -1;
+    if (!rows)
+        n_rows = K;
+    int group = Hq / Hkv;
+    double scale = tau / sqrt((double)d_h);
+    double* logit = (double*)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+    if (!logit)
+        return -1;
+
+    for (int64_t n = 0; n < n_rows; ++n) {
+        int64_t r = rows ? rows[n] : n;
+        if (r < 0 || r >= K) {
+            free(logit);
+            return -1;
+        }
+        for (int h = 0; h < Hq; ++h) {
+            int kvh = h / group;
+            const float* qr = q + (r * Hq + h) * (int64_t)d_h;
+            double gain = g ? (double)g[h] : 0.0;
+
+            /* logits of the visible keys, and their maximum */
+            double m = -INFINITY;
+            for (int64_t c = 0; c < K; ++c) {
+                int visible = pos ? (pos[c] <= pos[r]) : (c <= r);
+                if (!visible) {
+                    logit[c] = -INFINITY;
+                    continue;
+                }
+                const float* kc = k + (c * Hkv + kvh) * (int64_t)d_h;
+                double dot = 0.0;
+                for (int t = 0; t < d_h; ++t)
+                    dot += (double)qr[t] * (double)kc[t];
+                double l = scale * dot + gain * (s ? (double)s[c] : 0.0);
+                logit[c] = l;
+                if (l > m)
+                    m = l;
+            }
+
+            /* softmax-weighted sum of values */
+            double* o = out + (n * Hq + h) * (int64_t)d_h;
+            for (int t = 0; t < d_h; ++t)
+                o[t] = 0.0;
+            double denom = 0.0;
+            for (int64_t c = 0; c < K; ++c) {
+                if (logit[c] == -INFINITY)
+                    continue;
+                double p = exp(logit[c] - m);
+                denom += p;
+                const float* vc = v + (c * Hkv + kvh) * (int64_t)d_h;
+                for (int t = 0; t < d_h; ++t)
+                    o[t] += p * (double)vc[t];
+            }
+            for (int t = 0; t < d_h; ++t)
+                o[t] /= denom;
+            if (lse)
+                lse[n * Hq + h] = m + log(denom);
+        }
+    }
+    free(logit);
+    return 0;
+}
