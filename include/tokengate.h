@@ -1,0 +1,178 @@
+/*
+ * tokengate.h -- C ABI of libtokengate, the B200 (sm_100a) prefill hot path
+ * of TokenGate (learned token pruning for long-context prefill).
+ *
+ * The method, as the TokenGate pages describe it (aiproducthub.cn article,
+ * paragraph 事件详情; aisight.pl article, section Jak to działa; chathome.org
+ * article, sections TokenGate の学習可能なトークンプルーニングの仕組み and
+ * トークンゲート付きアテンションとは):
+ *   1. layers below the gate layer L process all N prompt tokens;
+ *   2. at layer L a small MLP scores every token from its post-attention
+ *      residual, and a top-K selector keeps the best-scored document tokens;
+ *      the question part of the prompt is never pruned;
+ *   3. layers above L process only the K kept tokens and create no KV entries
+ *      for the pruned ones;
+ *   4. in every attention above the gate, a kept token's score is a bias on
+ *      the attention logits, scaled by a learned per-head gain, with a learned
+ *      temperature that accounts for each query seeing fewer keys.
+ * The pages name these ingredients but print no formulas; the formulas used
+ * here are fixed by the specification and restated at each entry point.
+ *
+ * The four calls below are steps 2-4; tg_rope_apply is the rotary embedding
+ * applied at the tokens' original positions between the projections and the
+ * attention.
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates or frees device memory.  Scratch space is a caller-owned
+ *     device buffer of tg_workspace_bytes() bytes ("workspace"), zero-filled
+ *     once before its first use; a successful call leaves it ready for the
+ *     next call.  One workspace may be shared by all calls on one stream.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work and returns; none synchronizes, except
+ *     tg_device_status, which reads the workspace's status word back.
+ *   - bf16 tensors are passed as tg_bf16 (the 16-bit pattern of a bfloat16).
+ *   - Arguments are checked on the host before anything is launched:
+ *     TG_ERR_INVALID_ARG for NULL pointers, negative sizes, bad spans,
+ *     misaligned pointers; TG_ERR_UNSUPPORTED for shapes the kernels do not
+ *     implement (there is no fallback path); TG_ERR_CUDA when a launch fails.
+ *   - Kernels that wait on other thread blocks or on asynchronous copies wait
+ *     at most about one second; on timeout they set a bit in the workspace's
+ *     status word and return early (results are then undefined).
+ *     tg_device_status reports it as TG_ERR_TIMEOUT; re-zero the workspace
+ *     before reusing it after a timeout.
+ *   - tg_gate_score, tg_topk_select, tg_gather_compact, tg_rope_apply and
+ *     tg_gated_attention may be captured in a CUDA graph: they neither
+ *     synchronize nor allocate, and the kept count is known on the host.
+ */
+#ifndef TOKENGATE_H
+#define TOKENGATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t tg_bf16;
+
+typedef enum {
+    TG_OK = 0,
+    TG_ERR_INVALID_ARG = 1,
+    TG_ERR_UNSUPPORTED = 2,
+    TG_ERR_CUDA = 3,
+    TG_ERR_TIMEOUT = 4
+} tg_status;
+
+typedef enum {
+    TG_OP_GATE = 0,
+    TG_OP_SELECT = 1,
+    TG_OP_ATTENTION = 2,
+    TG_OP_ALL = 3 /* one buffer usable by every call */
+} tg_op;
+
+/* Bits of the device status word (first 4 bytes of the workspace). */
+#define TG_STATUS_SELECT_TIMEOUT 0x1u
+#define TG_STATUS_GATE_TIMEOUT 0x2u
+#define TG_STATUS_ATTENTION_TIMEOUT 0x4u
+
+/* Static description of a status code.  Never NULL. */
+const char* tg_status_string(tg_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t tg_version(void);
+
+/* Number of kept tokens (host-only, pure): min(k_doc, doc_end - doc_begin)
+ * document tokens plus every token outside the document span.  Returns -1 if
+ * the span is not inside [0, N] or k_doc < 0. */
+int64_t tg_kept_count(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_doc);
+
+/* Workspace bytes needed by `op` for N tokens, hidden size d, gate width d_g
+ * (arguments an op does not use are ignored).  Returns 0 for bad arguments. */
+size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g);
+
+/* Gate score (step 2: a small MLP on the post-attention residual):
+ *   r_i = (mean_c h_ic^2 + eps)^(-1/2)
+ *   u_ij = r_i * sum_c h_ic * W_jc + b1_j,   W = W1, or bf16(rms_weight (.) W1)
+ *   s_i = sum_j SiLU(u_ij) * w2_j + b2,      SiLU(u) = u / (1 + e^-u)
+ * h: [N, d] bf16, row stride ld_h elements (ld_h >= d, multiple of 8).
+ * rms_weight: [d] bf16 RMSNorm weight, or NULL for ones.  When given it is
+ *   folded into W1 once per call as bf16(rms_weight_c * W1_jc) (one rounding).
+ * W1: [d_g, d] bf16 row-major.  b1: [d_g] fp32 or NULL (zeros).
+ * w2: [d_g] fp32.  b2: scalar.  scores: [N] fp32 output.
+ * Supported: d a multiple of 64 (64..16384), d_g in {64, 128, 256},
+ * N in [0, 2^31).  h, W1 16-byte aligned.
+ * Tensor cores (tcgen05, bf16 in, fp32 accumulate in TMEM); the RMS factor,
+ * bias, SiLU and the d_g -> 1 projection are applied in the epilogue. */
+tg_status tg_gate_score(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
+                        const tg_bf16* rms_weight, float eps,
+                        const tg_bf16* W1, const float* b1, const float* w2, float b2,
+                        int32_t d_g, float* scores,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Top-K selection (step 2: top-K keeps the best-scored tokens; only the
+ * document part of the prompt is prunable, the question never is):
+ * keeps the first min(k_doc, doc_end - doc_begin) document tokens in the
+ * order (score descending, index ascending), where -0 == +0 and NaN ranks
+ * below every number, plus every token outside [doc_begin, doc_end).
+ * kept_idx: int32 output of tg_kept_count(...) entries, ascending.
+ * The result is unique, so it is bit-exact with any correct implementation.
+ * Supported: N < 2^31 and doc_end - doc_begin <= 2424832 (148 * 1024 * 16).
+ * Multi-pass radix select (11/11/10-bit digits of the order-preserving key
+ * of each fp32 score) in one cooperative launch. */
+tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_begin,
+                         int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Compaction (step 3: layers above the gate see only the K kept tokens):
+ *   h_out[r, :] = h[kept_idx[r], :]           (bit-exact copy)
+ *   pos_out[r]  = pos_in ? pos_in[kept_idx[r]] : kept_idx[r]
+ *   s_out[r]    = scores[kept_idx[r]]          (if both are non-NULL)
+ * h: [N, d] bf16 with row stride ld_h; h_out: [K, d] contiguous.
+ * kept_idx entries must lie in [0, N) (not checked on the device).
+ * Supported: d a multiple of 8; h, h_out 16-byte aligned, ld_h multiple of 8. */
+tg_status tg_gather_compact(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
+                            const int32_t* kept_idx, int64_t K, const int32_t* pos_in,
+                            const float* scores, tg_bf16* h_out, int32_t* pos_out,
+                            float* s_out, void* stream);
+
+/* Rotary embedding at the original positions, in place (rotate-half pairing
+ * (t, t + d_h/2), angle pos * base^(-2t/d_h) computed in fp64, cos/sin
+ * rounded to fp32, rotation in fp32, result rounded to bf16).
+ * q: [K, Hq, d_h] with token stride ld_q; k: [K, Hkv, d_h] with stride ld_k
+ * (strides in elements, multiples of 8; heads contiguous inside a token).
+ * pos: [K] int32.  Supported: d_h in {64, 128}. */
+tg_status tg_rope_apply(tg_bf16* q, int64_t ld_q, tg_bf16* k, int64_t ld_k,
+                        const int32_t* pos, int64_t K, int32_t Hq, int32_t Hkv,
+                        int32_t d_h, double base, void* stream);
+
+/* Token-gated causal GQA attention over the K kept tokens (step 4):
+ *   l_{r,c} = tau * (q_{r,h} . k_{c,kv(h)}) / sqrt(d_h) + gain_h * s_c,  c <= r
+ *   out_{r,h} = sum_c softmax_c(l_{r,.}) v_{c,kv(h)},  kv(h) = h / (Hq / Hkv)
+ * Causality on compacted indices equals causality on original positions
+ * because the kept indices are ascending.
+ * q: [K, Hq, d_h], k and v: [K, Hkv, d_h] bf16, token strides ld_q, ld_k,
+ * ld_v (elements, multiples of 8).  s_kept: [K] fp32 or NULL (no bias).
+ * gain: [Hq] fp32 or NULL (zeros).  out: [K, Hq, d_h] bf16 contiguous.
+ * lse: [Hq, K] fp32 natural-log sum of exp of the logits, or NULL.
+ * Supported: d_h in {64, 128}, Hq a multiple of Hkv, K < 2^31.
+ * Tensor cores for Q K^T and P V (tcgen05, accumulators in TMEM), K/V tiles
+ * staged by TMA, online softmax in fp32 with the bias added in registers,
+ * P rounded to bf16 for the P V product. */
+tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
+                             const tg_bf16* v, int64_t ld_v, int64_t K, int32_t Hq,
+                             int32_t Hkv, int32_t d_h, const float* s_kept,
+                             const float* gain, float tau, tg_bf16* out, float* lse,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads the workspace's status word after synchronizing `stream`.
+ * *status_word receives the raw TG_STATUS_* bits (may be NULL).
+ * Returns TG_ERR_TIMEOUT if any bit is set, TG_OK otherwise. */
+tg_status tg_device_status(const void* workspace, uint32_t* status_word, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOKENGATE_H */

@@ -1,0 +1,313 @@
+// topk_select.cu -- top-K over the prunable document span (TokenGate: a top-K
+// selector keeps the best-scored tokens and only the document part of the
+// prompt is prunable, the question never is; aiproducthub.cn article,
+// paragraph 事件详情; chathome.org article, section TokenGate の学習可能な
+// トークンプルーニングの仕組み).  Tie rule (lower index first) and ascending
+// output order are the specification's; NaN ranks below every number and
+// -0 equals +0.
+//
+// Design (one cooperative launch, G <= #SM blocks of 1024 threads):
+//   * every score is mapped to an order-preserving 32-bit key and kept in
+//     registers for the whole kernel (block b owns a contiguous chunk of the
+//     span, thread t the elements t, t+1024, ... of it);
+//   * three radix passes over 11/11/10-bit digits find the exact key T of the
+//     k-th document token: per pass, a shared-memory histogram built with
+//     warp-aggregated increments (__match_any_sync groups the lanes that share
+//     a digit, so skewed digit distributions do not serialise on one bank),
+//     merged into a global histogram, a grid barrier, then every block scans
+//     the global histogram redundantly and identically;
+//   * a compaction pass writes kept document indices in ascending order:
+//     position = #(keys > T before i) + min(#(keys == T before i), r), where r
+//     is the number of T-keys to keep; block prefixes come from per-block
+//     counts after one more grid barrier, in-block prefixes from ballots.
+// The grid barrier is a sense-reversing counter in the workspace that resets
+// itself; each wait is bounded and reports TG_STATUS_SELECT_TIMEOUT.
+#include "tg_host.cuh"
+
+namespace tg {
+
+__device__ __forceinline__ uint32_t radix_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN ranks lowest
+    if (u == 0x80000000u) u = 0u;                     // -0 == +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Grid-wide barrier.  Returns false (block-uniformly) if the wait timed out.
+__device__ __forceinline__ bool grid_sync(SelectScratch* sc, unsigned nblocks, unsigned int* status, int* s_ok) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        volatile unsigned int* vgen = &sc->bar_gen;
+        const unsigned int g = *vgen;
+        __threadfence();
+        const unsigned int arrived = atomicAdd(&sc->bar_count, 1u);
+        if (arrived == nblocks - 1) {
+            atomicExch(&sc->bar_count, 0u);
+            __threadfence();
+            atomicAdd(&sc->bar_gen, 1u);
+        } else {
+            const unsigned long long t0 = globaltimer_ns();
+            while (*vgen == g) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    atomicOr(status, TG_STATUS_SELECT_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        __threadfence();
+        *s_ok = ok;
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
+// Exclusive prefix of v over the 1024 threads of the block, in thread order;
+// *total receives the block sum.  s_warp: 32 words of shared memory.
+__device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* s_warp, unsigned* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        unsigned w = s_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_warp[lane] = w;
+    }
+    __syncthreads();
+    const unsigned res = (warp ? s_warp[warp - 1] : 0u) + x - v;
+    *total = s_warp[31];
+    __syncthreads();
+    return res;
+}
+
+struct SelectArgs {
+    const float* scores;
+    int64_t N, D0, D1;
+    unsigned int kd;   // document tokens kept, 0 < kd < n_doc
+    int32_t* out;
+    SelectScratch* sc;
+    unsigned int* status;
+    int ept;           // keys per thread actually used (<= EPT)
+};
+
+template <int EPT>
+__global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const SelectArgs a) {
+    __shared__ unsigned int s_hist[2048];
+    __shared__ unsigned int s_warp[32];
+    __shared__ unsigned int s_pick[2];
+    __shared__ int s_ok;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int64_t chunk = static_cast<int64_t>(a.ept) * kSelectThreads;
+    const int64_t base = a.D0 + static_cast<int64_t>(blockIdx.x) * chunk;
+    const int64_t end = min(base + chunk, a.D1);
+    const unsigned nblocks = gridDim.x;
+
+    uint32_t key[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
+        key[j] = (j < a.ept && i < end) ? radix_key(__ldg(a.scores + i)) : 0u;
+    }
+
+    uint32_t prefix = 0, pmask = 0;
+    unsigned int krem = a.kd;  // 1-based rank of the target among keys matching `prefix`
+#pragma unroll 1
+    for (int p = 0; p < 3; ++p) {
+        const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
+        const int nb = p == 2 ? 1024 : 2048;
+        const uint32_t dmask = static_cast<uint32_t>(nb - 1);
+        for (int b = tid; b < 2048; b += kSelectThreads) s_hist[b] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            if (j < a.ept) {
+                const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
+                const bool match = i < end && (key[j] & pmask) == prefix;
+                const unsigned active = __ballot_sync(0xffffffffu, match);
+                if (match) {
+                    const uint32_t digit = (key[j] >> shift) & dmask;
+                    const unsigned peers = __match_any_sync(active, digit);
+                    if (lane == __ffs(peers) - 1) atomicAdd(&s_hist[digit], static_cast<unsigned>(__popc(peers)));
+                }
+            }
+        }
+        __syncthreads();
+        for (int b = tid; b < nb; b += kSelectThreads) {
+            const unsigned c = s_hist[b];
+            if (c) atomicAdd(&a.sc->hist[p][b], c);
+        }
+        if (!grid_sync(a.sc, nblocks, a.status, &s_ok)) return;
+
+        // Locate the bin holding the krem-th largest key: scan bins from the top digit down.
+        const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
+        const unsigned c0 = d0 >= 0 ? __ldcg(&a.sc->hist[p][d0]) : 0u;
+        const unsigned c1 = d1 >= 0 ? __ldcg(&a.sc->hist[p][d1]) : 0u;
+        unsigned tot;
+        const unsigned e = block_excl_scan(c0 + c1, s_warp, &tot);
+        if (e < krem && krem <= e + c0) {
+            s_pick[0] = static_cast<unsigned>(d0);
+            s_pick[1] = e;
+        } else if (e + c0 < krem && krem <= e + c0 + c1) {
+            s_pick[0] = static_cast<unsigned>(d1);
+            s_pick[1] = e + c0;
+        }
+        __syncthreads();
+        prefix |= s_pick[0] << shift;
+        pmask |= dmask << shift;
+        krem -= s_pick[1];
+        __syncthreads();
+    }
+    const uint32_t T = prefix;
+
+    // Per-block counts of keys above T and equal to T (each < 2^16 per block).
+    unsigned cnt = 0;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
+        if (j < a.ept && i < end) cnt += (key[j] > T ? 1u : 0u) + (key[j] == T ? 0x10000u : 0u);
+    }
+    unsigned btot;
+    block_excl_scan(cnt, s_warp, &btot);
+    if (tid == 0) {
+        a.sc->blk_gt[blockIdx.x] = btot & 0xffffu;
+        a.sc->blk_eq[blockIdx.x] = btot >> 16;
+    }
+    if (!grid_sync(a.sc, nblocks, a.status, &s_ok)) return;
+
+    if (tid < 32) {
+        unsigned g = 0, q = 0;
+        for (unsigned b = lane; b < blockIdx.x; b += 32) {
+            g += __ldcg(&a.sc->blk_gt[b]);
+            q += __ldcg(&a.sc->blk_eq[b]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            q += __shfl_xor_sync(0xffffffffu, q, o);
+        }
+        if (lane == 0) {
+            s_pick[0] = g;
+            s_pick[1] = q;
+        }
+    }
+    __syncthreads();
+    unsigned run_g = s_pick[0], run_e = s_pick[1];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        if (j < a.ept) {
+            const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
+            const bool valid = i < end;
+            const bool fg = valid && key[j] > T;
+            const bool fe = valid && key[j] == T;
+            unsigned t2;
+            const unsigned ex = block_excl_scan((fg ? 1u : 0u) | (fe ? 0x10000u : 0u), s_warp, &t2);
+            const unsigned g_before = run_g + (ex & 0xffffu);
+            const unsigned e_before = run_e + (ex >> 16);
+            if (fg)
+                a.out[a.D0 + g_before + min(e_before, krem)] = static_cast<int32_t>(i);
+            else if (fe && e_before < krem)
+                a.out[a.D0 + g_before + e_before] = static_cast<int32_t>(i);
+            run_g += t2 & 0xffffu;
+            run_e += t2 >> 16;
+        }
+    }
+
+    // Tokens outside the span are always kept: [0, D0) first, [D1, N) after the kept document tokens.
+    const int64_t gstride = static_cast<int64_t>(nblocks) * kSelectThreads;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kSelectThreads + tid; i < a.D0; i += gstride)
+        a.out[i] = static_cast<int32_t>(i);
+    for (int64_t i = a.D1 + static_cast<int64_t>(blockIdx.x) * kSelectThreads + tid; i < a.N; i += gstride)
+        a.out[a.D0 + a.kd + (i - a.D1)] = static_cast<int32_t>(i);
+
+    // Every block has read the global histograms; block 0 clears them for the next call.
+    if (blockIdx.x == 0)
+        for (int b = tid; b < 3 * 2048; b += kSelectThreads) (&a.sc->hist[0][0])[b] = 0u;
+}
+
+// K_doc == 0 (only tokens outside the span) or K_doc >= N_doc (every token).
+__global__ void select_trivial_kernel(int64_t N, int64_t D0, int64_t D1, int keep_doc, int32_t* out) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N; i += stride) {
+        if (keep_doc)
+            out[i] = static_cast<int32_t>(i);
+        else if (i < D0)
+            out[i] = static_cast<int32_t>(i);
+        else if (i >= D1)
+            out[D0 + (i - D1)] = static_cast<int32_t>(i);
+    }
+}
+
+template <int EPT>
+static cudaError_t launch_select(const SelectArgs& a, int grid, cudaStream_t st) {
+    void* args[] = {const_cast<SelectArgs*>(&a)};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(topk_select_kernel<EPT>), dim3(grid),
+                                       dim3(kSelectThreads), args, 0, st);
+}
+
+}  // namespace tg
+
+using namespace tg;
+
+extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_begin, int64_t doc_end,
+                                    int64_t k_doc, int32_t* kept_idx, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+    const int64_t K = tg_kept_count(N, doc_begin, doc_end, k_doc);
+    if (K < 0) return TG_ERR_INVALID_ARG;
+    if (N > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
+    if (K == 0) return TG_OK;
+    if (!scores || !kept_idx) return TG_ERR_INVALID_ARG;
+    const int64_t n_doc = doc_end - doc_begin;
+    const int64_t kd = k_doc < n_doc ? k_doc : n_doc;
+    cudaStream_t st = as_stream(stream);
+    if (kd == 0 || kd == n_doc) {
+        const int64_t blocks = std::min<int64_t>((N + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
+        select_trivial_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(N, doc_begin, doc_end,
+                                                                             kd == n_doc ? 1 : 0, kept_idx);
+        return launch_status();
+    }
+    if (!workspace || workspace_bytes < tg_workspace_bytes(TG_OP_SELECT, N, 0, 0)) return TG_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return TG_ERR_INVALID_ARG;
+    const int sms = num_sms();
+    const int64_t per_block_min = kSelectThreads;
+    int64_t ept = (n_doc + static_cast<int64_t>(sms) * per_block_min - 1) / (static_cast<int64_t>(sms) * per_block_min);
+    if (ept < 1) ept = 1;
+    if (ept > kSelectMaxEpt) return TG_ERR_UNSUPPORTED;
+    const int64_t chunk = ept * kSelectThreads;
+    const int grid = static_cast<int>((n_doc + chunk - 1) / chunk);
+    if (grid > kSelectMaxBlocks) return TG_ERR_UNSUPPORTED;
+
+    SelectArgs a;
+    a.scores = scores;
+    a.N = N;
+    a.D0 = doc_begin;
+    a.D1 = doc_end;
+    a.kd = static_cast<unsigned int>(kd);
+    a.out = kept_idx;
+    a.sc = reinterpret_cast<SelectScratch*>(static_cast<char*>(workspace) + kWsHeader);
+    a.status = status_word(workspace);
+    a.ept = static_cast<int>(ept);
+    cudaError_t e;
+    if (ept <= 1)
+        e = launch_select<1>(a, grid, st);
+    else if (ept <= 2)
+        e = launch_select<2>(a, grid, st);
+    else if (ept <= 4)
+        e = launch_select<4>(a, grid, st);
+    else if (ept <= 8)
+        e = launch_select<8>(a, grid, st);
+    else
+        e = launch_select<16>(a, grid, st);
+    return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;
+}

@@ -1,0 +1,213 @@
+"""Thin Python binding of libtokengate (argument marshalling only).
+
+Every function has the name of the C entry point it calls (include/tokengate.h)
+and takes torch CUDA tensors; it checks dtypes, shapes and strides, passes raw
+device pointers and torch's current CUDA stream, and raises TokenGateError on a
+non-OK status.  All computation happens in the library's kernels.  There is no
+CPU fallback: if libtokengate.so is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtokengate.so")
+
+TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_CUDA, TG_ERR_TIMEOUT = range(5)
+TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL = range(4)
+
+_lib = None
+
+
+class TokenGateError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m learned_token_pruning_tg_b200.build` (no fallback path exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, f32, f64, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float,
+                                      ctypes.c_double, ctypes.c_size_t)
+        L.tg_status_string.argtypes = [ctypes.c_int]
+        L.tg_status_string.restype = ctypes.c_char_p
+        L.tg_version.restype = i32
+        L.tg_kept_count.argtypes = [i64, i64, i64, i64]
+        L.tg_kept_count.restype = i64
+        L.tg_workspace_bytes.argtypes = [ctypes.c_int, i64, i32, i32]
+        L.tg_workspace_bytes.restype = sz
+        L.tg_gate_score.argtypes = [vp, i64, i32, i64, vp, f32, vp, vp, vp, f32, i32, vp, vp, sz, vp]
+        L.tg_topk_select.argtypes = [vp, i64, i64, i64, i64, vp, vp, sz, vp]
+        L.tg_gather_compact.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, vp, vp, vp]
+        L.tg_rope_apply.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, f64, vp]
+        L.tg_gated_attention.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp,
+                                         vp, sz, vp]
+        L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
+        for fn in ("tg_gate_score", "tg_topk_select", "tg_gather_compact", "tg_rope_apply",
+                   "tg_gated_attention", "tg_device_status"):
+            getattr(L, fn).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().tg_status_string(status).decode()
+
+
+def _check(fn: str, status: int):
+    if status != TG_OK:
+        raise TokenGateError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _req(t, name, dtype, dim=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dims, got {t.dim()}")
+
+
+def _row_stride(t, name):
+    """Token stride (elements) of a [rows, ...] tensor whose trailing dims are dense."""
+    inner = 1
+    for d in range(t.dim() - 1, 0, -1):
+        if t.size(d) != 1 and t.stride(d) != inner:
+            raise ValueError(f"{name}: trailing dims must be contiguous")
+        inner *= t.size(d)
+    return t.stride(0) if t.size(0) > 1 else max(inner, 1)
+
+
+def tg_version() -> int:
+    return int(lib().tg_version())
+
+
+def tg_kept_count(N: int, doc_begin: int, doc_end: int, k_doc: int) -> int:
+    return int(lib().tg_kept_count(N, doc_begin, doc_end, k_doc))
+
+
+def tg_workspace_bytes(op: int, N: int, d: int = 0, d_g: int = 0) -> int:
+    return int(lib().tg_workspace_bytes(op, N, d, d_g))
+
+
+def new_workspace(N: int, d: int = 0, d_g: int = 0, op: int = TG_OP_ALL, device=None) -> torch.Tensor:
+    """A zero-filled device workspace usable by every call (torch allocates it)."""
+    n = tg_workspace_bytes(op, N, d, d_g)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def tg_gate_score(h, W1, w2, scores, workspace, b1=None, b2: float = 0.0, rms_weight=None,
+                  eps: float = 1e-6, stream=None):
+    _req(h, "h", torch.bfloat16, 2)
+    _req(W1, "W1", torch.bfloat16, 2)
+    _req(w2, "w2", torch.float32, 1)
+    _req(scores, "scores", torch.float32, 1)
+    _req(b1, "b1", torch.float32, 1)
+    _req(rms_weight, "rms_weight", torch.bfloat16, 1)
+    N, d = h.shape
+    d_g = W1.shape[0]
+    if h.stride(1) != 1 or not W1.is_contiguous() or not w2.is_contiguous() or not scores.is_contiguous():
+        raise ValueError("h rows, W1, w2 and scores must be dense")
+    if W1.shape[1] != d or w2.shape[0] != d_g or scores.shape[0] != N:
+        raise ValueError("shape mismatch")
+    ld_h = h.stride(0) if N > 1 else d
+    _check("tg_gate_score", lib().tg_gate_score(
+        _ptr(h), N, d, ld_h, _ptr(rms_weight), eps, _ptr(W1), _ptr(b1), _ptr(w2), b2, d_g,
+        _ptr(scores), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return scores
+
+
+def tg_topk_select(scores, doc_begin: int, doc_end: int, k_doc: int, kept_idx, workspace, stream=None):
+    _req(scores, "scores", torch.float32, 1)
+    _req(kept_idx, "kept_idx", torch.int32, 1)
+    N = scores.shape[0]
+    K = tg_kept_count(N, doc_begin, doc_end, k_doc)
+    if K < 0:
+        raise TokenGateError("tg_topk_select", TG_ERR_INVALID_ARG)
+    if kept_idx.numel() < K or not scores.is_contiguous() or not kept_idx.is_contiguous():
+        raise ValueError("kept_idx too small or not contiguous")
+    _check("tg_topk_select", lib().tg_topk_select(
+        _ptr(scores), N, doc_begin, doc_end, k_doc, _ptr(kept_idx), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return kept_idx
+
+
+def tg_gather_compact(h, kept_idx, h_out, pos_out, pos_in=None, scores=None, s_out=None, stream=None):
+    _req(h, "h", torch.bfloat16, 2)
+    _req(h_out, "h_out", torch.bfloat16, 2)
+    _req(kept_idx, "kept_idx", torch.int32, 1)
+    _req(pos_out, "pos_out", torch.int32, 1)
+    _req(pos_in, "pos_in", torch.int32, 1)
+    _req(scores, "scores", torch.float32, 1)
+    _req(s_out, "s_out", torch.float32, 1)
+    N, d = h.shape
+    K = kept_idx.shape[0]
+    if h.stride(1) != 1 or not h_out.is_contiguous() or h_out.shape != (K, d):
+        raise ValueError("h rows must be dense and h_out [K, d] contiguous")
+    ld_h = h.stride(0) if N > 1 else d
+    _check("tg_gather_compact", lib().tg_gather_compact(
+        _ptr(h), N, d, ld_h, _ptr(kept_idx), K, _ptr(pos_in), _ptr(scores), _ptr(h_out), _ptr(pos_out),
+        _ptr(s_out), _stream(stream)))
+    return h_out, pos_out, s_out
+
+
+def tg_rope_apply(q, k, pos, base: float = 1e6, stream=None):
+    """In place on q [K, Hq, d_h] and k [K, Hkv, d_h] (token stride may be padded)."""
+    _req(q, "q", torch.bfloat16, 3)
+    _req(k, "k", torch.bfloat16, 3)
+    _req(pos, "pos", torch.int32, 1)
+    K, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    _check("tg_rope_apply", lib().tg_rope_apply(
+        _ptr(q), _row_stride(q, "q"), _ptr(k), _row_stride(k, "k"), _ptr(pos), K, Hq, Hkv, d_h, base,
+        _stream(stream)))
+    return q, k
+
+
+def tg_gated_attention(q, k, v, out, workspace, s_kept=None, gain=None, tau: float = 1.0, lse=None,
+                       stream=None):
+    _req(q, "q", torch.bfloat16, 3)
+    _req(k, "k", torch.bfloat16, 3)
+    _req(v, "v", torch.bfloat16, 3)
+    _req(out, "out", torch.bfloat16, 3)
+    _req(s_kept, "s_kept", torch.float32, 1)
+    _req(gain, "gain", torch.float32, 1)
+    _req(lse, "lse", torch.float32, 2)
+    K, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    if not out.is_contiguous() or out.shape != (K, Hq, d_h):
+        raise ValueError("out must be a contiguous [K, Hq, d_h] tensor")
+    _check("tg_gated_attention", lib().tg_gated_attention(
+        _ptr(q), _row_stride(q, "q"), _ptr(k), _row_stride(k, "k"), _ptr(v), _row_stride(v, "v"), K, Hq, Hkv,
+        d_h, _ptr(s_kept), _ptr(gain), tau, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return out
+
+
+def tg_device_status(workspace, stream=None) -> int:
+    """Raw status bits of the workspace (synchronizes the stream); raises on timeout bits."""
+    w = ctypes.c_uint32(0)
+    st = lib().tg_device_status(_ptr(workspace), ctypes.byref(w), _stream(stream))
+    if st not in (TG_OK, TG_ERR_TIMEOUT):
+        raise TokenGateError("tg_device_status", st)
+    return int(w.value)

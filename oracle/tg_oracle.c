@@ -45,8 +45,9 @@ float tgo_round_bf16(float x)
 
 /* ------------------------------------------------------------------------ */
 /* Gate score.  The pages: a small MLP scores each token from its
- * post-attention residual at the gate layer (aiproducthub.cn "事件详情";
- * chathome.org "ゲートモジュール").  The MLP shape is the specification's:
+ * post-attention residual at the gate layer (aiproducthub.cn article,
+ * paragraph 事件详情; chathome.org article, section TokenGate の学習可能な
+ * トークンプルーニングの仕組み).  The MLP shape is the specification's:
  * RMSNorm -> Linear(d -> d_g) -> SiLU -> Linear(d_g -> 1). */
 int tgo_gate_score(const float* h, int64_t N, int d, int64_t ld_h,
                    const float* gamma, int fold_gamma_bf16, double eps,
@@ -100,8 +101,9 @@ int tgo_gate_score(const float* h, int64_t N, int d, int64_t ld_h,
 
 /* ------------------------------------------------------------------------ */
 /* Top-K over the document span; the question (and anything else outside the
- * span) is always kept (aiproducthub.cn "问题部分永远不会被剪掉"; chathome.org
- * "質問は決してプルーニングされない").  Tie rule and ascending output order
+ * span) is always kept (aiproducthub.cn article, paragraph 事件详情;
+ * chathome.org article, section TokenGate の学習可能なトークンプルーニングの
+ * 仕組み).  Tie rule and ascending output order
  * are the specification's. */
 static const float* g_sort_scores; /* qsort has no context argument */
 
@@ -183,8 +185,9 @@ double tgo_topk_threshold(const float* scores, int64_t N, int64_t doc_begin,
 
 /* ------------------------------------------------------------------------ */
 /* Compaction: the layers above the gate see only the kept rows, and pruned
- * tokens get no KV entries (aiproducthub.cn "被剪掉的 token 不会再生成对应的
- * KV 缓存条目"; chathome.org "プルーニング後の順伝播").  Original positions
+ * tokens get no KV entries (aiproducthub.cn article, paragraph 事件详情;
+ * chathome.org article, section TokenGate の学習可能なトークンプルーニングの
+ * 仕組み).  Original positions
  * travel with the rows so that RoPE stays correct (specification). */
 int tgo_gather_compact(const uint16_t* h, int64_t N, int d, int64_t ld_h,
                        const int32_t* idx, int64_t K, const int32_t* pos_in,
@@ -233,10 +236,11 @@ int tgo_rope(const float* x, int64_t K, int H, int d_h, const int32_t* pos,
 }
 
 /* ------------------------------------------------------------------------ */
-/* Token-gated attention (aiproducthub.cn "token 门控注意力": the kept token's
- * score becomes a bias on the attention logits, plus a learned per-head gain
- * and a learned temperature; aisight.pl "Główny problem"; chathome.org
- * "トークンゲート付きアテンションとは").  Formula from the specification:
+/* Token-gated attention: the kept token's score becomes a bias on the
+ * attention logits, plus a learned per-head gain and a learned temperature
+ * (aiproducthub.cn article, paragraph 事件详情; aisight.pl article, section
+ * Jak to działa; chathome.org article, section トークンゲート付きアテンション
+ * とは).  Formula from the specification:
  *   l_{r,c} = tau * (q_r . k_c) / sqrt(d_h) + g_h * s_c   for visible c,
  *   O_r = sum_c softmax_c(l_{r,.}) v_c. */
 int tgo_gated_attention(const float* q, const float* k, const float* v,

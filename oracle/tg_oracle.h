@@ -16,15 +16,16 @@
  * prefill", Patel, Ranjan, Stoica, Zaharia, Guestrin):
  *   - three-phase forward, gate on the post-attention residual at layer L,
  *     top-K keeps the best-scored tokens, upper layers see only K tokens:
- *     aiproducthub.cn article (paragraph "事件详情"), aisight.pl article
- *     ("Jak to działa"), chathome.org article ("TokenGate の学習可能な
- *     トークンプルーニングの仕組み");
+ *     aiproducthub.cn article (paragraph 事件详情), aisight.pl article
+ *     (section Jak to działa), chathome.org article (section TokenGate の
+ *     学習可能なトークンプルーニングの仕組み);
  *   - only the document part of the prompt is prunable, the question never:
  *     same three sections;
  *   - token-gated attention: each kept token's score becomes a bias on the
  *     attention logits above the gate, with a learned per-head gain and a
- *     learned temperature: aiproducthub.cn ("token 门控注意力"), aisight.pl
- *     ("Główny problem"), chathome.org ("トークンゲート付きアテンションとは").
+ *     learned temperature: aiproducthub.cn (paragraph 事件详情), aisight.pl
+ *     (section Jak to działa), chathome.org (section トークンゲート付き
+ *     アテンションとは).
  * The pages give the ingredients but not the formulas; the formulas below are
  * the task specification's:
  *   gate:  s_i = w2 . SiLU(r_i * (h_i . (gamma*W1)^T) + b1) + b2,

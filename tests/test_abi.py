@@ -1,0 +1,83 @@
+"""The C-ABI library builds, loads, and exports every entry point include/*.h declares.
+
+Host-only checks (no device work): kept count, workspace sizes, status strings.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from learned_token_pruning_tg_b200 import build as tg_build
+from learned_token_pruning_tg_b200 import tokengate as tg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(tg_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tg_build.build()
+    return tg.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "tg_gate_score" in names and "tg_gated_attention" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_only_tg_symbols_exported():
+    out = os.popen(f"nm -D --defined-only {tg.LIB_PATH}").read().split("\n")
+    syms = [l.split()[-1] for l in out if l.strip()]
+    bad = [s for s in syms if not s.startswith("tg_")]
+    assert not bad, bad
+
+
+def test_host_only_calls(lib):
+    assert tg.tg_kept_count(131072, 0, 130560, 4096) == 4608
+    assert tg.tg_kept_count(16384, 0, 16000, 1024) == 1408
+    assert tg.tg_kept_count(10, 2, 8, 100) == 10
+    assert tg.tg_kept_count(10, 2, 11, 1) == -1
+    assert tg.tg_kept_count(10, 3, 2, 1) == -1
+    assert tg.tg_kept_count(10, 2, 8, -1) == -1
+    assert tg.tg_workspace_bytes(tg.TG_OP_SELECT, 131072) > 256
+    assert tg.tg_workspace_bytes(tg.TG_OP_GATE, 131072, 2048, 256) >= 2048 * 256 * 2
+    assert tg.tg_workspace_bytes(tg.TG_OP_ALL, 131072, 2048, 256) >= tg.tg_workspace_bytes(tg.TG_OP_SELECT, 1)
+    assert tg.tg_workspace_bytes(tg.TG_OP_GATE, -1, 2048, 256) == 0
+    assert tg.status_string(tg.TG_OK) == "ok"
+    assert "timed out" in tg.status_string(tg.TG_ERR_TIMEOUT)
+    assert tg.tg_version() >= 100
+
+
+def test_argument_errors_before_launch(lib):
+    # Host validation rejects bad arguments without touching the device.
+    vp = ctypes.c_void_p
+    assert lib.tg_topk_select(None, 10, 2, 11, 1, None, None, 0, None) == tg.TG_ERR_INVALID_ARG
+    assert lib.tg_topk_select(vp(16), 10, 2, 8, 3, None, None, 0, None) == tg.TG_ERR_INVALID_ARG
+    assert lib.tg_gather_compact(vp(16), 10, 12, 12, None, 3, None, None, vp(16), vp(16), None,
+                                 None) == tg.TG_ERR_INVALID_ARG
+    assert lib.tg_gather_compact(vp(16), 10, 12, 12, vp(16), 3, None, None, vp(16), vp(16), None,
+                                 None) == tg.TG_ERR_UNSUPPORTED          # d % 8 != 0
+    assert lib.tg_rope_apply(vp(16), 96 * 2, vp(16), 96, vp(16), 4, 2, 1, 96, 1e6,
+                             None) == tg.TG_ERR_UNSUPPORTED              # d_h = 96
+    assert lib.tg_gate_score(vp(16), 10, 100, 100, None, 1e-6, vp(16), None, vp(16), 0.0, 64, vp(16),
+                             vp(256), 1 << 20, None) == tg.TG_ERR_UNSUPPORTED   # d % 64 != 0
+    assert lib.tg_gate_score(vp(16), 10, 128, 128, None, 1e-6, vp(16), None, vp(16), 0.0, 96, vp(16),
+                             vp(256), 1 << 20, None) == tg.TG_ERR_UNSUPPORTED   # d_g = 96
+    assert lib.tg_gated_attention(vp(16), 128, vp(16), 128, vp(16), 128, 5, 3, 2, 64, None, None, 1.0,
+                                  vp(16), None, vp(256), 256, None) == tg.TG_ERR_INVALID_ARG  # Hq % Hkv
+    assert lib.tg_gated_attention(vp(16), 96, vp(16), 96, vp(16), 96, 5, 1, 1, 96, None, None, 1.0,
+                                  vp(16), None, vp(256), 256, None) == tg.TG_ERR_UNSUPPORTED  # d_h = 96
+    assert lib.tg_gated_attention(vp(17), 128, vp(16), 128, vp(16), 128, 5, 2, 2, 64, None, None, 1.0,
+                                  vp(16), None, vp(256), 256, None) == tg.TG_ERR_INVALID_ARG  # misaligned

@@ -2,8 +2,9 @@
 
 Token-gated attention (TokenGate pages: kept-token score as a bias on the
 attention logits above the gate, a learned per-head gain and a learned
-temperature, aiproducthub.cn "token 门控注意力", aisight.pl "Główny problem",
-chathome.org "トークンゲート付きアテンションとは"); the formula
+temperature: aiproducthub.cn article, paragraph 事件详情; aisight.pl article,
+section Jak to działa; chathome.org article, section トークンゲート付き
+アテンションとは); the formula
 l = tau q.k / sqrt(d_h) + g_h s_c is the specification's.
 """
 import math

@@ -1,8 +1,9 @@
 """Pins of the oracle's gate score against facts that do not come from the oracle.
 
 Gate (TokenGate pages: a small MLP scores every token's post-attention
-residual at the gate layer, aiproducthub.cn "事件详情", chathome.org
-"ゲートモジュール"); the MLP shape RMSNorm -> Linear -> SiLU -> Linear is the
+residual at the gate layer: aiproducthub.cn article, paragraph 事件详情;
+chathome.org article, section TokenGate の学習可能なトークンプルーニングの仕組み);
+the MLP shape RMSNorm -> Linear -> SiLU -> Linear is the
 specification's.
 """
 import math

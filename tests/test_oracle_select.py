@@ -1,8 +1,9 @@
 """Pins of the oracle's top-K selection.
 
 Selection rule (TokenGate pages: top-K keeps the best-scored tokens and the
-question is never pruned, aiproducthub.cn "事件详情", aisight.pl "Jak to
-działa", chathome.org "ゲートモジュール"); tie rule (lower index first) and the
+question is never pruned: aiproducthub.cn article, paragraph 事件详情;
+aisight.pl article, section Jak to działa; chathome.org article, section
+TokenGate の学習可能なトークンプルーニングの仕組み); tie rule (lower index first) and the
 ascending output order are the specification's; NaN ranks below every number
 and -0 equals +0 (a reading where both are silent).
 """
