@@ -200,8 +200,10 @@ gate_score_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_const
         for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
             const int buf = static_cast<int>(it & 1);
             const uint32_t par = static_cast<uint32_t>(it >> 1) & 1;
-            if (!mbar_wait(&acc_full[buf], par, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT)) break;
-            if (!mbar_wait(&ss_full[buf], par, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT)) break;
+            // warp-uniform outcome: tcgen05.ld below is warp-collective
+            bool ok = mbar_wait(&acc_full[buf], par, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT) &&
+                      mbar_wait(&ss_full[buf], par, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT);
+            if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const float r = rsqrtf(ss_s[buf * kBM + row] * inv_d + a.eps);
             float acc = 0.0f;

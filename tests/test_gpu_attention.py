@@ -1,0 +1,129 @@
+"""GPU parity of tg_gated_attention against the oracle.
+
+Tolerance (the specification: max abs error 1e-2 with bf16 I/O and fp32
+accumulation).  The output itself is bf16, so the comparison removes the one
+unavoidable rounding of each output element: for every element,
+|O_gpu - O_oracle| - halfulp_bf16(O_oracle) <= 1e-2.  The remaining error is
+the kernel's arithmetic (P rounded to bf16 for the P V product, fp32 online
+softmax with ex2.approx).  The log-sum-exp agrees to 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from learned_token_pruning_tg_b200 import synth
+from learned_token_pruning_tg_b200 import tokengate as tg
+from tests import oracle_pool
+
+pytestmark = pytest.mark.gpu
+
+ATTN_TOL = 1e-2
+LSE_TOL = 1e-3
+
+
+def half_ulp_bf16(x):
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - 8), 0.0)
+
+
+def run_gpu(d, fused=False, want_lse=True, use_bias=True):
+    K, Hq, d_h = d.q.shape
+    Hkv = d.k.shape[1]
+    if fused:
+        # q, k, v as strided views of one [K, (Hq + 2 Hkv) d_h] projection output
+        buf = torch.cat([d.q.reshape(K, -1), d.k.reshape(K, -1), d.v.reshape(K, -1)], dim=1).cuda()
+        q = buf[:, : Hq * d_h].view(K, Hq, d_h)
+        k = buf[:, Hq * d_h: (Hq + Hkv) * d_h].view(K, Hkv, d_h)
+        v = buf[:, (Hq + Hkv) * d_h:].view(K, Hkv, d_h)
+    else:
+        q, k, v = d.q.cuda(), d.k.cuda(), d.v.cuda()
+    out = torch.full((K, Hq, d_h), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((Hq, K), float("nan"), device="cuda") if want_lse else None
+    ws = tg.new_workspace(K, op=tg.TG_OP_ATTENTION)
+    tg.tg_gated_attention(q, k, v, out, ws, s_kept=d.s.cuda() if use_bias else None,
+                          gain=d.gain.cuda() if use_bias else None, tau=d.tau, lse=lse)
+    torch.cuda.synchronize()
+    assert tg.tg_device_status(ws) == 0
+    return out.float().cpu().numpy(), (lse.cpu().numpy() if want_lse else None)
+
+
+def check(d, rows=None, fused=False, use_bias=True):
+    K = d.q.shape[0]
+    got, lse = run_gpu(d, fused=fused, use_bias=use_bias)
+    rows = np.arange(K) if rows is None else np.asarray(rows)
+    q, k, v = (t.float().numpy() for t in (d.q, d.k, d.v))
+    s = d.s.numpy() if use_bias else None
+    g = d.gain.numpy() if use_bias else None
+    want = oracle_pool.gated_attention(q, k, v, s=s, g=g, tau=d.tau, rows=rows)
+    g_rows = got[rows].astype(np.float64)
+    assert np.all(np.isfinite(g_rows))
+    excess = np.abs(g_rows - want) - half_ulp_bf16(want)
+    assert np.max(excess) <= ATTN_TOL, (np.max(excess), np.unravel_index(np.argmax(excess), excess.shape))
+    # log-sum-exp from the same logits (oracle: natural log of the sum of exp)
+    import oracle
+    _, want_lse = oracle.gated_attention(q, k, v, s=s, g=g, tau=d.tau, rows=rows[:64], want_lse=True)
+    assert np.max(np.abs(lse[:, rows[:64]].T - want_lse)) <= LSE_TOL
+    return float(np.max(np.abs(g_rows - want)))
+
+
+@pytest.mark.parametrize("K,Hq,Hkv,d_h", [
+    (256, 4, 2, 64),        # tiny workload shape
+    (1408, 16, 8, 128),     # 16k workload: K = 1024 + 384
+    (1, 2, 1, 128),         # single token: O = v_0
+    (127, 4, 4, 64),        # one ragged tile, MHA
+    (129, 8, 2, 128),       # two tiles, 1-row tail, GQA 4
+    (1000, 16, 8, 64),
+    (2561, 16, 8, 128),     # 32k sweep K_doc=2048 plus question, ragged
+])
+def test_attention_small(K, Hq, Hkv, d_h):
+    d = synth.qkv(K, Hq, Hkv, d_h, seed=K * 7 + d_h)
+    check(d)
+
+
+def test_attention_strided_views_and_no_bias():
+    d = synth.qkv(777, 16, 8, 128, seed=5)
+    check(d, fused=True)
+    check(d, use_bias=False)
+
+
+def test_attention_k_eq_n_plain_causal_against_torch():
+    # K = N, g = 0, tau = 1: ordinary causal attention (the 32k full-prefill run's reduction).
+    d = synth.qkv(1024, 16, 8, 128, seed=9)
+    d.gain.zero_()
+    d.tau = 1.0
+    got, _ = run_gpu(d)
+    q, k, v = (t.cuda().transpose(0, 1).float() for t in (d.q, d.k, d.v))
+    k = k.repeat_interleave(2, 0)
+    v = v.repeat_interleave(2, 0)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True).transpose(0, 1).cpu().numpy()
+    excess = np.abs(got - ref) - half_ulp_bf16(ref)
+    assert np.max(excess) <= ATTN_TOL
+    check(d, rows=np.arange(0, 1024, 5))
+
+
+def test_attention_128k_workload_sampled_rows():
+    # K = 4608 kept tokens of the 128k workload with 3% of rows scaled x3 (heavy rows).
+    d = synth.qkv(4608, 16, 8, 128, seed=128, n_pos=131072, heavy_frac=0.03)
+    rows = np.unique(np.concatenate([np.arange(0, 4608, 23), np.arange(4608 - 130, 4608), np.arange(0, 130)]))
+    check(d, rows=rows)
+
+
+def test_attention_large_k_sampled_rows():
+    d = synth.qkv(16896, 16, 8, 128, seed=3204, n_pos=32768)
+    rows = np.unique(np.concatenate([np.arange(0, 16896, 131), np.arange(16896 - 40, 16896)]))
+    check(d, rows=rows)
+
+
+def test_attention_dominant_key_and_bias_matters():
+    # One key with a very large score and gain dominates every later row: output -> v_c.
+    d = synth.qkv(300, 4, 2, 64, seed=11)
+    d.s[57] = 60.0
+    d.gain.fill_(1.5)
+    got, _ = run_gpu(d)
+    v57 = d.v[57].float().numpy()            # [Hkv, d_h]
+    want = np.repeat(v57, 2, axis=0)          # query heads 2g, 2g+1 read kv head g
+    assert np.max(np.abs(got[57:] - want[None])) <= 1e-2
+    check(d)
