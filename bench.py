@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the TokenGate prefill hot path on B200: prefill tokens/s through
+gate -> top-K -> gather -> (QKV projection, RoPE) -> token-gated attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tokengate|reference]
+
+One step = one pass of the whole path over the 128k-token workload (Qwen3-1.7B
+gate layer: N = 131072 tokens, document 130560, question 512, hidden 2048,
+gate 2048 -> 256 -> 1, K_doc = 4096 so K = 4608 kept tokens, 16 query / 8 KV
+heads of 128, 3% of the rows scaled x3).  Inputs are synthetic and seeded;
+h (537 MB) is larger than the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs its own replica (independent prefills,
+"scaling": "weak"); the only collectives are the barrier and the max-over-ranks
+of the device time.  Rank 0 prints one JSON line.
+
+--impl reference runs the CPU oracle (single thread) on a bounded sample of
+each step's work and extrapolates to the full workload; only rank 0 works.
+"""
+import argparse
+import faulthandler
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from learned_token_pruning_tg_b200 import synth  # noqa: E402
+
+METRIC = "prefill tokens/s through gate+top-K+gated attention at 16k–128k; % roofline"
+WORKLOAD = synth.L128K
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def config_dict(w):
+    return {"workload": f"{w.name}: gate layer, N={w.N} (document {w.n_doc}, question {w.N - w.n_doc}), "
+                        f"K_doc={w.k_doc} -> K={w.K}",
+            "N": w.N, "doc_span": [w.doc_begin, w.doc_end], "k_doc": w.k_doc, "K": w.K, "d": w.d, "d_g": w.d_g,
+            "Hq": w.Hq, "Hkv": w.Hkv, "d_h": w.d_h, "heavy_rows": f"{w.n_scaled} rows x{w.scale}",
+            "l2": "inputs larger than L2 (h is N*d*2 = 537 MB > 126 MB L2); no flush",
+            "path": "gate, select, gather, qkv (cuBLAS glue), rope, attention", "seed": w.seed}
+
+
+# ---------------------------------------------------------------- algorithmic work per stage
+def stage_work(w):
+    """Algorithmic FLOPs and bytes of each stage (per step)."""
+    N, d, dg, K, Hq, Hkv, dh = w.N, w.d, w.d_g, w.K, w.Hq, w.Hkv, w.d_h
+    return {
+        "gate": {"flops": 2.0 * N * d * dg, "bytes": N * d * 2 + dg * d * 2 + dg * 4 + N * 4},
+        "select": {"flops": 0.0, "bytes": N * 4 + K * 4},
+        "gather": {"flops": 0.0, "bytes": 2.0 * K * d * 2 + K * 4 * 4},
+        "rope": {"flops": 0.0, "bytes": 2.0 * K * (Hq + Hkv) * dh * 2 + K * 4},
+        "attn": {"flops": 4.0 * (K * K / 2.0) * dh * Hq,
+                 "bytes": (K * Hq * dh + 2 * K * Hkv * dh + K * Hq * dh) * 2 + K * 4},
+        "qkv": {"flops": 2.0 * K * d * (Hq + 2 * Hkv) * dh, "bytes": (K * d + d * (Hq + 2 * Hkv) * dh +
+                                                                   K * (Hq + 2 * Hkv) * dh) * 2},
+    }
+
+
+KERNEL_SOURCES = {
+    "gate": ["gate_score.cu"], "select": ["topk_select.cu"], "gather": ["gather_compact.cu"],
+    "rope": ["rope_apply.cu"], "attn": ["gated_attention.cu"],
+}
+
+
+def kernel_src_hash(stage):
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "learned_token_pruning_tg_b200", "csrc")
+    for f in KERNEL_SOURCES[stage] + ["tg_device.cuh"]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(stage):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        e = j.get(stage)
+        if e and e.get("src_sha") == kernel_src_hash(stage):
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, cuda_index, period=0.01):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            props = torch.cuda.get_device_properties(cuda_index)
+            dom, bus, dev = (getattr(props, k, None) for k in ("pci_domain_id", "pci_bus_id", "pci_device_id"))
+            if all(isinstance(x, int) for x in (dom, bus, dev)):
+                # NVML wants the bus id as a string "dddddddd:bb:dd.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{dev:02x}.0".encode())
+            else:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+                idx = int(vis.split(",")[cuda_index]) if vis else cuda_index
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = self._reasons_fn(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        reasons = sorted(r for r in self.reasons if r != "gpu_idle")
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- oracle (CPU) timing
+_ORACLE_CACHE = {}
+
+
+def oracle_sample(w, gi, ap, budget_s, seed=0):
+    """Time the single-threaded oracle on a bounded sample of one step and extrapolate the step time.
+
+    Sample: gate on n_g rows; select over the full document (scores drawn N(0, 1)); gather of the
+    full kept set; RoPE on n_r rows; attention on n_a query rows (all heads) spread evenly over the
+    kept set, scaled by the causal work they represent.  The QKV projection (glue) is not an oracle
+    step and is not timed."""
+    import numpy as np
+
+    import oracle
+
+    rng = np.random.default_rng(seed)
+    n_g = max(8, int(0.45 * budget_s / 4.6e-4))
+    n_a = max(1, int(0.35 * budget_s / 1.3e-2))
+    N, K, d_h, Hq, Hkv = w.N, w.K, w.d_h, w.Hq, w.Hkv
+    n_r = min(K, max(8, int(0.02 * budget_s / 6e-5)))
+    c = _ORACLE_CACHE.get(w.name)
+    if c is None:
+        g0 = np.random.default_rng(12345)
+        c = {"W1": gi.W1.float().numpy(), "w2": gi.w2.numpy(),
+             "h_bits": gi.h.view(torch.int16).numpy().view(np.uint16),
+             "scores": g0.standard_normal(N).astype(np.float32),
+             "q": g0.standard_normal((K, Hq, d_h)).astype(np.float32),
+             "k": g0.standard_normal((K, Hkv, d_h)).astype(np.float32),
+             "v": g0.standard_normal((K, Hkv, d_h)).astype(np.float32),
+             "x": g0.standard_normal((K, Hq + Hkv, d_h)).astype(np.float32)}
+        _ORACLE_CACHE[w.name] = c
+    rows_g = np.sort(rng.choice(N, size=min(n_g, N), replace=False))
+    hs = gi.h[torch.from_numpy(rows_g)].float().numpy()
+    t0 = time.perf_counter()
+    oracle.gate_score(hs, c["W1"], c["w2"])
+    t_gate = (time.perf_counter() - t0) * N / len(rows_g)
+    t0 = time.perf_counter()
+    kept = oracle.topk_select(c["scores"], w.doc_begin, w.doc_end, w.k_doc)
+    t_select = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.gather_compact(c["h_bits"], kept, scores=c["scores"])
+    t_gather = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.rope(c["x"][:n_r], kept[:n_r].astype(np.int32))
+    t_rope = (time.perf_counter() - t0) * K / n_r
+    rows_a = np.unique(np.linspace(0, K - 1, n_a).astype(np.int64))
+    t0 = time.perf_counter()
+    oracle.gated_attention(c["q"], c["k"], c["v"], s=c["scores"][:K], g=ap.gain.numpy(), tau=ap.tau, rows=rows_a)
+    t_attn = (time.perf_counter() - t0) * (K * (K + 1) / 2.0) / float(np.sum(rows_a + 1))
+    total = t_gate + t_select + t_gather + t_rope + t_attn
+    sample = (f"oracle, 1 thread: gate {len(rows_g)}/{N} rows, select and gather in full, rope {n_r}/{K} rows, "
+              f"attention {len(rows_a)}/{K} query rows x {Hq} heads (causal work-weighted); "
+              f"extrapolated to the full step; QKV glue not timed")
+    parts = {"gate_s": t_gate, "select_s": t_select, "gather_s": t_gather, "rope_s": t_rope, "attn_s": t_attn}
+    return total, sample, parts
+
+
+def pin_one_core():
+    try:
+        os.sched_setaffinity(0, {sorted(os.sched_getaffinity(0))[0]})
+        return 1
+    except Exception:
+        return 1
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args, rank, world):
+    w = WORKLOAD
+    if rank != 0:
+        return None
+    gi = synth.gate_inputs(w)
+    ap = synth.attn_params(w)
+    budget = min(15.0, 100.0 / max(1, args.steps + args.warmup))
+    cores = pin_one_core()
+    for _ in range(args.warmup):
+        oracle_sample(w, gi, ap, budget)
+    ts = []
+    for i in range(args.steps):
+        t, sample, _ = oracle_sample(w, gi, ap, budget, seed=i)
+        ts.append(t)
+    t_step = statistics.mean(ts)
+    value = w.N / t_step
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_dict(w),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_tokengate(args, rank, world, local_rank):
+    from learned_token_pruning_tg_b200 import tokengate as tg
+    from learned_token_pruning_tg_b200.path import STAGES, GatedPrefillLayer
+
+    if not os.path.exists(tg.LIB_PATH):
+        from learned_token_pruning_tg_b200 import build as tg_build
+        tg_build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOAD
+    gi = synth.gate_inputs(w, seed=w.seed + rank)
+    ap = synth.attn_params(w, seed=w.seed + rank)
+    Wqkv = torch.cat([ap.Wq, ap.Wk, ap.Wv], dim=0)
+    layer = GatedPrefillLayer(w.N, w.doc_begin, w.doc_end, w.k_doc, gi.W1, gi.w2, Wqkv, w.Hq, w.Hkv, w.d_h,
+                              ap.gain, ap.tau, eps=w.eps, rope_base=w.rope_base, device=dev)
+    h = gi.h.to(dev)
+    for _ in range(args.warmup):
+        layer.run(h)
+    torch.cuda.synchronize()
+    assert tg.tg_device_status(layer.ws) == 0, "device wait timed out during warm-up"
+
+    # per-stage CUDA events on the launching (current) stream
+    K = args.steps
+    marks = [[None] * (len(STAGES) + 1) for _ in range(K)]
+    ev_pool = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(K)]
+    names = list(STAGES) + ["end"]
+
+    def marker(i):
+        def m(name):
+            e = ev_pool[i][names.index(name)]
+            e.record()
+            marks[i][names.index(name)] = e
+        return m
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record()
+        for i in range(K):
+            layer.run(h, mark=marker(i))
+        end.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = start.elapsed_time(end)
+    ms_step = ms_total / K
+    stage_ms = {s: 0.0 for s in STAGES}
+    for i in range(K):
+        for j, s in enumerate(STAGES):
+            stage_ms[s] += marks[i][j].elapsed_time(marks[i][j + 1]) / K
+    status = tg.tg_device_status(layer.ws)
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_step = float(t.item())
+    value = w.N * world / (ms_step * 1e-3)
+
+    # end to end through the same API from pinned host memory: H2D of h, the path, D2H of out + kept
+    h_host = gi.h.pin_memory()
+    out_host = torch.empty(layer.out.shape, dtype=torch.bfloat16).pin_memory()
+    kept_host = torch.empty(layer.K, dtype=torch.int32).pin_memory()
+    h_dev = torch.empty_like(h)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        layer.run_host(h_host, h_dev, out_host, kept_host)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        layer.run_host(h_host, h_dev, out_host, kept_host)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": w.N * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h_host.numel() * h_host.element_size(),
+           "d2h_bytes_per_step": out_host.numel() * out_host.element_size() + kept_host.numel() * 4,
+           "ms_per_step": e2e_ms}
+
+    if rank != 0:
+        return None
+
+    # roofline of the dominant libtokengate kernel, and of the whole path
+    peaks = load_peaks()
+    work = stage_work(w)
+    ours = ["gate", "select", "gather", "rope", "attn"]
+    dom = max(ours, key=lambda s: stage_ms[s])
+    tensor_peak = peaks["bf16_tflops_sustained"]     # kernels timed inside a long back-to-back loop
+    t_flop = work[dom]["flops"] / (tensor_peak * 1e12)
+    t_byte = work[dom]["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    sec = stage_ms[dom] * 1e-3
+    if t_flop >= t_byte:
+        roof = {"bound": "tensor", "achieved": work[dom]["flops"] / sec / 1e12, "peak": tensor_peak,
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": work[dom]["bytes"] / sec / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = ncu_traffic(dom)
+    roof["kernel"] = dom
+    roof["algorithmic_per_launch"] = {"flops": work[dom]["flops"], "bytes": work[dom]["bytes"]}
+    roof["peak_source"] = peaks["source"] + (" (sustained bf16)" if roof["bound"] == "tensor" else " (HBM copy)")
+
+    def lower_bound(s, tpk):
+        return max(work[s]["flops"] / (tpk * 1e12), work[s]["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    path = ["gate", "select", "gather", "attn"]
+    t_path = sum(stage_ms[s] for s in path) * 1e-3
+    path_roof = sum(lower_bound(s, tensor_peak) for s in path) / t_path
+    path_roof_burst = sum(lower_bound(s, peaks["bf16_tflops"]) for s in path) / t_path
+    kernels = {}
+    for s in STAGES:
+        sec_s = stage_ms[s] * 1e-3
+        kernels[s] = {"us": stage_ms[s] * 1e3,
+                      "tflops": work[s]["flops"] / sec_s / 1e12 if work[s]["flops"] else None,
+                      "gbs": work[s]["bytes"] / sec_s / 1e9,
+                      "roofline_frac": lower_bound(s, tensor_peak) / sec_s}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cores = pin_one_core()
+        t, sample, parts = oracle_sample(w, gi, ap, args.cpu_budget)
+        cpu = {"value": w.N / t, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+               "extrapolated_s_per_step": t, "parts_s": parts}
+
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; stands in for NIAH-style 128k prompts)",
+            "config": config_dict(w), "impl": "tokengate",
+            "path_ms": t_path * 1e3, "path_tokens_per_s": w.N * world / t_path,
+            "path_roofline_frac": path_roof, "path_roofline_frac_burst_peak": path_roof_burst,
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": layer.launches_per_step() * K, "clocks": clk.summary(), "device_status": status,
+            "peaks": peaks}
+
+
+def main():
+    faulthandler.enable()
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["tokengate", "reference"], default="tokengate")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_tokengate(args, rank, world, local_rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,99 @@
+"""One TokenGate gate layer's prefill hot path, as a user calls it.
+
+Layers below the gate run over all N tokens; at the gate layer every token is
+scored, the best document tokens are kept (the question always is), the kept
+rows are compacted, and the attention of the next layer runs over the K kept
+tokens with the token-gated logit bias (TokenGate pages: aiproducthub.cn
+article, paragraph 事件详情; chathome.org article, sections TokenGate の学習可能な
+トークンプルーニングの仕組み and トークンゲート付きアテンションとは).
+
+Steps, in order, all on the caller's current CUDA stream:
+  gate     tg_gate_score        libtokengate (tcgen05 GEMM + fused epilogue)
+  select   tg_topk_select       libtokengate (radix select)
+  gather   tg_gather_compact    libtokengate (row copy)
+  qkv      h' Wqkv^T            torch.matmul (cuBLAS): projection glue
+  rope     tg_rope_apply        libtokengate
+  attn     tg_gated_attention   libtokengate (tcgen05 flash attention)
+torch allocates every buffer once (plumbing); the kept count K is known on the
+host, so nothing synchronizes inside a step.
+"""
+from __future__ import annotations
+
+from typing import Callable, Optional
+
+import torch
+
+from . import tokengate as tg
+
+STAGES = ("gate", "select", "gather", "qkv", "rope", "attn")
+
+
+class GatedPrefillLayer:
+    def __init__(self, N: int, doc_begin: int, doc_end: int, k_doc: int, W1: torch.Tensor, w2: torch.Tensor,
+                 Wqkv: torch.Tensor, Hq: int, Hkv: int, d_h: int, gain: torch.Tensor, tau: float,
+                 b1: Optional[torch.Tensor] = None, b2: float = 0.0, rms_weight: Optional[torch.Tensor] = None,
+                 eps: float = 1e-6, rope_base: float = 1e6, device="cuda"):
+        self.N, self.doc_begin, self.doc_end, self.k_doc = N, doc_begin, doc_end, k_doc
+        self.K = tg.tg_kept_count(N, doc_begin, doc_end, k_doc)
+        if self.K < 0:
+            raise ValueError("bad document span or budget")
+        dev = torch.device(device)
+        self.d_g, self.d = W1.shape
+        self.Hq, self.Hkv, self.d_h = Hq, Hkv, d_h
+        self.W1 = W1.to(dev, torch.bfloat16).contiguous()
+        self.w2 = w2.to(dev, torch.float32).contiguous()
+        self.b1 = None if b1 is None else b1.to(dev, torch.float32).contiguous()
+        self.b2 = float(b2)
+        self.rms_weight = None if rms_weight is None else rms_weight.to(dev, torch.bfloat16).contiguous()
+        self.eps, self.rope_base, self.tau = eps, rope_base, float(tau)
+        self.WqkvT = Wqkv.to(dev, torch.bfloat16).t().contiguous()      # [d, (Hq + 2 Hkv) d_h]
+        self.gain = gain.to(dev, torch.float32).contiguous()
+        K, d = self.K, self.d
+        self.ws = tg.new_workspace(N, d, self.d_g, device=dev)
+        self.scores = torch.empty(N, dtype=torch.float32, device=dev)
+        self.kept = torch.empty(max(K, 1), dtype=torch.int32, device=dev)
+        self.h_kept = torch.empty(K, d, dtype=torch.bfloat16, device=dev)
+        self.pos = torch.empty(max(K, 1), dtype=torch.int32, device=dev)
+        self.s_kept = torch.empty(max(K, 1), dtype=torch.float32, device=dev)
+        self.qkv = torch.empty(K, (Hq + 2 * Hkv) * d_h, dtype=torch.bfloat16, device=dev)
+        self.q = self.qkv[:, : Hq * d_h].view(K, Hq, d_h)
+        self.k = self.qkv[:, Hq * d_h: (Hq + Hkv) * d_h].view(K, Hkv, d_h)
+        self.v = self.qkv[:, (Hq + Hkv) * d_h:].view(K, Hkv, d_h)
+        self.out = torch.empty(K, Hq, d_h, dtype=torch.bfloat16, device=dev)
+
+    def run(self, h: torch.Tensor, mark: Optional[Callable[[str], None]] = None):
+        """Runs the six steps on device-resident h [N, d]; returns (out [K, Hq, d_h], kept [K]).
+        `mark(name)` is called before each step and with "end" after the last (event hooks)."""
+        m = mark or (lambda _n: None)
+        K = self.K
+        m("gate")
+        tg.tg_gate_score(h, self.W1, self.w2, self.scores, self.ws, b1=self.b1, b2=self.b2,
+                         rms_weight=self.rms_weight, eps=self.eps)
+        m("select")
+        tg.tg_topk_select(self.scores, self.doc_begin, self.doc_end, self.k_doc, self.kept[:K], self.ws)
+        m("gather")
+        tg.tg_gather_compact(h, self.kept[:K], self.h_kept, self.pos[:K], scores=self.scores,
+                             s_out=self.s_kept[:K])
+        m("qkv")
+        torch.matmul(self.h_kept, self.WqkvT, out=self.qkv)
+        m("rope")
+        tg.tg_rope_apply(self.q, self.k, self.pos[:K], self.rope_base)
+        m("attn")
+        tg.tg_gated_attention(self.q, self.k, self.v, self.out, self.ws, s_kept=self.s_kept[:K], gain=self.gain,
+                              tau=self.tau)
+        m("end")
+        return self.out, self.kept[:K]
+
+    def run_host(self, h_host: torch.Tensor, h_dev: torch.Tensor, out_host: torch.Tensor,
+                 kept_host: torch.Tensor):
+        """End to end from host memory: copies pinned h_host into h_dev, runs the layer, and copies
+        the attention output and kept indices back into pinned host tensors (all asynchronous)."""
+        h_dev.copy_(h_host, non_blocking=True)
+        out, kept = self.run(h_dev)
+        out_host.copy_(out, non_blocking=True)
+        kept_host.copy_(kept, non_blocking=True)
+        return out_host, kept_host
+
+    def launches_per_step(self) -> int:
+        """libtokengate kernels per run(): gate (+ the RMSNorm-weight fold), select, gather, rope, attention."""
+        return 5 + (1 if self.rms_weight is not None else 0)
