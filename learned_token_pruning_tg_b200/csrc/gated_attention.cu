@@ -9,23 +9,36 @@
 //   l_{r,c} = tau * (q_r . k_c) / sqrt(d_h) + g_h * s_c,   c <= r
 //   O_r = sum_c softmax_c(l_{r,.}) v_c
 //
-// Kernel (one CTA per (128-query tile, query head); heaviest tiles first):
-//   warp 0     TMA: the Q tile once, then K and V tiles (128 keys) into a
-//              2-stage ring (separate K and V barriers so S can start early)
-//   warp 1     TMEM allocation and the single MMA-issuing thread:
-//                S_j = Q K_j^T   (tcgen05 kind::f16, M=128, N=128, K=d_h)
-//                O  += P_j V_j   (A = P_j read from TMEM, B = V_j MN-major)
-//              S is double-buffered in TMEM so S_{j+1} overlaps softmax j
-//   warps 4-7  softmax, one query row per thread: tcgen05.ld of the S row,
-//              x = S * tau/sqrt(d_h) * log2(e) + g_h s_c log2(e) (bias added
-//              in registers from a per-tile shared-memory vector), causal mask
-//              on the diagonal tile only, online max with lazy rescaling (O is
-//              rescaled only when a row max grows by more than 2^8), P = 2^(x-m)
-//              written to TMEM as two bf16 halves P_hi + P_lo (P_lo = the
-//              rounding residual), so the P V product (two MMAs per step) sees P
-//              to ~16 significant bits: the output error no longer grows with
-//              the magnitude of v; at the end O / l to bf16 and the log-sum-exp.
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+d_h) P_hi, P_lo (64 each).
+// Kernel: one CTA per (128-query tile, NQ query heads of one GQA group), the
+// heaviest query tiles first.  NQ = 2 when the group size is even: the two
+// heads share every K/V tile and their softmax warpgroups ping-pong, so the
+// tensor core works on one head while the other head's softmax runs.
+//   warp 0      TMA: the NQ Q tiles once, then K and V tiles of 128 keys into
+//               two 2-stage rings (K runs one tile ahead of V)
+//   warp 1      TMEM allocation and the single MMA-issuing thread:
+//                 S_h = Q_h K_j^T   (kind::f16 bf16 x bf16 -> fp32, N = 128)
+//                 O_h += P_h V_j    (kind::f16 fp16 x fp16 -> fp32; P_h read
+//                                    from TMEM, V_j MN-major from smem)
+//   warps 2-3   convert each V tile to fp16 in place in shared memory (the
+//               swizzled layout is unchanged because both types are 2 bytes)
+//   warps 4+4h  softmax of head h, one query row per thread, two passes over
+//               the S row in TMEM: (1) x = S tau/sqrt(d_h) log2(e) + g_h s_c
+//               log2(e) and the row max; (2) P = 2^(x - m) written as fp16
+//               over the S columns already read.  The key bias comes from a
+//               per-tile shared vector whose scores are prefetched a tile
+//               ahead.  Lazy rescaling: O is rescaled (in TMEM) only when a
+//               row max grows by more than 2^8, so P <= 256.  Causal masking
+//               only on the diagonal tile.  At the end O / l to bf16 and the
+//               log-sum-exp.
+// P in fp16 (11 significant bits) rather than bf16 keeps the P V product's
+// relative error below 2^-11 per weight, which bounds the output error for
+// large-magnitude values; V is converted exactly (bf16 values in fp16's normal
+// range convert without rounding).
+//
+// Ordering: a tcgen05.commit arrives only when ALL earlier MMAs of the issuing
+// thread are complete, so "S_h(j) ready" also means P_h(j-1) V_{j-1} is done:
+// softmax may then rescale O_h and overwrite the S_h/P_h columns.
+// TMEM columns: S_h/P_h at 128 h, O_h at 128 NQ + d_h h.
 // Every wait is bounded (TG_STATUS_ATTENTION_TIMEOUT).
 #include <cmath>
 
@@ -34,34 +47,36 @@
 namespace tg {
 namespace attn {
 
-constexpr int kBM = 128;       // query rows per tile
-constexpr int kBN = 128;       // keys per tile
-constexpr int kStages = 2;     // K/V ring depth
-constexpr int kThreads = 256;  // 8 warps
+constexpr int kBM = 128;    // query rows per tile
+constexpr int kBN = 128;    // keys per tile
+constexpr int kStages = 2;  // depth of the K ring and of the V ring
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 
-template <int D>
+template <int D, int NQ>
 struct Cfg {
-    static constexpr int kTile = kBM * D * 2;  // bytes of one 128 x D bf16 tile
+    static constexpr int kTile = kBM * D * 2;  // bytes of one 128 x D 16-bit tile
     static constexpr int kChunks = D / 64;     // 64-column (128-byte) swizzle chunks per row
+    static constexpr int kThreads = 32 * (4 + 4 * NQ);
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTile;
+    static constexpr int kOffK = kOffQ + NQ * kTile;
     static constexpr int kOffV = kOffK + kStages * kTile;
-    static constexpr int kOffBias = kOffV + kStages * kTile;  // float [2][128]
-    static constexpr int kOffBar = kOffBias + 2 * kBN * 4;
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 3 + 2 + 1;
+    static constexpr int kOffBias = kOffV + kStages * kTile;  // float [NQ][2][128]
+    static constexpr int kOffBar = kOffBias + NQ * 2 * kBN * 4;
+    static constexpr int kNumBars = 1 + 5 * kStages + 5 * NQ + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmem = kOffMisc + 16 + 1024;
-    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColPhi = 256 + D, kColPlo = 256 + D + 64;
-    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kTmemCols = (NQ == 2) ? 512 : 256;
+    static __device__ __forceinline__ uint32_t col_s(int h) { return static_cast<uint32_t>(h * 128); }
+    static __device__ __forceinline__ uint32_t col_o(int h) { return static_cast<uint32_t>(NQ * 128 + h * D); }
 };
 
 struct Args {
     int64_t K;
     int Hq, Hkv;
     int num_q_tiles;
-    float scale_log2;  // tau / sqrt(d_h) * log2(e)
+    int pairs_per_group;  // (Hq / Hkv) / NQ
+    float scale_log2;     // tau / sqrt(d_h) * log2(e)
     const float* s_kept;
     const float* gain;
     __nv_bfloat16* out;
@@ -75,6 +90,45 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 up2(uint64_t u) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(u));
+    return r;
+}
+// Blackwell paired fp32 arithmetic: two lanes of work per issue slot.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pk2(a.x, a.y)), "l"(pk2(b.x, b.y)), "l"(pk2(c.x, c.y)));
+    return up2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk2(a.x, a.y)), "l"(pk2(b.x, b.y)));
+    return up2(d);
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// Instruction descriptor for kind::f16 with fp16 A and B, fp32 accumulator
+// (A/B format field 0 = f16; same layout as idesc_bf16_f32 otherwise).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major) {
+    return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Bounded wait whose result is the same on every lane of the warp, so that the
 // warp-collective tcgen05.ld/st and shuffles that follow never see a partial warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -83,34 +137,35 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int NQ>
+__global__ void __launch_bounds__(Cfg<D, NQ>::kThreads, 1)
 gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const Args a) {
-    using C = Cfg<D>;
+    using C = Cfg<D, NQ>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* bias_s = reinterpret_cast<float*>(smem + C::kOffBias);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* q_full = bars;                     // TMA -> MMA
-    uint64_t* k_full = bars + 1;                 // [kStages] TMA -> MMA
-    uint64_t* k_empty = k_full + kStages;        // [kStages] MMA commit after S_j -> TMA
-    uint64_t* v_full = k_empty + kStages;        // [kStages] TMA -> MMA
-    uint64_t* v_empty = v_full + kStages;        // [kStages] MMA commit after P_j V_j -> TMA
-    uint64_t* s_full = v_empty + kStages;        // [2] MMA commit -> softmax
-    uint64_t* s_empty = s_full + 2;              // [2] 128 softmax threads -> MMA
-    uint64_t* p_full = s_empty + 2;              // 128 softmax threads -> MMA (P_j written)
-    uint64_t* pv_done = p_full + 1;              // MMA commit after P_j V_j (completion j)
-    uint64_t* bias_full = pv_done + 1;           // [2] 128 softmax threads (key-bias vector written)
-    uint64_t* drain = bias_full + 2;             // abort path
+    uint64_t* q_full = bars;                      // TMA -> MMA
+    uint64_t* k_full = bars + 1;                  // [kStages] TMA -> MMA
+    uint64_t* k_empty = k_full + kStages;         // [kStages] commit after the last S of a K tile -> TMA
+    uint64_t* v_full = k_empty + kStages;         // [kStages] TMA -> converters
+    uint64_t* v_ready = v_full + kStages;         // [kStages] 64 converter threads -> MMA
+    uint64_t* v_empty = v_ready + kStages;        // [kStages] commit after the last P V of a V tile -> TMA
+    uint64_t* s_full = v_empty + kStages;         // [NQ] commit after S_h(j) -> softmax h
+    uint64_t* p_full = s_full + NQ;               // [NQ] 128 softmax threads of head h -> MMA
+    uint64_t* o_final = p_full + NQ;              // [NQ] commit after the last P V -> epilogue
+    uint64_t* bias_full = o_final + NQ;           // [NQ][2] 128 softmax threads (key-bias vector written)
+    uint64_t* drain = bias_full + 2 * NQ;         // abort path
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // heaviest (last) query tiles first
-    const int m_tile = a.num_q_tiles - 1 - static_cast<int>(blockIdx.x / a.Hq);
-    const int h = static_cast<int>(blockIdx.x % a.Hq);
-    const int kvh = h / (a.Hq / a.Hkv);
+    const int per_tile = a.Hkv * a.pairs_per_group;
+    const int m_tile = a.num_q_tiles - 1 - static_cast<int>(blockIdx.x / per_tile);  // heaviest first
+    const int rem = static_cast<int>(blockIdx.x % per_tile);
+    const int kvh = rem / a.pairs_per_group;
+    const int head0 = kvh * (a.Hq / a.Hkv) + (rem % a.pairs_per_group) * NQ;
     const int n_kv = m_tile + 1;  // causal: kv tiles 0..m_tile, the last one on the diagonal
 
     if (threadIdx.x == 0) {
@@ -119,15 +174,16 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1);
+            mbar_init(&v_ready[s], 64);
             mbar_init(&v_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&s_full[b], 1);
-            mbar_init(&s_empty[b], 128);
-            mbar_init(&bias_full[b], 128);
+        for (int h = 0; h < NQ; ++h) {
+            mbar_init(&s_full[h], 1);
+            mbar_init(&p_full[h], 128);
+            mbar_init(&o_final[h], 1);
+            mbar_init(&bias_full[2 * h], 128);
+            mbar_init(&bias_full[2 * h + 1], 128);
         }
-        mbar_init(p_full, 128);
-        mbar_init(pv_done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -149,42 +205,31 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         if (lane == 0) {
             int k_last[kStages], v_last[kStages];  // parity of the last phase loaded per stage, -1 if none
             for (int i = 0; i < kStages; ++i) k_last[i] = v_last[i] = -1;
-            mbar_arrive_expect_tx(q_full, C::kTile);
-#pragma unroll
-            for (int c = 0; c < C::kChunks; ++c)
-                tma_load_3d(smem + C::kOffQ + c * (kBM * 128), &tmap_q, q_full, c * 64, h, m_tile * kBM,
-                            kEvictFirst);
-            auto load_k = [&](int j) -> bool {
-                const int st = j % kStages;
-                const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
-                if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT))
-                    return false;
-                uint8_t* dst = smem + C::kOffK + st * C::kTile;
-                mbar_arrive_expect_tx(&k_full[st], C::kTile);
+            mbar_arrive_expect_tx(q_full, NQ * C::kTile);
+            for (int h = 0; h < NQ; ++h)
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(dst + c * (kBN * 128), &tmap_k, &k_full[st], c * 64, kvh, j * kBN, kEvictLast);
-                k_last[st] = static_cast<int>(ph);
-                return true;
-            };
-            auto load_v = [&](int j) -> bool {
+                    tma_load_3d(smem + C::kOffQ + h * C::kTile + c * (kBM * 128), &tmap_q, q_full, c * 64,
+                                head0 + h, m_tile * kBM, kEvictFirst);
+            auto load = [&](int j, uint64_t* empty, uint64_t* full, int off, const CUtensorMap* map,
+                            int* last) -> bool {
                 const int st = j % kStages;
                 const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
-                if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT))
+                if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT))
                     return false;
-                uint8_t* dst = smem + C::kOffV + st * C::kTile;
-                mbar_arrive_expect_tx(&v_full[st], C::kTile);
+                uint8_t* dst = smem + off + st * C::kTile;
+                mbar_arrive_expect_tx(&full[st], C::kTile);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(dst + c * (kBN * 128), &tmap_v, &v_full[st], c * 64, kvh, j * kBN, kEvictLast);
-                v_last[st] = static_cast<int>(ph);
+                    tma_load_3d(dst + c * (kBN * 128), map, &full[st], c * 64, kvh, j * kBN, kEvictLast);
+                last[st] = static_cast<int>(ph);
                 return true;
             };
-            // K runs one tile ahead of V: S_{j+1} only needs K_{j+1}, P_j V_j comes after softmax j.
-            bool ok = load_k(0);
+            // K runs one tile ahead of V: S(j+1) needs only K(j+1); P(j) V(j) waits for softmax j anyway.
+            bool ok = load(0, k_empty, k_full, C::kOffK, &tmap_k, k_last);
             for (int j = 0; j < n_kv && ok; ++j) {
-                if (j + 1 < n_kv) ok = load_k(j + 1);
-                if (ok) ok = load_v(j);
+                if (j + 1 < n_kv) ok = load(j + 1, k_empty, k_full, C::kOffK, &tmap_k, k_last);
+                if (ok) ok = load(j, v_empty, v_full, C::kOffV, &tmap_v, v_last);
             }
             // Every issued copy must land before shared memory is released (matters on abort only).
             volatile int no_abort = 0;
@@ -202,108 +247,142 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false);  // Q K^T: both K-major
-            constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, true);     // P V: B (= V) MN-major
-            const uint32_t q_addr = smem_u32(smem + C::kOffQ);
+            constexpr uint32_t idesc_o = idesc_f16_f32(kBM, D, true);      // P V: V MN-major
             bool ok = mbar_wait(q_full, 0, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
-            tc_fence_after();
-            // S_j = Q K_j^T into S buffer j % 2; the K stage is released when these MMAs finish
-            auto issue_s = [&](int j) -> bool {
-                const int st = j % kStages;
-                const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
-                const int b = j & 1;
-                if (!mbar_wait(&k_full[st], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT)) return false;
-                if (!mbar_wait(&s_empty[b], (static_cast<uint32_t>(j >> 1) & 1) ^ 1, abort_flag, a.status,
-                               TG_STATUS_ATTENTION_TIMEOUT))
-                    return false;
-                tc_fence_after();
-                const uint32_t k_addr = smem_u32(smem + C::kOffK + st * C::kTile);
-                const uint32_t d_tmem = tmem + (b ? C::kColS1 : C::kColS0);
+            auto wait_k = [&](int j) -> bool {
+                return mbar_wait(&k_full[j % kStages], static_cast<uint32_t>(j / kStages) & 1, abort_flag,
+                                 a.status, TG_STATUS_ATTENTION_TIMEOUT);
+            };
+            // S_h = Q_h K_j^T, then signal softmax h (the commit also covers every earlier MMA)
+            auto issue_s = [&](int h, int j) {
+                const uint32_t q_addr = smem_u32(smem + C::kOffQ + h * C::kTile);
+                const uint32_t k_addr = smem_u32(smem + C::kOffK + (j % kStages) * C::kTile);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = static_cast<uint32_t>((k >> 2) * (kBM * 128) + (k & 3) * 32);
-                    mma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024),
+                    mma_ss(tmem + C::col_s(h), smem_desc_sw128(q_addr + off, 16, 1024),
                            smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, k > 0);
                 }
-                mma_commit(&s_full[b]);
-                mma_commit(&k_empty[st]);
-                return true;
+                mma_commit(&s_full[h]);
             };
-            if (ok) ok = issue_s(0);
+            if (ok) ok = wait_k(0);
+            if (ok) {
+                tc_fence_after();
+                for (int h = 0; h < NQ; ++h) issue_s(h, 0);
+                mma_commit(&k_empty[0]);
+            }
             for (int j = 0; j < n_kv && ok; ++j) {
-                if (j + 1 < n_kv && !(ok = issue_s(j + 1))) break;
                 const int st = j % kStages;
-                const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
-                const int b = j & 1;
-                (void)b;
-                if (!(ok = mbar_wait(p_full, static_cast<uint32_t>(j) & 1, abort_flag, a.status,
+                const bool next = j + 1 < n_kv;
+                if (!(ok = mbar_wait(&v_ready[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
                                      TG_STATUS_ATTENTION_TIMEOUT)))
                     break;
-                if (!(ok = mbar_wait(&v_full[st], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT))) break;
-                tc_fence_after();
                 const uint32_t v_addr = smem_u32(smem + C::kOffV + st * C::kTile);
+                for (int h = 0; h < NQ && ok; ++h) {
+                    if (!(ok = mbar_wait(&p_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status,
+                                         TG_STATUS_ATTENTION_TIMEOUT)))
+                        break;
+                    tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < kBN / 16; ++k) {  // 16 keys per step: 16 rows of 128 bytes in each chunk
-                    const uint64_t vd =
-                        smem_desc_sw128(v_addr + static_cast<uint32_t>(k * 2048), kBN * 128, 1024);
-                    // P = P_hi + P_lo: two bf16 products keep P at ~16 significant bits
-                    mma_ts(tmem + C::kColO, tmem + C::kColPhi + static_cast<uint32_t>(k * 8), vd, idesc_o,
-                           (j > 0 || k > 0) ? 1u : 0u);
-                    mma_ts(tmem + C::kColO, tmem + C::kColPlo + static_cast<uint32_t>(k * 8), vd, idesc_o, 1u);
+                    for (int k = 0; k < kBN / 16; ++k)  // 16 keys per step: 16 rows of 128 bytes in each chunk
+                        mma_ts(tmem + C::col_o(h), tmem + C::col_s(h) + static_cast<uint32_t>(k * 8),
+                               smem_desc_sw128(v_addr + static_cast<uint32_t>(k * 2048), kBN * 128, 1024),
+                               idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+                    if (next) {
+                        if (h == 0 && !(ok = wait_k(j + 1))) break;
+                        tc_fence_after();
+                        issue_s(h, j + 1);  // overwrites S_h/P_h after the P V above (MMAs run in order)
+                    }
                 }
+                if (!ok) break;
                 mma_commit(&v_empty[st]);
-                mma_commit(pv_done);
+                if (next) mma_commit(&k_empty[(j + 1) % kStages]);
             }
-            if (!ok) {
+            if (ok) {
+                for (int h = 0; h < NQ; ++h) mma_commit(&o_final[h]);
+            } else {
                 mma_commit(drain);
                 volatile int no_abort = 0;
                 mbar_wait(drain, 0, &no_abort, a.status, TG_STATUS_ATTENTION_TIMEOUT);
             }
         }
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------ softmax + epilogue
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ V tile -> fp16, in place
+        const int t = threadIdx.x - 64;
+        for (int j = 0; j < n_kv; ++j) {
+            const int st = j % kStages;
+            if (!mbar_wait(&v_full[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
+                           TG_STATUS_ATTENTION_TIMEOUT))
+                break;
+            uint4* vt = reinterpret_cast<uint4*>(smem + C::kOffV + st * C::kTile);
+#pragma unroll 4
+            for (int i = t; i < C::kTile / 16; i += 64) {
+                uint4 x = vt[i];
+                uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    w[e] = f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+                vt[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();  // generic-proxy writes -> tensor-core (async proxy) reads
+            mbar_arrive(&v_ready[st]);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue of head h
+        const int h = (warp - 4) >> 2;
         const int q = warp & 3;
         const int row = q * 32 + lane;  // query row inside the tile == TMEM lane
-        const int tid = threadIdx.x - 128;
+        const int t = threadIdx.x - 128 - 128 * h;
+        const int head = head0 + h;
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-        const float gain = a.gain ? a.gain[h] * kLog2e : 0.0f;
+        const uint32_t s_addr = tmem + lane_off + C::col_s(h);
+        const uint32_t o_addr = tmem + lane_off + C::col_o(h);
+        const float gain = a.gain ? a.gain[head] * kLog2e : 0.0f;
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+        float* bias_h = bias_s + h * 2 * kBN;
+        float s_pref = (a.s_kept && t < a.K) ? a.s_kept[t] : 0.0f;
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < n_kv && ok; ++j) {
             const int b = j & 1;
-            const uint32_t par = static_cast<uint32_t>(j >> 1) & 1;
-            // this tile's key bias g_h * s_c, in log2 units (one key per thread)
+            // this tile's key bias g_h * s_c in log2 units (one key per thread), next tile's score prefetched
+            bias_h[b * kBN + t] = gain * s_pref;
+            mbar_arrive(&bias_full[2 * h + b]);
             {
-                const int64_t c = static_cast<int64_t>(j) * kBN + tid;
-                bias_s[b * kBN + tid] = (a.s_kept && c < a.K) ? gain * a.s_kept[c] : 0.0f;
-                mbar_arrive(&bias_full[b]);
+                const int64_t cn = static_cast<int64_t>(j + 1) * kBN + t;
+                s_pref = (a.s_kept && j + 1 < n_kv && cn < a.K) ? a.s_kept[cn] : 0.0f;
             }
-            if (!(ok = warp_wait(&bias_full[b], par, abort_flag, a.status))) break;
-            if (!(ok = warp_wait(&s_full[b], par, abort_flag, a.status))) break;
+            if (!(ok = warp_wait(&bias_full[2 * h + b], static_cast<uint32_t>(j >> 1) & 1, abort_flag, a.status)))
+                break;
+            if (!(ok = warp_wait(&s_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status))) break;
             tc_fence_after();
-            float x[kBN];
-            {
-                const uint32_t sa = tmem + lane_off + (b ? C::kColS1 : C::kColS0);
-#pragma unroll
-                for (int c0 = 0; c0 < kBN; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(sa + c0, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) x[c0 + i] = __uint_as_float(v[i]);
-                }
-                tmem_ld_wait();
-            }
-            tc_fence_before();
-            mbar_arrive(&s_empty[b]);
-
-            const float* bias = bias_s + b * kBN;
+            const float* bias = bias_h + b * kBN;
             const bool diag = (j == n_kv - 1);
+
+            // pass 1: row max of x = S * scale + bias
             float mx = -INFINITY;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kBN; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(s_addr + c0, v);
+                tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) {
-                float v = fmaf(x[c], a.scale_log2, bias[c]);
-                if (diag && c > row) v = -INFINITY;
-                x[c] = v;
-                mx = fmaxf(mx, v);
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 bb = *reinterpret_cast<const float4*>(bias + c0 + i);
+                    float2 x0 = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), sc2,
+                                      make_float2(bb.x, bb.y));
+                    float2 x1 = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), sc2,
+                                      make_float2(bb.z, bb.w));
+                    if (diag) {
+                        const int c = c0 + i;
+                        if (c > row) x0.x = -INFINITY;
+                        if (c + 1 > row) x0.y = -INFINITY;
+                        if (c + 2 > row) x1.x = -INFINITY;
+                        if (c + 3 > row) x1.y = -INFINITY;
+                    }
+                    mx = fmax3(mx, x0.x, x0.y);
+                    mx = fmax3(mx, x1.x, x1.y);
+                }
             }
             // lazy rescaling: keep the stale max unless this row's max grew by more than 2^8
             const bool need = mx > m_run + kRescaleThreshold;
@@ -313,74 +392,81 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 m_run = mx;
                 l_run *= alpha;
             }
-            // P_{j-1} V_{j-1} must be complete before O is rescaled and before P is overwritten
-            if (j > 0) {
-                if (!(ok = warp_wait(pv_done, static_cast<uint32_t>(j - 1) & 1, abort_flag, a.status))) break;
-                tc_fence_after();
-            }
             if (j > 0 && __any_sync(0xffffffffu, need)) {
-                const uint32_t oa = tmem + lane_off + C::kColO;
+                // O_h holds exactly P(j-1) V(j-1) and earlier here (see the ordering note above)
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 16) {
                     uint32_t v[16];
-                    tmem_ld16(oa + c0, v);
+                    tmem_ld16(o_addr + c0, v);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                    tmem_st16(oa + c0, v);
+                    tmem_st16(o_addr + c0, v);
                 }
             }
-            float lsum = 0.0f;
-            const uint32_t pa_hi = tmem + lane_off + C::kColPhi;
-            const uint32_t pa_lo = tmem + lane_off + C::kColPlo;
-#pragma unroll
+            // pass 2: P = 2^(x - m) as fp16, written over the S columns already consumed
+            const float2 neg_m = make_float2(-m_run, -m_run);
+            float2 lsum = make_float2(0.0f, 0.0f);
+#pragma unroll 1
             for (int c0 = 0; c0 < kBN; c0 += 32) {
-                uint32_t hi[16], lo[16];
+                uint32_t v[32];
+                tmem_ld32(s_addr + c0, v);
+                tmem_ld_wait();
+                uint32_t p16[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = ex2(x[c0 + 2 * i] - m_run);
-                    const float p1 = ex2(x[c0 + 2 * i + 1] - m_run);
-                    lsum += p0 + p1;
-                    hi[i] = pack_bf16x2(p0, p1);
-                    lo[i] = pack_bf16x2(p0 - __uint_as_float(hi[i] << 16), p1 - __uint_as_float(hi[i] & 0xffff0000u));
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 bb = *reinterpret_cast<const float4*>(bias + c0 + i);
+                    float2 x0 = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), sc2,
+                                      make_float2(bb.x, bb.y));
+                    float2 x1 = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), sc2,
+                                      make_float2(bb.z, bb.w));
+                    if (diag) {
+                        const int c = c0 + i;
+                        if (c > row) x0.x = -INFINITY;
+                        if (c + 1 > row) x0.y = -INFINITY;
+                        if (c + 2 > row) x1.x = -INFINITY;
+                        if (c + 3 > row) x1.y = -INFINITY;
+                    }
+                    x0 = fadd2(x0, neg_m);
+                    x1 = fadd2(x1, neg_m);
+                    const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+                    const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+                    lsum = fadd2(lsum, p0);
+                    lsum = fadd2(lsum, p1);
+                    p16[i / 2] = f16x2(p0.x, p0.y);
+                    p16[i / 2 + 1] = f16x2(p1.x, p1.y);
                 }
-                tmem_st16(pa_hi + (c0 >> 1), hi);
-                tmem_st16(pa_lo + (c0 >> 1), lo);
+                tmem_st16(s_addr + (c0 >> 1), p16);
             }
             tmem_st_wait();
-            l_run += lsum;
+            l_run += lsum.x + lsum.y;
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[h]);
         }
-        if (ok) {
-            // epilogue: wait for the last P V, normalise, store bf16 rows and the log-sum-exp
-            const int jl = n_kv - 1;
-            if (warp_wait(pv_done, static_cast<uint32_t>(jl) & 1, abort_flag, a.status)) {
-                tc_fence_after();
-                const int64_t grow = static_cast<int64_t>(m_tile) * kBM + row;
-                const float inv_l = 1.0f / l_run;
-                __nv_bfloat16* orow = a.out + (grow * a.Hq + h) * D;
-                const uint32_t oa = tmem + lane_off + C::kColO;
+        if (ok && warp_wait(&o_final[h], 0, abort_flag, a.status)) {
+            // epilogue: normalise, store bf16 rows and the log-sum-exp
+            tc_fence_after();
+            const int64_t grow = static_cast<int64_t>(m_tile) * kBM + row;
+            const float inv_l = 1.0f / l_run;
+            __nv_bfloat16* orow = a.out + (grow * a.Hq + head) * D;
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(oa + c0, v);
-                    tmem_ld_wait();
-                    if (grow < a.K) {
-                        uint32_t o[16];
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(o_addr + c0, v);
+                tmem_ld_wait();
+                if (grow < a.K) {
+                    uint32_t o[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            o[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
-                                               __uint_as_float(v[2 * i + 1]) * inv_l);
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                    for (int i = 0; i < 16; ++i)
+                        o[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-                    }
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
                 }
-                if (a.lse && grow < a.K)
-                    a.lse[static_cast<int64_t>(h) * a.K + grow] = (m_run + log2f(l_run)) / kLog2e;
             }
+            if (a.lse && grow < a.K)
+                a.lse[static_cast<int64_t>(head) * a.K + grow] = (m_run + log2f(l_run)) / kLog2e;
         }
     }
 
@@ -392,16 +478,17 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     }
 }
 
-template <int D>
-static tg_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Args& a,
+template <int D, int NQ>
+static tg_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, Args a,
                         cudaStream_t st) {
-    using C = Cfg<D>;
-    auto kern = gated_attention_kernel<D>;
+    using C = Cfg<D, NQ>;
+    auto kern = gated_attention_kernel<D, NQ>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess)
         return TG_ERR_CUDA;
-    const int64_t grid = static_cast<int64_t>(a.num_q_tiles) * a.Hq;
+    a.pairs_per_group = (a.Hq / a.Hkv) / NQ;
+    const int64_t grid = static_cast<int64_t>(a.num_q_tiles) * a.Hkv * a.pairs_per_group;
     if (grid > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
-    kern<<<static_cast<unsigned>(grid), kThreads, C::kSmem, st>>>(mq, mk, mv, a);
+    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, st>>>(mq, mk, mv, a);
     return launch_status();
 }
 
@@ -445,6 +532,7 @@ extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg
     a.Hq = Hq;
     a.Hkv = Hkv;
     a.num_q_tiles = static_cast<int>((K + attn::kBM - 1) / attn::kBM);
+    a.pairs_per_group = 1;
     a.scale_log2 = tau / std::sqrt(static_cast<float>(d_h)) * attn::kLog2e;
     a.s_kept = s_kept;
     a.gain = gain;
@@ -452,5 +540,7 @@ extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg
     a.lse = lse;
     a.status = status_word(workspace);
     cudaStream_t st = as_stream(stream);
-    return d_h == 128 ? attn::launch<128>(mq, mk, mv, a, st) : attn::launch<64>(mq, mk, mv, a, st);
+    const bool pairs = ((Hq / Hkv) % 2) == 0;
+    if (d_h == 128) return pairs ? attn::launch<128, 2>(mq, mk, mv, a, st) : attn::launch<128, 1>(mq, mk, mv, a, st);
+    return pairs ? attn::launch<64, 2>(mq, mk, mv, a, st) : attn::launch<64, 1>(mq, mk, mv, a, st);
 }
