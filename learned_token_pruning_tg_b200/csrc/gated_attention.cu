@@ -11,35 +11,33 @@
 //
 // Kernel: one CTA per (128-query tile, NQ query heads of one GQA group), the
 // heaviest query tiles first.  NQ = 2 when the group size is even: the two
-// heads share every K/V tile and their softmax warpgroups ping-pong, so the
-// tensor core works on one head while the other head's softmax runs.
-//   warp 0      TMA: the NQ Q tiles once, then K and V tiles of 128 keys into
-//               two 2-stage rings (K runs one tile ahead of V)
+// heads share every K/V tile and their softmax warpgroups run side by side.
+//   warp 0      TMA: the NQ Q tiles once, then K and V tiles of 64 keys into
+//               two 4-stage rings (K runs one tile ahead of V)
 //   warp 1      TMEM allocation and the single MMA-issuing thread:
-//                 S_h = Q_h K_j^T   (kind::f16 bf16 x bf16 -> fp32, N = 128)
+//                 S_h = Q_h K_j^T   (kind::f16 bf16 x bf16 -> fp32, N = 64)
 //                 O_h += P_h V_j    (kind::f16 fp16 x fp16 -> fp32; P_h read
 //                                    from TMEM, V_j MN-major from smem)
+//               S_h(j+1) is issued as soon as softmax h has read S_h(j), so it
+//               runs while softmax h computes P_h(j): the MMA latency stays off
+//               the softmax's critical path.
 //   warps 2-3   convert each V tile to fp16 in place in shared memory (the
 //               swizzled layout is unchanged because both types are 2 bytes)
-//   warps 4+4h  softmax of head h, one query row per thread, two passes over
-//               the S row in TMEM: (1) x = S tau/sqrt(d_h) log2(e) + g_h s_c
-//               log2(e) and the row max; (2) P = 2^(x - m) written as fp16
-//               over the S columns already read.  The key bias comes from a
-//               per-tile shared vector whose scores are prefetched a tile
-//               ahead.  Lazy rescaling: O is rescaled (in TMEM) only when a
-//               row max grows by more than 2^8, so P <= 256.  Causal masking
-//               only on the diagonal tile.  At the end O / l to bf16 and the
-//               log-sum-exp.
+//   warps 4+4h  softmax of head h, one query row per thread: the 64 S values of
+//               the row are read from TMEM once into registers, x = S tau /
+//               sqrt(d_h) log2(e) + g_h s_c log2(e) (key bias from a per-tile
+//               shared vector whose scores are prefetched a tile ahead), row
+//               max, P = 2^(x - m) as fp16 into TMEM.  Lazy rescaling: O is
+//               rescaled (in TMEM) only when a row max grows by more than 2^8,
+//               so P <= 256.  Causal masking only on the diagonal tiles.  At
+//               the end O / l to bf16 and the log-sum-exp.
 // P in fp16 (11 significant bits) rather than bf16 keeps the P V product's
 // relative error below 2^-11 per weight, which bounds the output error for
 // large-magnitude values; V is converted exactly (bf16 values in fp16's normal
 // range convert without rounding).
 //
-// Ordering: a tcgen05.commit arrives only when ALL earlier MMAs of the issuing
-// thread are complete, so "S_h(j) ready" also means P_h(j-1) V_{j-1} is done:
-// softmax may then rescale O_h and overwrite the S_h/P_h columns.
-// TMEM columns: S_h/P_h at 128 h, O_h at 128 NQ + d_h h.
-// Every wait is bounded (TG_STATUS_ATTENTION_TIMEOUT).
+// TMEM columns: S_h at 64 h, P_h at 128 + 32 h, O_h at 256 + d_h h (512 in all
+// for two heads of 128).  Every wait is bounded (TG_STATUS_ATTENTION_TIMEOUT).
 #include <cmath>
 
 #include "tg_host.cuh"
@@ -48,27 +46,31 @@ namespace tg {
 namespace attn {
 
 constexpr int kBM = 128;    // query rows per tile
-constexpr int kBN = 128;    // keys per tile
-constexpr int kStages = 2;  // depth of the K ring and of the V ring
+constexpr int kBN = 64;     // keys per tile
+constexpr int kStages = 4;  // depth of the K ring and of the V ring
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 
 template <int D, int NQ>
 struct Cfg {
-    static constexpr int kTile = kBM * D * 2;  // bytes of one 128 x D 16-bit tile
-    static constexpr int kChunks = D / 64;     // 64-column (128-byte) swizzle chunks per row
+    static constexpr int kQTile = kBM * D * 2;   // bytes of a 128 x D 16-bit tile
+    static constexpr int kKVTile = kBN * D * 2;  // bytes of a 64 x D 16-bit tile
+    static constexpr int kChunks = D / 64;       // 64-column (128-byte) swizzle chunks per row
     static constexpr int kThreads = 32 * (4 + 4 * NQ);
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + NQ * kTile;
-    static constexpr int kOffV = kOffK + kStages * kTile;
-    static constexpr int kOffBias = kOffV + kStages * kTile;  // float [NQ][2][128]
+    static constexpr int kOffK = kOffQ + NQ * kQTile;
+    static constexpr int kOffV = kOffK + kStages * kKVTile;
+    static constexpr int kOffBias = kOffV + kStages * kKVTile;  // float [NQ][2][64]
     static constexpr int kOffBar = kOffBias + NQ * 2 * kBN * 4;
-    static constexpr int kNumBars = 1 + 5 * kStages + 5 * NQ + 1;
+    static constexpr int kNumBars = 1 + 5 * kStages + 6 * NQ + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmem = kOffMisc + 16 + 1024;
     static constexpr uint32_t kTmemCols = (NQ == 2) ? 512 : 256;
-    static __device__ __forceinline__ uint32_t col_s(int h) { return static_cast<uint32_t>(h * 128); }
-    static __device__ __forceinline__ uint32_t col_o(int h) { return static_cast<uint32_t>(NQ * 128 + h * D); }
+    static __device__ __forceinline__ uint32_t col_s(int h) { return static_cast<uint32_t>(h * kBN); }
+    static __device__ __forceinline__ uint32_t col_p(int h) { return static_cast<uint32_t>(NQ * kBN + h * (kBN / 2)); }
+    static __device__ __forceinline__ uint32_t col_o(int h) {
+        return static_cast<uint32_t>((NQ == 2 ? 256 : 128) + h * D);
+    }
 };
 
 struct Args {
@@ -153,9 +155,10 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     uint64_t* v_ready = v_full + kStages;         // [kStages] 64 converter threads -> MMA
     uint64_t* v_empty = v_ready + kStages;        // [kStages] commit after the last P V of a V tile -> TMA
     uint64_t* s_full = v_empty + kStages;         // [NQ] commit after S_h(j) -> softmax h
-    uint64_t* p_full = s_full + NQ;               // [NQ] 128 softmax threads of head h -> MMA
-    uint64_t* o_final = p_full + NQ;              // [NQ] commit after the last P V -> epilogue
-    uint64_t* bias_full = o_final + NQ;           // [NQ][2] 128 softmax threads (key-bias vector written)
+    uint64_t* s_empty = s_full + NQ;              // [NQ] 128 softmax threads read S_h(j) -> MMA
+    uint64_t* p_full = s_empty + NQ;              // [NQ] 128 softmax threads wrote P_h(j) -> MMA
+    uint64_t* pv_done = p_full + NQ;              // [NQ] commit after P_h(j) V_j -> softmax h, epilogue
+    uint64_t* bias_full = pv_done + NQ;           // [NQ][2] 128 softmax threads (key-bias vector written)
     uint64_t* drain = bias_full + 2 * NQ;         // abort path
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -166,7 +169,9 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     const int rem = static_cast<int>(blockIdx.x % per_tile);
     const int kvh = rem / a.pairs_per_group;
     const int head0 = kvh * (a.Hq / a.Hkv) + (rem % a.pairs_per_group) * NQ;
-    const int n_kv = m_tile + 1;  // causal: kv tiles 0..m_tile, the last one on the diagonal
+    // causal: key tiles 0..n_kv-1; the last kBM / kBN of them touch the diagonal
+    const int n_kv = static_cast<int>((static_cast<int64_t>(m_tile + 1) * kBM + kBN - 1) / kBN);
+    const int first_diag = (m_tile * kBM) / kBN;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -179,8 +184,9 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         }
         for (int h = 0; h < NQ; ++h) {
             mbar_init(&s_full[h], 1);
+            mbar_init(&s_empty[h], 128);
             mbar_init(&p_full[h], 128);
-            mbar_init(&o_final[h], 1);
+            mbar_init(&pv_done[h], 1);
             mbar_init(&bias_full[2 * h], 128);
             mbar_init(&bias_full[2 * h + 1], 128);
         }
@@ -205,11 +211,11 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         if (lane == 0) {
             int k_last[kStages], v_last[kStages];  // parity of the last phase loaded per stage, -1 if none
             for (int i = 0; i < kStages; ++i) k_last[i] = v_last[i] = -1;
-            mbar_arrive_expect_tx(q_full, NQ * C::kTile);
+            mbar_arrive_expect_tx(q_full, NQ * C::kQTile);
             for (int h = 0; h < NQ; ++h)
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(smem + C::kOffQ + h * C::kTile + c * (kBM * 128), &tmap_q, q_full, c * 64,
+                    tma_load_3d(smem + C::kOffQ + h * C::kQTile + c * (kBM * 128), &tmap_q, q_full, c * 64,
                                 head0 + h, m_tile * kBM, kEvictFirst);
             auto load = [&](int j, uint64_t* empty, uint64_t* full, int off, const CUtensorMap* map,
                             int* last) -> bool {
@@ -217,8 +223,8 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
                 if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT))
                     return false;
-                uint8_t* dst = smem + off + st * C::kTile;
-                mbar_arrive_expect_tx(&full[st], C::kTile);
+                uint8_t* dst = smem + off + st * C::kKVTile;
+                mbar_arrive_expect_tx(&full[st], C::kKVTile);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d(dst + c * (kBN * 128), map, &full[st], c * 64, kvh, j * kBN, kEvictLast);
@@ -253,15 +259,17 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 return mbar_wait(&k_full[j % kStages], static_cast<uint32_t>(j / kStages) & 1, abort_flag,
                                  a.status, TG_STATUS_ATTENTION_TIMEOUT);
             };
-            // S_h = Q_h K_j^T, then signal softmax h (the commit also covers every earlier MMA)
+            // S_h = Q_h K_j^T into head h's S columns, then signal softmax h
             auto issue_s = [&](int h, int j) {
-                const uint32_t q_addr = smem_u32(smem + C::kOffQ + h * C::kTile);
-                const uint32_t k_addr = smem_u32(smem + C::kOffK + (j % kStages) * C::kTile);
+                const uint32_t q_addr = smem_u32(smem + C::kOffQ + h * C::kQTile);
+                const uint32_t k_addr = smem_u32(smem + C::kOffK + (j % kStages) * C::kKVTile);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t off = static_cast<uint32_t>((k >> 2) * (kBM * 128) + (k & 3) * 32);
-                    mma_ss(tmem + C::col_s(h), smem_desc_sw128(q_addr + off, 16, 1024),
-                           smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, k > 0);
+                    const uint32_t koff = static_cast<uint32_t>((k & 3) * 32);
+                    mma_ss(tmem + C::col_s(h),
+                           smem_desc_sw128(q_addr + static_cast<uint32_t>((k >> 2) * (kBM * 128)) + koff, 16, 1024),
+                           smem_desc_sw128(k_addr + static_cast<uint32_t>((k >> 2) * (kBN * 128)) + koff, 16, 1024),
+                           idesc_s, k > 0);
                 }
                 mma_commit(&s_full[h]);
             };
@@ -273,11 +281,24 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             }
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int st = j % kStages;
-                const bool next = j + 1 < n_kv;
+                // next S of each head as soon as its softmax has read the current one
+                if (j + 1 < n_kv) {
+                    if (!(ok = wait_k(j + 1))) break;
+                    for (int h = 0; h < NQ && ok; ++h) {
+                        if (!(ok = mbar_wait(&s_empty[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status,
+                                             TG_STATUS_ATTENTION_TIMEOUT)))
+                            break;
+                        tc_fence_after();
+                        issue_s(h, j + 1);
+                    }
+                    if (!ok) break;
+                    mma_commit(&k_empty[(j + 1) % kStages]);
+                }
+                // P_h(j) V_j for each head once its softmax has written P_h(j)
                 if (!(ok = mbar_wait(&v_ready[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
                                      TG_STATUS_ATTENTION_TIMEOUT)))
                     break;
-                const uint32_t v_addr = smem_u32(smem + C::kOffV + st * C::kTile);
+                const uint32_t v_addr = smem_u32(smem + C::kOffV + st * C::kKVTile);
                 for (int h = 0; h < NQ && ok; ++h) {
                     if (!(ok = mbar_wait(&p_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status,
                                          TG_STATUS_ATTENTION_TIMEOUT)))
@@ -285,22 +306,15 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < kBN / 16; ++k)  // 16 keys per step: 16 rows of 128 bytes in each chunk
-                        mma_ts(tmem + C::col_o(h), tmem + C::col_s(h) + static_cast<uint32_t>(k * 8),
+                        mma_ts(tmem + C::col_o(h), tmem + C::col_p(h) + static_cast<uint32_t>(k * 8),
                                smem_desc_sw128(v_addr + static_cast<uint32_t>(k * 2048), kBN * 128, 1024),
                                idesc_o, (j > 0 || k > 0) ? 1u : 0u);
-                    if (next) {
-                        if (h == 0 && !(ok = wait_k(j + 1))) break;
-                        tc_fence_after();
-                        issue_s(h, j + 1);  // overwrites S_h/P_h after the P V above (MMAs run in order)
-                    }
+                    mma_commit(&pv_done[h]);
                 }
                 if (!ok) break;
                 mma_commit(&v_empty[st]);
-                if (next) mma_commit(&k_empty[(j + 1) % kStages]);
             }
-            if (ok) {
-                for (int h = 0; h < NQ; ++h) mma_commit(&o_final[h]);
-            } else {
+            if (!ok) {
                 mma_commit(drain);
                 volatile int no_abort = 0;
                 mbar_wait(drain, 0, &no_abort, a.status, TG_STATUS_ATTENTION_TIMEOUT);
@@ -314,9 +328,9 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             if (!mbar_wait(&v_full[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
                            TG_STATUS_ATTENTION_TIMEOUT))
                 break;
-            uint4* vt = reinterpret_cast<uint4*>(smem + C::kOffV + st * C::kTile);
+            uint4* vt = reinterpret_cast<uint4*>(smem + C::kOffV + st * C::kKVTile);
 #pragma unroll 4
-            for (int i = t; i < C::kTile / 16; i += 64) {
+            for (int i = t; i < C::kKVTile / 16; i += 64) {
                 uint4 x = vt[i];
                 uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -336,54 +350,60 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         const int head = head0 + h;
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + C::col_s(h);
+        const uint32_t p_addr = tmem + lane_off + C::col_p(h);
         const uint32_t o_addr = tmem + lane_off + C::col_o(h);
         const float gain = a.gain ? a.gain[head] * kLog2e : 0.0f;
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
         float* bias_h = bias_s + h * 2 * kBN;
-        float s_pref = (a.s_kept && t < a.K) ? a.s_kept[t] : 0.0f;
+        float s_pref = (a.s_kept && t < kBN && t < a.K) ? a.s_kept[t] : 0.0f;
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < n_kv && ok; ++j) {
             const int b = j & 1;
             // this tile's key bias g_h * s_c in log2 units (one key per thread), next tile's score prefetched
-            bias_h[b * kBN + t] = gain * s_pref;
+            if (t < kBN) bias_h[b * kBN + t] = gain * s_pref;
             mbar_arrive(&bias_full[2 * h + b]);
             {
                 const int64_t cn = static_cast<int64_t>(j + 1) * kBN + t;
-                s_pref = (a.s_kept && j + 1 < n_kv && cn < a.K) ? a.s_kept[cn] : 0.0f;
+                s_pref = (a.s_kept && t < kBN && j + 1 < n_kv && cn < a.K) ? a.s_kept[cn] : 0.0f;
             }
             if (!(ok = warp_wait(&bias_full[2 * h + b], static_cast<uint32_t>(j >> 1) & 1, abort_flag, a.status)))
                 break;
             if (!(ok = warp_wait(&s_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status))) break;
             tc_fence_after();
-            const float* bias = bias_h + b * kBN;
-            const bool diag = (j == n_kv - 1);
-
-            // pass 1: row max of x = S * scale + bias
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld32(s_addr + c0, v);
+            // the row's 64 S values, then hand the S columns back to the MMA warp
+            float x[kBN];
+            {
+                uint32_t* xv = reinterpret_cast<uint32_t*>(x);
+                tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(xv));
+                tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(xv + 32));
                 tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float4 bb = *reinterpret_cast<const float4*>(bias + c0 + i);
-                    float2 x0 = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), sc2,
-                                      make_float2(bb.x, bb.y));
-                    float2 x1 = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), sc2,
-                                      make_float2(bb.z, bb.w));
-                    if (diag) {
-                        const int c = c0 + i;
-                        if (c > row) x0.x = -INFINITY;
-                        if (c + 1 > row) x0.y = -INFINITY;
-                        if (c + 2 > row) x1.x = -INFINITY;
-                        if (c + 3 > row) x1.y = -INFINITY;
-                    }
-                    mx = fmax3(mx, x0.x, x0.y);
-                    mx = fmax3(mx, x1.x, x1.y);
-                }
             }
+            tc_fence_before();
+            mbar_arrive(&s_empty[h]);
+            const float* bias = bias_h + b * kBN;
+            // keys c with j * kBN + c > m_tile * kBM + row are in the future of this query row
+            const int lim = m_tile * kBM + row - j * kBN;
+            const bool diag = j >= first_diag;
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < kBN; c += 4) {
+                const float4 bb = *reinterpret_cast<const float4*>(bias + c);
+                float2 x0 = ffma2(make_float2(x[c], x[c + 1]), sc2, make_float2(bb.x, bb.y));
+                float2 x1 = ffma2(make_float2(x[c + 2], x[c + 3]), sc2, make_float2(bb.z, bb.w));
+                if (diag) {
+                    if (c > lim) x0.x = -INFINITY;
+                    if (c + 1 > lim) x0.y = -INFINITY;
+                    if (c + 2 > lim) x1.x = -INFINITY;
+                    if (c + 3 > lim) x1.y = -INFINITY;
+                }
+                x[c] = x0.x;
+                x[c + 1] = x0.y;
+                x[c + 2] = x1.x;
+                x[c + 3] = x1.y;
+                mx4[(c >> 2) & 3] = fmax3(mx4[(c >> 2) & 3], fmaxf(x0.x, x0.y), fmaxf(x1.x, x1.y));
+            }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             // lazy rescaling: keep the stale max unless this row's max grew by more than 2^8
             const bool need = mx > m_run + kRescaleThreshold;
             float alpha = 1.0f;
@@ -392,58 +412,48 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 m_run = mx;
                 l_run *= alpha;
             }
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-                // O_h holds exactly P(j-1) V(j-1) and earlier here (see the ordering note above)
+            // P_h(j-1) V_{j-1} must be complete before O is rescaled and P_h is overwritten
+            if (j > 0) {
+                if (!(ok = warp_wait(&pv_done[h], static_cast<uint32_t>(j - 1) & 1, abort_flag, a.status))) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld16(o_addr + c0, v);
+                        tmem_ld_wait();
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(o_addr + c0, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                    tmem_st16(o_addr + c0, v);
+                        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                        tmem_st16(o_addr + c0, v);
+                    }
                 }
             }
-            // pass 2: P = 2^(x - m) as fp16, written over the S columns already consumed
+            // P = 2^(x - m) as fp16 into P_h
             const float2 neg_m = make_float2(-m_run, -m_run);
-            float2 lsum = make_float2(0.0f, 0.0f);
-#pragma unroll 1
+            float2 ls[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll
             for (int c0 = 0; c0 < kBN; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld32(s_addr + c0, v);
-                tmem_ld_wait();
                 uint32_t p16[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 4) {
-                    const float4 bb = *reinterpret_cast<const float4*>(bias + c0 + i);
-                    float2 x0 = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), sc2,
-                                      make_float2(bb.x, bb.y));
-                    float2 x1 = ffma2(make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), sc2,
-                                      make_float2(bb.z, bb.w));
-                    if (diag) {
-                        const int c = c0 + i;
-                        if (c > row) x0.x = -INFINITY;
-                        if (c + 1 > row) x0.y = -INFINITY;
-                        if (c + 2 > row) x1.x = -INFINITY;
-                        if (c + 3 > row) x1.y = -INFINITY;
-                    }
-                    x0 = fadd2(x0, neg_m);
-                    x1 = fadd2(x1, neg_m);
-                    const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
-                    const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
-                    lsum = fadd2(lsum, p0);
-                    lsum = fadd2(lsum, p1);
+                    const float2 y0 = fadd2(make_float2(x[c0 + i], x[c0 + i + 1]), neg_m);
+                    const float2 y1 = fadd2(make_float2(x[c0 + i + 2], x[c0 + i + 3]), neg_m);
+                    const float2 p0 = make_float2(ex2(y0.x), ex2(y0.y));
+                    const float2 p1 = make_float2(ex2(y1.x), ex2(y1.y));
+                    ls[0] = fadd2(ls[0], p0);
+                    ls[1] = fadd2(ls[1], p1);
                     p16[i / 2] = f16x2(p0.x, p0.y);
                     p16[i / 2 + 1] = f16x2(p1.x, p1.y);
                 }
-                tmem_st16(s_addr + (c0 >> 1), p16);
+                tmem_st16(p_addr + (c0 >> 1), p16);
             }
+            const float2 lsum = fadd2(ls[0], ls[1]);
             tmem_st_wait();
             l_run += lsum.x + lsum.y;
             tc_fence_before();
             mbar_arrive(&p_full[h]);
         }
-        if (ok && warp_wait(&o_final[h], 0, abort_flag, a.status)) {
+        if (ok && warp_wait(&pv_done[h], static_cast<uint32_t>(n_kv - 1) & 1, abort_flag, a.status)) {
             // epilogue: normalise, store bf16 rows and the log-sum-exp
             tc_fence_after();
             const int64_t grow = static_cast<int64_t>(m_tile) * kBM + row;
@@ -514,17 +524,18 @@ extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg
         return TG_ERR_INVALID_ARG;
 
     CUtensorMap mq, mk, mv;
-    const uint32_t box[3] = {64, 1, 128};
+    const uint32_t qbox[3] = {64, 1, 128};
+    const uint32_t kvbox[3] = {64, 1, static_cast<uint32_t>(attn::kBN)};
     {
         const uint64_t dims[3] = {static_cast<uint64_t>(d_h), static_cast<uint64_t>(Hq), static_cast<uint64_t>(K)};
         const uint64_t str[2] = {static_cast<uint64_t>(d_h) * 2, static_cast<uint64_t>(ld_q) * 2};
-        if (!make_tmap_bf16(&mq, q, 3, dims, str, box)) return TG_ERR_CUDA;
+        if (!make_tmap_bf16(&mq, q, 3, dims, str, qbox)) return TG_ERR_CUDA;
     }
     {
         const uint64_t dims[3] = {static_cast<uint64_t>(d_h), static_cast<uint64_t>(Hkv), static_cast<uint64_t>(K)};
         const uint64_t sk[2] = {static_cast<uint64_t>(d_h) * 2, static_cast<uint64_t>(ld_k) * 2};
         const uint64_t sv[2] = {static_cast<uint64_t>(d_h) * 2, static_cast<uint64_t>(ld_v) * 2};
-        if (!make_tmap_bf16(&mk, k, 3, dims, sk, box) || !make_tmap_bf16(&mv, v, 3, dims, sv, box))
+        if (!make_tmap_bf16(&mk, k, 3, dims, sk, kvbox) || !make_tmap_bf16(&mv, v, 3, dims, sv, kvbox))
             return TG_ERR_CUDA;
     }
     attn::Args a;
