@@ -253,6 +253,9 @@ gate_score_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_const
                         ss1 = fmaf(hi, hi, ss1);
                     }
                 }
+                // These generic-proxy reads must be ordered before the TMA (async proxy) that
+                // refills this stage once it is released; the mbarrier alone does not order them.
+                fence_proxy_async_smem();
                 mbar_arrive(&empty[s]);
                 if (++s == C::kStages) {
                     s = 0;

@@ -112,3 +112,13 @@ def test_rope_against_oracle(K, Hq, Hkv, d_h, max_pos):
         tol = np.abs(ref) * (2.0 ** -8 + 1e-6) + 1e-6
         assert np.all(np.abs(got - ref) <= tol), np.max(np.abs(got - ref) - tol)
     assert torch.equal(d[:, (Hq + Hkv) * d_h:], v_before)          # v untouched
+
+
+@pytest.mark.parametrize("N,db,de,k", [(131072, 0, 130560, 4096), (300000, 1000, 299000, 100000)])
+def test_select_repeatable(N, db, de, k):
+    s = synth.score_vector(N, 21, "ties")
+    ws = tg.new_workspace(N)
+    first = _select_gpu(s, db, de, k, ws)
+    for _ in range(5):
+        assert np.array_equal(_select_gpu(s, db, de, k, ws), first)
+    assert np.array_equal(first, oracle.topk_select(s.numpy(), db, de, k))
