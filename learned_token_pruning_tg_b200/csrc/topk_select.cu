@@ -6,10 +6,7 @@
 // output order are the specification's; NaN ranks below every number and
 // -0 equals +0.
 //
-// Two launch shapes, same algorithm.  Spans up to 8 * 1024 * 32 keys run in
-// one 8-CTA thread-block cluster (see topk_select_cluster_kernel: histograms
-// merged through distributed shared memory, hardware cluster barriers).
-// Longer spans use one cooperative launch, G <= #SM blocks of 1024 threads:
+// Design (one cooperative launch, G <= #SM blocks of 1024 threads):
 //   * every score is mapped to an order-preserving 32-bit key and kept in
 //     registers for the whole kernel (block b owns a contiguous chunk of the
 //     span, thread t the elements t, t+1024, ... of it);
@@ -252,183 +249,6 @@ __global__ void select_trivial_kernel(int64_t N, int64_t D0, int64_t D1, int kee
     }
 }
 
-// ---------------------------------------------------------------- one-cluster variant
-// For spans up to kClusterCtas * 1024 * 32 keys, one cluster of kClusterCtas
-// CTAs (one per SM) holds every key in registers.  The per-pass histograms are
-// merged in CTA 0's shared memory through distributed shared memory (remote
-// atomics) and read back the same way; hardware cluster barriers replace the
-// global-memory grid barriers, and no global scratch is needed.
-constexpr int kClusterCtas = 8;
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Address of the same shared-memory variable in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void dsmem_add(uint32_t addr, uint32_t v) {
-    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void dsmem_st(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-template <int EPT>
-__global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(const SelectArgs a) {
-    __shared__ unsigned int s_hist[2048];
-    __shared__ unsigned int s_red[3][2048];     // cluster-merged histograms (meaningful in CTA 0)
-    __shared__ unsigned int s_cnt[2][kClusterCtas];  // per-CTA counts above / equal to T (in CTA 0)
-    __shared__ unsigned int s_warp[32];
-    __shared__ unsigned int s_pick[2];
-    const int tid = threadIdx.x, lane = tid & 31;
-    const uint32_t rank = cluster_rank();
-    const int64_t chunk = static_cast<int64_t>(a.ept) * kSelectThreads;
-    const int64_t base = a.D0 + static_cast<int64_t>(rank) * chunk;
-    const int64_t end = min(base + chunk, a.D1);
-
-    uint32_t key[EPT];
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-        const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
-        key[j] = (j < a.ept && i < end) ? radix_key(__ldg(a.scores + i)) : 0u;
-    }
-    if (rank == 0)
-        for (int b = tid; b < 3 * 2048; b += kSelectThreads) (&s_red[0][0])[b] = 0u;
-    cluster_sync();  // CTA 0's merge buffers are zero before anyone adds into them
-
-    uint32_t prefix = 0, pmask = 0;
-    unsigned int krem = a.kd;  // 1-based rank of the target among keys matching `prefix`
-#pragma unroll 1
-    for (int p = 0; p < 3; ++p) {
-        const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
-        const int nb = p == 2 ? 1024 : 2048;
-        const uint32_t dmask = static_cast<uint32_t>(nb - 1);
-        for (int b = tid; b < 2048; b += kSelectThreads) s_hist[b] = 0;
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < EPT; ++j) {
-            if (j < a.ept) {
-                const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
-                const bool match = i < end && (key[j] & pmask) == prefix;
-                const unsigned active = __ballot_sync(0xffffffffu, match);
-                if (match) {
-                    const uint32_t digit = (key[j] >> shift) & dmask;
-                    const unsigned peers = __match_any_sync(active, digit);
-                    if (lane == __ffs(peers) - 1) atomicAdd(&s_hist[digit], static_cast<unsigned>(__popc(peers)));
-                }
-            }
-        }
-        __syncthreads();
-        for (int b = tid; b < nb; b += kSelectThreads) {
-            const unsigned c = s_hist[b];
-            if (c) dsmem_add(dsmem_addr(&s_red[p][b], 0), c);
-        }
-        cluster_sync();
-        // every CTA scans the merged histogram (identically) from the top digit down
-        const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
-        const unsigned c0 = d0 >= 0 ? dsmem_ld(dsmem_addr(&s_red[p][d0], 0)) : 0u;
-        const unsigned c1 = d1 >= 0 ? dsmem_ld(dsmem_addr(&s_red[p][d1], 0)) : 0u;
-        unsigned tot;
-        const unsigned e = block_excl_scan(c0 + c1, s_warp, &tot);
-        if (e < krem && krem <= e + c0) {
-            s_pick[0] = static_cast<unsigned>(d0);
-            s_pick[1] = e;
-        } else if (e + c0 < krem && krem <= e + c0 + c1) {
-            s_pick[0] = static_cast<unsigned>(d1);
-            s_pick[1] = e + c0;
-        }
-        __syncthreads();
-        prefix |= s_pick[0] << shift;
-        pmask |= dmask << shift;
-        krem -= s_pick[1];
-        __syncthreads();
-    }
-    const uint32_t T = prefix;
-
-    // per-CTA counts of keys above T and equal to T, published to CTA 0
-    unsigned cnt = 0;
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-        const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
-        if (j < a.ept && i < end) cnt += (key[j] > T ? 1u : 0u) + (key[j] == T ? 0x10000u : 0u);
-    }
-    unsigned btot;
-    block_excl_scan(cnt, s_warp, &btot);
-    if (tid == 0) {
-        dsmem_st(dsmem_addr(&s_cnt[0][rank], 0), btot & 0xffffu);
-        dsmem_st(dsmem_addr(&s_cnt[1][rank], 0), btot >> 16);
-    }
-    cluster_sync();
-    if (tid == 0) {
-        unsigned g = 0, q = 0;
-        for (uint32_t r = 0; r < rank; ++r) {
-            g += dsmem_ld(dsmem_addr(&s_cnt[0][r], 0));
-            q += dsmem_ld(dsmem_addr(&s_cnt[1][r], 0));
-        }
-        s_pick[0] = g;
-        s_pick[1] = q;
-    }
-    __syncthreads();
-    unsigned run_g = s_pick[0], run_e = s_pick[1];
-#pragma unroll
-    for (int j = 0; j < EPT; ++j) {
-        if (j < a.ept) {
-            const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
-            const bool valid = i < end;
-            const bool fg = valid && key[j] > T;
-            const bool fe = valid && key[j] == T;
-            unsigned t2;
-            const unsigned ex = block_excl_scan((fg ? 1u : 0u) | (fe ? 0x10000u : 0u), s_warp, &t2);
-            const unsigned g_before = run_g + (ex & 0xffffu);
-            const unsigned e_before = run_e + (ex >> 16);
-            if (fg)
-                a.out[a.D0 + g_before + min(e_before, krem)] = static_cast<int32_t>(i);
-            else if (fe && e_before < krem)
-                a.out[a.D0 + g_before + e_before] = static_cast<int32_t>(i);
-            run_g += t2 & 0xffffu;
-            run_e += t2 >> 16;
-        }
-    }
-    // Tokens outside the span are always kept: [0, D0) first, [D1, N) after the kept document tokens.
-    const int64_t gstride = static_cast<int64_t>(kClusterCtas) * kSelectThreads;
-    for (int64_t i = static_cast<int64_t>(rank) * kSelectThreads + tid; i < a.D0; i += gstride)
-        a.out[i] = static_cast<int32_t>(i);
-    for (int64_t i = a.D1 + static_cast<int64_t>(rank) * kSelectThreads + tid; i < a.N; i += gstride)
-        a.out[a.D0 + a.kd + (i - a.D1)] = static_cast<int32_t>(i);
-    cluster_sync();  // CTA 0's shared memory stays alive until every CTA has read it
-}
-
-template <int EPT>
-static cudaError_t launch_select_cluster(const SelectArgs& a, cudaStream_t st) {
-    auto kern = topk_select_cluster_kernel<EPT>;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kClusterCtas);
-    cfg.blockDim = dim3(kSelectThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kClusterCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a);
-}
-
 template <int EPT>
 static cudaError_t launch_select(const SelectArgs& a, int grid, cudaStream_t st) {
     void* args[] = {const_cast<SelectArgs*>(&a)};
@@ -459,33 +279,6 @@ extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_
     }
     if (!workspace || workspace_bytes < tg_workspace_bytes(TG_OP_SELECT, N, 0, 0)) return TG_ERR_INVALID_ARG;
     if (!aligned16(workspace)) return TG_ERR_INVALID_ARG;
-    {
-        // one cluster when every key fits in registers (up to 32 per thread)
-        const int64_t per_cta = (n_doc + kClusterCtas - 1) / kClusterCtas;
-        const int64_t ept_c = (per_cta + kSelectThreads - 1) / kSelectThreads;
-        if (ept_c <= 32) {
-            SelectArgs a;
-            a.scores = scores;
-            a.N = N;
-            a.D0 = doc_begin;
-            a.D1 = doc_end;
-            a.kd = static_cast<unsigned int>(kd);
-            a.out = kept_idx;
-            a.sc = nullptr;
-            a.status = status_word(workspace);
-            a.ept = static_cast<int>(ept_c);
-            cudaError_t e;
-            if (ept_c <= 4)
-                e = launch_select_cluster<4>(a, st);
-            else if (ept_c <= 8)
-                e = launch_select_cluster<8>(a, st);
-            else if (ept_c <= 16)
-                e = launch_select_cluster<16>(a, st);
-            else
-                e = launch_select_cluster<32>(a, st);
-            return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;
-        }
-    }
     const int sms = num_sms();
     const int64_t per_block_min = kSelectThreads;
     int64_t ept = (n_doc + static_cast<int64_t>(sms) * per_block_min - 1) / (static_cast<int64_t>(sms) * per_block_min);
