@@ -125,6 +125,31 @@ tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_begin,
                          int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Top-K selection that allocates nothing and takes no workspace.
+ * There is no counterpart on the TokenGate pages: this is a calling-convention
+ * variant of tg_topk_select for callers that cannot allocate device memory
+ * when they select (code running inside an allocator or memory-pool callback,
+ * a serving process whose device memory is fully reserved up front by its own
+ * pool, a host environment that only lends the library the buffers it owns).
+ * Same arguments (minus the workspace), same result, bit for bit, as
+ * tg_topk_select.
+ * Scratch: a static device array of 34,560 bytes inside the library, which
+ * every GPU that loads the library keeps until the process exits.  The first
+ * call on each device looks up that array's device address (with the device
+ * current), so make the first call on a device before any stream capture.
+ * Every call shares the array and clears it on the stream before use; calls
+ * that overlap on the GPU (different streams, or several host threads) race
+ * on it and must be serialised by the caller.  It never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ * Limit: doc_end - doc_begin <= #SMs * 1024 * 16 (2,424,832 on a 148-SM B200,
+ * the largest grid the select kernel uses); longer spans return
+ * TG_ERR_UNSUPPORTED before anything is launched.
+ * A device-side wait that times out leaves kept_idx undefined; this entry
+ * point reports launch errors only. */
+tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int64_t doc_begin,
+                                 int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
+                                 void* stream);
+
 /* Compaction (step 3: layers above the gate see only the K kept tokens):
  *   h_out[r, :] = h[kept_idx[r], :]           (bit-exact copy)
  *   pos_out[r]  = pos_in ? pos_in[kept_idx[r]] : kept_idx[r]

@@ -22,6 +22,8 @@
 //     counts after one more grid barrier, in-block prefixes from ballots.
 // The grid barrier is a sense-reversing counter in the workspace that resets
 // itself; each wait is bounded and reports TG_STATUS_SELECT_TIMEOUT.
+#include <mutex>
+
 #include "tg_host.cuh"
 
 namespace tg {
@@ -297,6 +299,102 @@ extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_
     a.out = kept_idx;
     a.sc = reinterpret_cast<SelectScratch*>(static_cast<char*>(workspace) + kWsHeader);
     a.status = status_word(workspace);
+    a.ept = static_cast<int>(ept);
+    cudaError_t e;
+    if (ept <= 1)
+        e = launch_select<1>(a, grid, st);
+    else if (ept <= 2)
+        e = launch_select<2>(a, grid, st);
+    else if (ept <= 4)
+        e = launch_select<4>(a, grid, st);
+    else if (ept <= 8)
+        e = launch_select<8>(a, grid, st);
+    else
+        e = launch_select<16>(a, grid, st);
+    return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- allocation-free entry point
+// Some callers cannot allocate device memory at the point where they select
+// tokens: code that runs inside an allocator or memory-pool callback, a serving
+// process whose device memory is fully reserved up front and handed out by its
+// own pool, or a host environment that only hands the library pointers to
+// buffers it owns.  tg_topk_select_noalloc serves them: it needs no workspace
+// argument, because its scratch lives in the static device array below, which
+// every GPU that loads this library keeps for the lifetime of the process.
+namespace tg {
+namespace noalloc {
+
+// status word (first 256 bytes) + the select scratch: 34,560 bytes in all.
+constexpr size_t kScratchBytes = kWsHeader + ((sizeof(SelectScratch) + 255) / 256) * 256;
+static_assert(kScratchBytes == 34560, "the documented size of the static scratch");
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+// Device address of g_scratch per device.  In host code the symbol name is only
+// a host-side stand-in, so the address has to be queried with the device current.
+constexpr int kMaxDevices = 64;
+static void* g_addr[kMaxDevices] = {nullptr};
+static std::mutex g_mu;
+
+static tg_status scratch_for_current_device(unsigned char** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TG_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return TG_ERR_CUDA;
+        }
+        g_addr[dev] = p;
+    }
+    *out = static_cast<unsigned char*>(g_addr[dev]);
+    return TG_OK;
+}
+
+}  // namespace noalloc
+}  // namespace tg
+
+extern "C" tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int64_t doc_begin, int64_t doc_end,
+                                            int64_t k_doc, int32_t* kept_idx, void* stream) {
+    const int64_t K = tg_kept_count(N, doc_begin, doc_end, k_doc);
+    if (K < 0) return TG_ERR_INVALID_ARG;
+    if (N > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
+    if (K == 0) return TG_OK;
+    if (!scores || !kept_idx) return TG_ERR_INVALID_ARG;
+    const int64_t n_doc = doc_end - doc_begin;
+    const int64_t kd = k_doc < n_doc ? k_doc : n_doc;
+    cudaStream_t st = as_stream(stream);
+    if (kd == 0 || kd == n_doc) {
+        const int64_t blocks = std::min<int64_t>((N + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
+        select_trivial_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(N, doc_begin, doc_end,
+                                                                             kd == n_doc ? 1 : 0, kept_idx);
+        return launch_status();
+    }
+    // the same launch shape as tg_topk_select; spans beyond its largest grid are rejected
+    const int sms = num_sms();
+    int64_t ept = (n_doc + static_cast<int64_t>(sms) * kSelectThreads - 1) / (static_cast<int64_t>(sms) * kSelectThreads);
+    if (ept < 1) ept = 1;
+    if (ept > kSelectMaxEpt) return TG_ERR_UNSUPPORTED;
+    const int64_t chunk = ept * kSelectThreads;
+    const int grid = static_cast<int>((n_doc + chunk - 1) / chunk);
+    if (grid > kSelectMaxBlocks) return TG_ERR_UNSUPPORTED;
+
+    unsigned char* scratch = nullptr;
+    if (noalloc::scratch_for_current_device(&scratch) != TG_OK) return TG_ERR_CUDA;
+    // The array keeps whatever the previous call left; the barrier counters, the
+    // histograms and the status word must start at zero, so clear them first.
+    if (cudaMemsetAsync(scratch, 0, noalloc::kScratchBytes, st) != cudaSuccess) return TG_ERR_CUDA;
+
+    SelectArgs a;
+    a.scores = scores;
+    a.N = N;
+    a.D0 = doc_begin;
+    a.D1 = doc_end;
+    a.kd = static_cast<unsigned int>(kd);
+    a.out = kept_idx;
+    a.sc = reinterpret_cast<SelectScratch*>(scratch + kWsHeader);
+    a.status = reinterpret_cast<unsigned int*>(scratch);
     a.ept = static_cast<int>(ept);
     cudaError_t e;
     if (ept <= 1)

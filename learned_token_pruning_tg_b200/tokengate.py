@@ -47,12 +47,13 @@ def lib() -> ctypes.CDLL:
         L.tg_workspace_bytes.restype = sz
         L.tg_gate_score.argtypes = [vp, i64, i32, i64, vp, f32, vp, vp, vp, f32, i32, vp, vp, sz, vp]
         L.tg_topk_select.argtypes = [vp, i64, i64, i64, i64, vp, vp, sz, vp]
+        L.tg_topk_select_noalloc.argtypes = [vp, i64, i64, i64, i64, vp, vp]
         L.tg_gather_compact.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, vp, vp, vp]
         L.tg_rope_apply.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, f64, vp]
         L.tg_gated_attention.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp,
                                          vp, sz, vp]
         L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
-        for fn in ("tg_gate_score", "tg_topk_select", "tg_gather_compact", "tg_rope_apply",
+        for fn in ("tg_gate_score", "tg_topk_select", "tg_topk_select_noalloc", "tg_gather_compact", "tg_rope_apply",
                    "tg_gated_attention", "tg_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -149,6 +150,23 @@ def tg_topk_select(scores, doc_begin: int, doc_end: int, k_doc: int, kept_idx, w
     _check("tg_topk_select", lib().tg_topk_select(
         _ptr(scores), N, doc_begin, doc_end, k_doc, _ptr(kept_idx), _ptr(workspace), workspace.numel(),
         _stream(stream)))
+    return kept_idx
+
+
+def tg_topk_select_noalloc(scores, doc_begin: int, doc_end: int, k_doc: int, kept_idx, stream=None):
+    """tg_topk_select without a workspace: for callers that cannot allocate device memory
+    when they select.  Its scratch is a static array inside the library shared by every call,
+    so calls must not overlap on the GPU."""
+    _req(scores, "scores", torch.float32, 1)
+    _req(kept_idx, "kept_idx", torch.int32, 1)
+    N = scores.shape[0]
+    K = tg_kept_count(N, doc_begin, doc_end, k_doc)
+    if K < 0:
+        raise TokenGateError("tg_topk_select_noalloc", TG_ERR_INVALID_ARG)
+    if kept_idx.numel() < K or not scores.is_contiguous() or not kept_idx.is_contiguous():
+        raise ValueError("kept_idx too small or not contiguous")
+    _check("tg_topk_select_noalloc", lib().tg_topk_select_noalloc(
+        _ptr(scores), N, doc_begin, doc_end, k_doc, _ptr(kept_idx), _stream(stream)))
     return kept_idx
 
 
