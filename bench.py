@@ -60,6 +60,28 @@ def config_dict(w):
             "path": "gate, select, gather, qkv (cuBLAS glue), rope, attention", "seed": w.seed}
 
 
+# ---------------------------------------------------------------- multi-rank plumbing
+def reduce_max(x: float, device) -> float:
+    """Max of x over all ranks (a no-op on one process).  Replicas run independent prefills,
+    so the job's time is that of its slowest rank."""
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(w, rank: int) -> int:
+    """Each rank prefills its own prompt (independent problems): a different seed per rank."""
+    return w.seed + rank
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: tokens all ranks processed over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
+
+
 # ---------------------------------------------------------------- algorithmic work per stage
 def stage_work(w):
     """Algorithmic FLOPs and bytes of each stage (per step)."""
@@ -267,8 +289,8 @@ def run_tokengate(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = WORKLOAD
-    gi = synth.gate_inputs(w, seed=w.seed + rank)
-    ap = synth.attn_params(w, seed=w.seed + rank)
+    gi = synth.gate_inputs(w, seed=replica_seed(w, rank))
+    ap = synth.attn_params(w, seed=replica_seed(w, rank))
     Wqkv = torch.cat([ap.Wq, ap.Wk, ap.Wv], dim=0)
     layer = GatedPrefillLayer(w.N, w.doc_begin, w.doc_end, w.k_doc, gi.W1, gi.w2, Wqkv, w.Hq, w.Hkv, w.d_h,
                               ap.gain, ap.tau, eps=w.eps, rope_base=w.rope_base, device=dev)
@@ -310,11 +332,8 @@ def run_tokengate(args, rank, world, local_rank):
         for j, s in enumerate(STAGES):
             stage_ms[s] += marks[i][j].elapsed_time(marks[i][j + 1]) / K
     status = tg.tg_device_status(layer.ws)
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = w.N * world / (ms_step * 1e-3)
+    ms_step = reduce_max(ms_step, dev)
+    value = job_throughput(w.N, world, ms_step)
 
     # end to end through the same API from pinned host memory: H2D of h, the path, D2H of out + kept
     h_host = gi.h.pin_memory()
@@ -334,11 +353,8 @@ def run_tokengate(args, rank, world, local_rank):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": w.N * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+    e2e_ms = reduce_max(e2e_ms, dev)
+    e2e = {"value": job_throughput(w.N, world, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h_host.numel() * h_host.element_size(),
            "d2h_bytes_per_step": out_host.numel() * out_host.element_size() + kept_host.numel() * 4,
            "ms_per_step": e2e_ms}
