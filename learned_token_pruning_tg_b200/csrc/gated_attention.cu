@@ -259,17 +259,23 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 return mbar_wait(&k_full[j % kStages], static_cast<uint32_t>(j / kStages) & 1, abort_flag,
                                  a.status, TG_STATUS_ATTENTION_TIMEOUT);
             };
+            // Descriptors as 32-bit start/LBO words over one shared high word (SBO 1024,
+            // 128-byte swizzle): every MMA below moves its operands by compile-time
+            // offsets, so the issuing thread keeps ahead of the tensor pipe.
+            const uint32_t dhi = sw128_desc_hi(1024);
+            const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffQ), 16);
+            const uint32_t k_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffK), 16);
+            const uint32_t v_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffV), kBN * 128);
             // S_h = Q_h K_j^T into head h's S columns, then signal softmax h
             auto issue_s = [&](int h, int j) {
-                const uint32_t q_addr = smem_u32(smem + C::kOffQ + h * C::kQTile);
-                const uint32_t k_addr = smem_u32(smem + C::kOffK + (j % kStages) * C::kKVTile);
+                const uint32_t q_lo = q_lo0 + static_cast<uint32_t>(h * (C::kQTile >> 4));
+                const uint32_t k_lo = k_lo0 + static_cast<uint32_t>((j % kStages) * (C::kKVTile >> 4));
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t koff = static_cast<uint32_t>((k & 3) * 32);
-                    mma_ss(tmem + C::col_s(h),
-                           smem_desc_sw128(q_addr + static_cast<uint32_t>((k >> 2) * (kBM * 128)) + koff, 16, 1024),
-                           smem_desc_sw128(k_addr + static_cast<uint32_t>((k >> 2) * (kBN * 128)) + koff, 16, 1024),
-                           idesc_s, k > 0);
+                    // K step k: 64-column chunk k / 4, 32-byte column offset k % 4 inside the swizzle atom
+                    const uint32_t qo = static_cast<uint32_t>(((k >> 2) * (kBM * 128) + (k & 3) * 32) >> 4);
+                    const uint32_t ko = static_cast<uint32_t>(((k >> 2) * (kBN * 128) + (k & 3) * 32) >> 4);
+                    mma_ss_lo(tmem + C::col_s(h), q_lo + qo, k_lo + ko, dhi, idesc_s, k > 0);
                 }
                 mma_commit(&s_full[h]);
             };
@@ -284,6 +290,7 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 // next S of each head as soon as its softmax has read the current one
                 if (j + 1 < n_kv) {
                     if (!(ok = wait_k(j + 1))) break;
+#pragma unroll
                     for (int h = 0; h < NQ && ok; ++h) {
                         if (!(ok = mbar_wait(&s_empty[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status,
                                              TG_STATUS_ATTENTION_TIMEOUT)))
@@ -298,7 +305,8 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 if (!(ok = mbar_wait(&v_ready[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
                                      TG_STATUS_ATTENTION_TIMEOUT)))
                     break;
-                const uint32_t v_addr = smem_u32(smem + C::kOffV + st * C::kKVTile);
+                const uint32_t v_lo = v_lo0 + static_cast<uint32_t>(st * (C::kKVTile >> 4));
+#pragma unroll
                 for (int h = 0; h < NQ && ok; ++h) {
                     if (!(ok = mbar_wait(&p_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status,
                                          TG_STATUS_ATTENTION_TIMEOUT)))
@@ -306,9 +314,9 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < kBN / 16; ++k)  // 16 keys per step: 16 rows of 128 bytes in each chunk
-                        mma_ts(tmem + C::col_o(h), tmem + C::col_p(h) + static_cast<uint32_t>(k * 8),
-                               smem_desc_sw128(v_addr + static_cast<uint32_t>(k * 2048), kBN * 128, 1024),
-                               idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+                        mma_ts_lo(tmem + C::col_o(h), tmem + C::col_p(h) + static_cast<uint32_t>(k * 8),
+                                  v_lo + static_cast<uint32_t>(k * (2048 >> 4)), dhi, idesc_o,
+                                  (j > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&pv_done[h]);
                 }
                 if (!ok) break;
