@@ -298,7 +298,7 @@ def run_tokengate(args, rank, world, local_rank):
     for _ in range(args.warmup):
         layer.run(h)
     torch.cuda.synchronize()
-    assert tg.tg_device_status(layer.ws) == 0, "device wait timed out during warm-up"
+    assert layer.device_status() == 0, "device wait timed out during warm-up"
 
     # per-stage CUDA events on the launching (current) stream
     K = args.steps
@@ -331,7 +331,7 @@ def run_tokengate(args, rank, world, local_rank):
     for i in range(K):
         for j, s in enumerate(STAGES):
             stage_ms[s] += marks[i][j].elapsed_time(marks[i][j + 1]) / K
-    status = tg.tg_device_status(layer.ws)
+    status = layer.device_status()
     ms_step = reduce_max(ms_step, dev)
     value = job_throughput(w.N, world, ms_step)
 

@@ -88,8 +88,14 @@ int32_t tg_version(void);
  * the span is not inside [0, N] or k_doc < 0. */
 int64_t tg_kept_count(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_doc);
 
-/* Workspace bytes needed by `op` for N tokens, hidden size d, gate width d_g
- * (arguments an op does not use are ignored).  Returns 0 for bad arguments. */
+/* Workspace bytes needed by `op` (arguments an op does not use are ignored):
+ *   TG_OP_GATE       N tokens of hidden size d, gate width d_g
+ *   TG_OP_SELECT     N scores
+ *   TG_OP_ATTENTION  N = K kept tokens, d = Hkv * d_h (the width of one
+ *                    token's V row; the workspace holds an fp16 copy of V)
+ *   TG_OP_ALL        every op above with these N, d, d_g (attention over at
+ *                    most N tokens whose V rows are at most d wide)
+ * Returns 0 for bad arguments. */
 size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g);
 
 /* Gate score (step 2: a small MLP on the post-attention residual):
@@ -181,10 +187,13 @@ tg_status tg_rope_apply(tg_bf16* q, int64_t ld_q, tg_bf16* k, int64_t ld_k,
  * ld_v (elements, multiples of 8).  s_kept: [K] fp32 or NULL (no bias).
  * gain: [Hq] fp32 or NULL (zeros).  out: [K, Hq, d_h] bf16 contiguous.
  * lse: [Hq, K] fp32 natural-log sum of exp of the logits, or NULL.
+ * tau > 0 (TG_ERR_INVALID_ARG otherwise).  workspace: at least
+ * tg_workspace_bytes(TG_OP_ATTENTION, K, Hkv * d_h, 0) bytes.
  * Supported: d_h in {64, 128}, Hq a multiple of Hkv, K < 2^31.
- * Tensor cores for Q K^T and P V (tcgen05, accumulators in TMEM), K/V tiles
- * staged by TMA, online softmax in fp32 with the bias added in registers,
- * P rounded to bf16 for the P V product. */
+ * Two launches: V to fp16 into the workspace, then the attention kernel:
+ * tensor cores for Q K^T (the key bias added by one extra MMA step) and P V
+ * (tcgen05, accumulators in TMEM), K/V tiles staged by TMA, online softmax in
+ * fp32, P and V in fp16 for the P V product. */
 tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
                              const tg_bf16* v, int64_t ld_v, int64_t K, int32_t Hq,
                              int32_t Hkv, int32_t d_h, const float* s_kept,

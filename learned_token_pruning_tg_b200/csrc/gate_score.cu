@@ -27,8 +27,6 @@
 #include "tg_host.cuh"
 
 namespace tg {
-size_t ws_gate_offset();
-
 namespace gate {
 
 constexpr int kBM = 128;       // rows per tile

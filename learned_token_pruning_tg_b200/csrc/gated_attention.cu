@@ -11,33 +11,46 @@
 //
 // Kernel: one CTA per (128-query tile, NQ query heads of one GQA group), the
 // heaviest query tiles first.  NQ = 2 when the group size is even: the two
-// heads share every K/V tile and their softmax warpgroups run side by side.
-//   warp 0      TMA: the NQ Q tiles once, then K and V tiles of 64 keys into
-//               two 4-stage rings (K runs one tile ahead of V)
-//   warp 1      TMEM allocation and the single MMA-issuing thread:
-//                 S_h = Q_h K_j^T   (kind::f16 bf16 x bf16 -> fp32, N = 64)
-//                 O_h += P_h V_j    (kind::f16 fp16 x fp16 -> fp32; P_h read
-//                                    from TMEM, V_j MN-major from smem)
-//               S_h(j+1) is issued as soon as softmax h has read S_h(j), so it
-//               runs while softmax h computes P_h(j): the MMA latency stays off
-//               the softmax's critical path.
-//   warps 2-3   convert each V tile to fp16 in place in shared memory (the
-//               swizzled layout is unchanged because both types are 2 bytes)
-//   warps 4+4h  softmax of head h, one query row per thread: the 64 S values of
-//               the row are read from TMEM once into registers, x = S tau /
-//               sqrt(d_h) log2(e) + g_h s_c log2(e) (key bias from a per-tile
-//               shared vector whose scores are prefetched a tile ahead), row
-//               max, P = 2^(x - m) as fp16 into TMEM.  Lazy rescaling: O is
-//               rescaled (in TMEM) only when a row max grows by more than 2^8,
-//               so P <= 256.  Causal masking only on the diagonal tiles.  At
-//               the end O / l to bf16 and the log-sum-exp.
+// heads share every K/V tile and their softmax warpgroups run side by side, so
+// the tensor pipe works on one head while the other head's softmax runs.
+// Tiles are 128 queries x 128 keys.
+//   warp 0      TMA: the NQ Q tiles once, then K and V tiles into two rings
+//               (K runs one tile ahead of V)
+//   warp 1      TMEM allocation and the single MMA-issuing thread, per key
+//               tile j and head h:
+//                 O_h += P_h(j) V_j      (kind::f16, fp16 x fp16 -> fp32; P_h
+//                                          read from TMEM, V_j MN-major in smem)
+//                 S_h(j+1) = Q_h K_{j+1}^T  (kind::f16, bf16 x bf16 -> fp32)
+//               P_h(j) is written over S_h(j)'s own columns, so S_h(j+1) is
+//               issued right behind P_h(j) V_j; the tensor pipe runs one
+//               thread's MMAs in order, so S_h(j+1) finishing also means
+//               P_h(j) V_j has finished and O_h may be rescaled.
+//   warp 2      the key-bias operand of each K tile (below)
+//   warps 3-6, 7-10   softmax of head 0, head 1 (one query row per thread;
+//               warp w owns TMEM lanes 32 (w mod 4) ..): the row's 128 S values
+//               are read from TMEM into registers, row max, then
+//               P = 2^(S c - m) with c = tau / sqrt(d_h) log2(e), as fp16 into
+//               the S columns.
+//               Lazy rescaling: O is rescaled (in TMEM) only when a row max
+//               grows by more than 2^8, so P <= 256.  Causal masking only on
+//               the diagonal tile.  At the end O / l to bf16 and the
+//               log-sum-exp.
+// The key bias rides in the tensor core: S is computed as
+//   S_h = Q_h K^T + A_h B^T,   A_h[r, 3i+k] = gamma_h^(i),   B[c, 3i+k] = s_c^(k)
+// (one extra K = 16 MMA step; gamma_h = g_h sqrt(d_h) / tau and s_c each split
+// into three bf16 parts whose sum is the fp32 value, so the nine products add
+// up to gamma_h s_c to fp32 accuracy), hence S c = tau q.k / sqrt(d_h) log2(e)
+// + g_h s_c log2(e): the logit in log2 units, with no per-element bias work.
+// This needs c > 0 (tau > 0).
 // P in fp16 (11 significant bits) rather than bf16 keeps the P V product's
 // relative error below 2^-11 per weight, which bounds the output error for
-// large-magnitude values; V is converted exactly (bf16 values in fp16's normal
-// range convert without rounding).
+// large-magnitude values.  V is converted to fp16 once, by a small pass into
+// the workspace before the attention kernel (bf16 values in fp16's normal
+// range convert without rounding); converting inside the attention kernel would
+// redo it for every query tile that reads the V tile.
 //
-// TMEM columns: S_h at 64 h, P_h at 128 + 32 h, O_h at 256 + d_h h (512 in all
-// for two heads of 128).  Every wait is bounded (TG_STATUS_ATTENTION_TIMEOUT).
+// TMEM columns: S_h (and P_h over it) at 128 h, O_h at 128 NQ + d_h h.  Every
+// wait is bounded (TG_STATUS_ATTENTION_TIMEOUT).
 #include <cmath>
 
 #include "tg_host.cuh"
@@ -45,32 +58,33 @@
 namespace tg {
 namespace attn {
 
-constexpr int kBM = 128;    // query rows per tile
-constexpr int kBN = 64;     // keys per tile
-constexpr int kStages = 4;  // depth of the K ring and of the V ring
+constexpr int kBM = 128;        // query rows per tile
+constexpr int kBN = 128;        // keys per tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 
 template <int D, int NQ>
 struct Cfg {
+    static constexpr int kStages = (D == 64) ? 4 : 2;  // depth of the K ring and of the V ring
     static constexpr int kQTile = kBM * D * 2;   // bytes of a 128 x D 16-bit tile
-    static constexpr int kKVTile = kBN * D * 2;  // bytes of a 64 x D 16-bit tile
+    static constexpr int kKVTile = kBN * D * 2;  // bytes of a 128 x D 16-bit tile
     static constexpr int kChunks = D / 64;       // 64-column (128-byte) swizzle chunks per row
-    static constexpr int kThreads = 32 * (4 + 4 * NQ);
+    static constexpr int kSoftmaxWarp0 = 3;
+    static constexpr int kThreads = 32 * (kSoftmaxWarp0 + 4 * NQ);
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + NQ * kQTile;
     static constexpr int kOffV = kOffK + kStages * kKVTile;
-    static constexpr int kOffBias = kOffV + kStages * kKVTile;  // float [NQ][2][64]
-    static constexpr int kOffBar = kOffBias + NQ * 2 * kBN * 4;
-    static constexpr int kNumBars = 1 + 5 * kStages + 6 * NQ + 1;
+    // bias operands, 128 rows x 16 bf16 each in the no-swizzle K-major layout (4 KB)
+    static constexpr int kAugTile = 4096;
+    static constexpr int kOffAugA = kOffV + kStages * kKVTile;  // [NQ]      gamma_h parts, every row alike
+    static constexpr int kOffAugB = kOffAugA + NQ * kAugTile;   // [kStages] s_c parts of a K tile's keys
+    static constexpr int kOffBar = kOffAugB + kStages * kAugTile;
+    static constexpr int kNumBars = 1 + 5 * kStages + 3 * NQ + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmem = kOffMisc + 16 + 1024;
-    static constexpr uint32_t kTmemCols = (NQ == 2) ? 512 : 256;
+    static constexpr uint32_t kTmemCols = (NQ * kBN + NQ * D > 256) ? 512 : 256;
     static __device__ __forceinline__ uint32_t col_s(int h) { return static_cast<uint32_t>(h * kBN); }
-    static __device__ __forceinline__ uint32_t col_p(int h) { return static_cast<uint32_t>(NQ * kBN + h * (kBN / 2)); }
-    static __device__ __forceinline__ uint32_t col_o(int h) {
-        return static_cast<uint32_t>((NQ == 2 ? 256 : 128) + h * D);
-    }
+    static __device__ __forceinline__ uint32_t col_o(int h) { return static_cast<uint32_t>(NQ * kBN + h * D); }
 };
 
 struct Args {
@@ -124,6 +138,21 @@ __device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
     return d;
 }
 
+// x as three bf16 parts (round to nearest at each step); their exact sum is x
+// to within fp32's own precision.
+__device__ __forceinline__ void split3_bf16(float x, __nv_bfloat16 (&p)[3]) {
+    p[0] = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(p[0]);
+    p[1] = __float2bfloat16_rn(r1);
+    p[2] = __float2bfloat16_rn(r1 - __bfloat162float(p[1]));
+}
+__device__ __forceinline__ uint32_t bf2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+// Row r's two 16-byte core-matrix rows of a 128 x 16 no-swizzle K-major tile
+// (LBO 128 bytes, SBO 256 bytes), in uint4 units from the tile start.
+__device__ __forceinline__ int aug_slot(int r, int chunk) { return (r >> 3) * 16 + chunk * 8 + (r & 7); }
+
 // Instruction descriptor for kind::f16 with fp16 A and B, fp32 accumulator
 // (A/B format field 0 = f16; same layout as idesc_bf16_f32 otherwise).
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major) {
@@ -144,24 +173,23 @@ __global__ void __launch_bounds__(Cfg<D, NQ>::kThreads, 1)
 gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const Args a) {
     using C = Cfg<D, NQ>;
+    constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* bias_s = reinterpret_cast<float*>(smem + C::kOffBias);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* q_full = bars;                      // TMA -> MMA
-    uint64_t* k_full = bars + 1;                  // [kStages] TMA -> MMA
-    uint64_t* k_empty = k_full + kStages;         // [kStages] commit after the last S of a K tile -> TMA
-    uint64_t* v_full = k_empty + kStages;         // [kStages] TMA -> converters
-    uint64_t* v_ready = v_full + kStages;         // [kStages] 64 converter threads -> MMA
-    uint64_t* v_empty = v_ready + kStages;        // [kStages] commit after the last P V of a V tile -> TMA
-    uint64_t* s_full = v_empty + kStages;         // [NQ] commit after S_h(j) -> softmax h
-    uint64_t* s_empty = s_full + NQ;              // [NQ] 128 softmax threads read S_h(j) -> MMA
-    uint64_t* p_full = s_empty + NQ;              // [NQ] 128 softmax threads wrote P_h(j) -> MMA
-    uint64_t* pv_done = p_full + NQ;              // [NQ] commit after P_h(j) V_j -> softmax h, epilogue
-    uint64_t* bias_full = pv_done + NQ;           // [NQ][2] 128 softmax threads (key-bias vector written)
-    uint64_t* drain = bias_full + 2 * NQ;         // abort path
+    uint64_t* q_full = bars;                        // TMA -> MMA
+    uint64_t* k_full = bars + 1;                    // [kStages] TMA -> MMA
+    uint64_t* k_empty = k_full + kStages;           // [kStages] commit after the last S of a K tile -> TMA
+    uint64_t* v_full = k_empty + kStages;           // [kStages] TMA -> MMA
+    uint64_t* v_empty = v_full + kStages;           // [kStages] commit after the last P V of a V tile -> TMA
+    uint64_t* aug_full = v_empty + kStages;         // [kStages] converter (32 lanes) wrote B of a K tile -> MMA
+    uint64_t* s_full = aug_full + kStages;          // [NQ] commit after S_h(j) (and P_h(j-1) V) -> softmax h
+    uint64_t* p_full = s_full + NQ;                 // [NQ] 128 softmax threads wrote P_h(j) -> MMA
+    uint64_t* o_full = p_full + NQ;                 // [NQ] commit after the last P_h V -> epilogue h
+    uint64_t* drain = o_full + NQ;                  // abort path
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    (void)kStages;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int per_tile = a.Hkv * a.pairs_per_group;
@@ -169,9 +197,8 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     const int rem = static_cast<int>(blockIdx.x % per_tile);
     const int kvh = rem / a.pairs_per_group;
     const int head0 = kvh * (a.Hq / a.Hkv) + (rem % a.pairs_per_group) * NQ;
-    // causal: key tiles 0..n_kv-1; the last kBM / kBN of them touch the diagonal
-    const int n_kv = static_cast<int>((static_cast<int64_t>(m_tile + 1) * kBM + kBN - 1) / kBN);
-    const int first_diag = (m_tile * kBM) / kBN;
+    // causal: key tiles 0..m_tile, the last one on the diagonal
+    const int n_kv = m_tile + 1;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -179,16 +206,13 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1);
-            mbar_init(&v_ready[s], 64);
             mbar_init(&v_empty[s], 1);
+            mbar_init(&aug_full[s], 32);
         }
         for (int h = 0; h < NQ; ++h) {
             mbar_init(&s_full[h], 1);
-            mbar_init(&s_empty[h], 128);
             mbar_init(&p_full[h], 128);
-            mbar_init(&pv_done[h], 1);
-            mbar_init(&bias_full[2 * h], 128);
-            mbar_init(&bias_full[2 * h + 1], 128);
+            mbar_init(&o_full[h], 1);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -200,6 +224,23 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
+    }
+    if (warp == 2) {
+        // A_h: every row holds gamma_h's parts (i = col / 3 for col < 9, zeros after)
+        uint4* aug_a = reinterpret_cast<uint4*>(smem + C::kOffAugA);
+#pragma unroll
+        for (int h = 0; h < NQ; ++h) {
+            __nv_bfloat16 g[3];
+            split3_bf16(a.gain ? a.gain[head0 + h] * kLog2e / a.scale_log2 : 0.0f, g);
+            const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
+            const uint4 c0 = make_uint4(bf2(g[0], g[0]), bf2(g[0], g[1]), bf2(g[1], g[1]), bf2(g[2], g[2]));
+            const uint4 c1 = make_uint4(bf2(g[2], z), 0u, 0u, 0u);
+            for (int r = lane; r < kBM; r += 32) {
+                aug_a[h * (C::kAugTile / 16) + aug_slot(r, 0)] = c0;
+                aug_a[h * (C::kAugTile / 16) + aug_slot(r, 1)] = c1;
+            }
+        }
+        fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads (after the sync below)
     }
     tc_fence_before();
     __syncthreads();
@@ -254,11 +295,6 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false);  // Q K^T: both K-major
             constexpr uint32_t idesc_o = idesc_f16_f32(kBM, D, true);      // P V: V MN-major
-            bool ok = mbar_wait(q_full, 0, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
-            auto wait_k = [&](int j) -> bool {
-                return mbar_wait(&k_full[j % kStages], static_cast<uint32_t>(j / kStages) & 1, abort_flag,
-                                 a.status, TG_STATUS_ATTENTION_TIMEOUT);
-            };
             // Descriptors as 32-bit start/LBO words over one shared high word (SBO 1024,
             // 128-byte swizzle): every MMA below moves its operands by compile-time
             // offsets, so the issuing thread keeps ahead of the tensor pipe.
@@ -266,7 +302,17 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             const uint32_t q_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffQ), 16);
             const uint32_t k_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffK), 16);
             const uint32_t v_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffV), kBN * 128);
-            // S_h = Q_h K_j^T into head h's S columns, then signal softmax h
+            const uint32_t ahi = noswz_desc_hi(256);
+            const uint32_t aa_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffAugA), 128);
+            const uint32_t ab_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffAugB), 128);
+            // K tile j and its bias operand B both in shared memory
+            auto wait_k = [&](int j) -> bool {
+                const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
+                return mbar_wait(&k_full[j % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT) &&
+                       mbar_wait(&aug_full[j % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
+            };
+            // S_h = Q_h K_j^T into head h's S columns, then signal softmax h (the commit
+            // also covers every earlier MMA of this thread, P_h(j-1) V_{j-1} included)
             auto issue_s = [&](int h, int j) {
                 const uint32_t q_lo = q_lo0 + static_cast<uint32_t>(h * (C::kQTile >> 4));
                 const uint32_t k_lo = k_lo0 + static_cast<uint32_t>((j % kStages) * (C::kKVTile >> 4));
@@ -277,50 +323,48 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                     const uint32_t ko = static_cast<uint32_t>(((k >> 2) * (kBN * 128) + (k & 3) * 32) >> 4);
                     mma_ss_lo(tmem + C::col_s(h), q_lo + qo, k_lo + ko, dhi, idesc_s, k > 0);
                 }
+                // + A_h B^T: the key bias g_h s_c / c, one more K step
+                mma_ss_lo(tmem + C::col_s(h), aa_lo0 + static_cast<uint32_t>(h * (C::kAugTile >> 4)),
+                          ab_lo0 + static_cast<uint32_t>((j % kStages) * (C::kAugTile >> 4)), ahi, idesc_s, 1u);
                 mma_commit(&s_full[h]);
             };
+            bool ok = mbar_wait(q_full, 0, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
             if (ok) ok = wait_k(0);
             if (ok) {
                 tc_fence_after();
+#pragma unroll
                 for (int h = 0; h < NQ; ++h) issue_s(h, 0);
                 mma_commit(&k_empty[0]);
             }
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int st = j % kStages;
-                // next S of each head as soon as its softmax has read the current one
-                if (j + 1 < n_kv) {
-                    if (!(ok = wait_k(j + 1))) break;
-#pragma unroll
-                    for (int h = 0; h < NQ && ok; ++h) {
-                        if (!(ok = mbar_wait(&s_empty[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status,
-                                             TG_STATUS_ATTENTION_TIMEOUT)))
-                            break;
-                        tc_fence_after();
-                        issue_s(h, j + 1);
-                    }
-                    if (!ok) break;
-                    mma_commit(&k_empty[(j + 1) % kStages]);
-                }
-                // P_h(j) V_j for each head once its softmax has written P_h(j)
-                if (!(ok = mbar_wait(&v_ready[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
+                const bool more = j + 1 < n_kv;
+                if (!(ok = mbar_wait(&v_full[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
                                      TG_STATUS_ATTENTION_TIMEOUT)))
                     break;
+                if (more && !(ok = wait_k(j + 1))) break;
                 const uint32_t v_lo = v_lo0 + static_cast<uint32_t>(st * (C::kKVTile >> 4));
 #pragma unroll
                 for (int h = 0; h < NQ && ok; ++h) {
+                    // O_h += P_h(j) V_j once softmax h has written P_h(j) ...
                     if (!(ok = mbar_wait(&p_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status,
                                          TG_STATUS_ATTENTION_TIMEOUT)))
                         break;
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < kBN / 16; ++k)  // 16 keys per step: 16 rows of 128 bytes in each chunk
-                        mma_ts_lo(tmem + C::col_o(h), tmem + C::col_p(h) + static_cast<uint32_t>(k * 8),
+                        mma_ts_lo(tmem + C::col_o(h), tmem + C::col_s(h) + static_cast<uint32_t>(k * 8),
                                   v_lo + static_cast<uint32_t>(k * (2048 >> 4)), dhi, idesc_o,
                                   (j > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(&pv_done[h]);
+                    // ... then, behind it in the same pipe, S_h(j+1) over the same columns
+                    if (more)
+                        issue_s(h, j + 1);
+                    else
+                        mma_commit(&o_full[h]);
                 }
                 if (!ok) break;
                 mma_commit(&v_empty[st]);
+                if (more) mma_commit(&k_empty[(j + 1) % kStages]);
             }
             if (!ok) {
                 mma_commit(drain);
@@ -328,90 +372,67 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 mbar_wait(drain, 0, &no_abort, a.status, TG_STATUS_ATTENTION_TIMEOUT);
             }
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ V tile -> fp16, in place
-        const int t = threadIdx.x - 64;
-        for (int j = 0; j < n_kv; ++j) {
-            const int st = j % kStages;
-            if (!mbar_wait(&v_full[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ bias operand B
+        // B for K tile jb: row c holds s_c's parts (k = col mod 3 for col < 9, zeros after)
+        uint4* aug_b = reinterpret_cast<uint4*>(smem + C::kOffAugB);
+        auto fill_aug = [&](int jb) -> bool {
+            const int st = jb % kStages;
+            // the slot is free once the S MMAs of tile jb - kStages are done (same release as K)
+            if (!mbar_wait(&k_empty[st], (static_cast<uint32_t>(jb / kStages) & 1) ^ 1, abort_flag, a.status,
                            TG_STATUS_ATTENTION_TIMEOUT))
-                break;
-            uint4* vt = reinterpret_cast<uint4*>(smem + C::kOffV + st * C::kKVTile);
-#pragma unroll 4
-            for (int i = t; i < C::kKVTile / 16; i += 64) {
-                uint4 x = vt[i];
-                uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                return false;
+            uint4* dst = aug_b + st * (C::kAugTile / 16);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    w[e] = f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
-                vt[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int i = 0; i < kBN / 32; ++i) {
+                const int c = i * 32 + lane;
+                const int64_t key = static_cast<int64_t>(jb) * kBN + c;
+                __nv_bfloat16 p[3];
+                split3_bf16((a.s_kept && key < a.K) ? a.s_kept[key] : 0.0f, p);
+                const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
+                dst[aug_slot(c, 0)] = make_uint4(bf2(p[0], p[1]), bf2(p[2], p[0]), bf2(p[1], p[2]), bf2(p[0], p[1]));
+                dst[aug_slot(c, 1)] = make_uint4(bf2(p[2], z), 0u, 0u, 0u);
             }
             fence_proxy_async_smem();  // generic-proxy writes -> tensor-core (async proxy) reads
-            mbar_arrive(&v_ready[st]);
-        }
+            mbar_arrive(&aug_full[st]);
+            return true;
+        };
+        for (int j = 0; j < n_kv; ++j)
+            if (!fill_aug(j)) break;
     } else {
         // ------------------------------------------------------------ softmax + epilogue of head h
-        const int h = (warp - 4) >> 2;
-        const int q = warp & 3;
+        const int sw = warp - C::kSoftmaxWarp0;
+        const int h = sw >> 2;
+        const int q = warp & 3;         // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;  // query row inside the tile == TMEM lane
-        const int t = threadIdx.x - 128 - 128 * h;
         const int head = head0 + h;
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + C::col_s(h);
-        const uint32_t p_addr = tmem + lane_off + C::col_p(h);
         const uint32_t o_addr = tmem + lane_off + C::col_o(h);
-        const float gain = a.gain ? a.gain[head] * kLog2e : 0.0f;
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-        float* bias_h = bias_s + h * 2 * kBN;
-        float s_pref = (a.s_kept && t < kBN && t < a.K) ? a.s_kept[t] : 0.0f;
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         for (int j = 0; j < n_kv && ok; ++j) {
-            const int b = j & 1;
-            // this tile's key bias g_h * s_c in log2 units (one key per thread), next tile's score prefetched
-            if (t < kBN) bias_h[b * kBN + t] = gain * s_pref;
-            mbar_arrive(&bias_full[2 * h + b]);
-            {
-                const int64_t cn = static_cast<int64_t>(j + 1) * kBN + t;
-                s_pref = (a.s_kept && t < kBN && j + 1 < n_kv && cn < a.K) ? a.s_kept[cn] : 0.0f;
-            }
-            if (!(ok = warp_wait(&bias_full[2 * h + b], static_cast<uint32_t>(j >> 1) & 1, abort_flag, a.status)))
-                break;
             if (!(ok = warp_wait(&s_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status))) break;
             tc_fence_after();
-            // the row's 64 S values, then hand the S columns back to the MMA warp
+            // the row's 128 S values (bias included)
             float x[kBN];
             {
                 uint32_t* xv = reinterpret_cast<uint32_t*>(x);
-                tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(xv));
-                tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(xv + 32));
+#pragma unroll
+                for (int c = 0; c < kBN; c += 32) tmem_ld32(s_addr + c, *reinterpret_cast<uint32_t(*)[32]>(xv + c));
                 tmem_ld_wait();
             }
-            tc_fence_before();
-            mbar_arrive(&s_empty[h]);
-            const float* bias = bias_h + b * kBN;
-            // keys c with j * kBN + c > m_tile * kBM + row are in the future of this query row
-            const int lim = m_tile * kBM + row - j * kBN;
-            const bool diag = j >= first_diag;
+            // on the diagonal tile, key c is in the future of query row r when c > r
+            if (j == n_kv - 1) {
+#pragma unroll
+                for (int c = 0; c < kBN; ++c)
+                    if (c > row) x[c] = -INFINITY;
+            }
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < kBN; c += 4) {
-                const float4 bb = *reinterpret_cast<const float4*>(bias + c);
-                float2 x0 = ffma2(make_float2(x[c], x[c + 1]), sc2, make_float2(bb.x, bb.y));
-                float2 x1 = ffma2(make_float2(x[c + 2], x[c + 3]), sc2, make_float2(bb.z, bb.w));
-                if (diag) {
-                    if (c > lim) x0.x = -INFINITY;
-                    if (c + 1 > lim) x0.y = -INFINITY;
-                    if (c + 2 > lim) x1.x = -INFINITY;
-                    if (c + 3 > lim) x1.y = -INFINITY;
-                }
-                x[c] = x0.x;
-                x[c + 1] = x0.y;
-                x[c + 2] = x1.x;
-                x[c + 3] = x1.y;
-                mx4[(c >> 2) & 3] = fmax3(mx4[(c >> 2) & 3], fmaxf(x0.x, x0.y), fmaxf(x1.x, x1.y));
-            }
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            for (int c = 0; c < kBN; c += 2) mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], x[c], x[c + 1]);
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
             // lazy rescaling: keep the stale max unless this row's max grew by more than 2^8
             const bool need = mx > m_run + kRescaleThreshold;
             float alpha = 1.0f;
@@ -420,23 +441,19 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 m_run = mx;
                 l_run *= alpha;
             }
-            // P_h(j-1) V_{j-1} must be complete before O is rescaled and P_h is overwritten
-            if (j > 0) {
-                if (!(ok = warp_wait(&pv_done[h], static_cast<uint32_t>(j - 1) & 1, abort_flag, a.status))) break;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, need)) {
+            // S_h(j) complete implies P_h(j-1) V_{j-1} complete: O_h may be rescaled now
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 16) {
-                        uint32_t v[16];
-                        tmem_ld16(o_addr + c0, v);
-                        tmem_ld_wait();
+                for (int c0 = 0; c0 < D; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(o_addr + c0, v);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                        tmem_st16(o_addr + c0, v);
-                    }
+                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                    tmem_st16(o_addr + c0, v);
                 }
             }
-            // P = 2^(x - m) as fp16 into P_h
+            // P = 2^(S c - m) as fp16 over the first kBN / 2 S columns (already read)
             const float2 neg_m = make_float2(-m_run, -m_run);
             float2 ls[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
@@ -444,8 +461,8 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 uint32_t p16[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 4) {
-                    const float2 y0 = fadd2(make_float2(x[c0 + i], x[c0 + i + 1]), neg_m);
-                    const float2 y1 = fadd2(make_float2(x[c0 + i + 2], x[c0 + i + 3]), neg_m);
+                    const float2 y0 = ffma2(make_float2(x[c0 + i], x[c0 + i + 1]), sc2, neg_m);
+                    const float2 y1 = ffma2(make_float2(x[c0 + i + 2], x[c0 + i + 3]), sc2, neg_m);
                     const float2 p0 = make_float2(ex2(y0.x), ex2(y0.y));
                     const float2 p1 = make_float2(ex2(y1.x), ex2(y1.y));
                     ls[0] = fadd2(ls[0], p0);
@@ -453,7 +470,7 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                     p16[i / 2] = f16x2(p0.x, p0.y);
                     p16[i / 2 + 1] = f16x2(p1.x, p1.y);
                 }
-                tmem_st16(p_addr + (c0 >> 1), p16);
+                tmem_st16(s_addr + (c0 >> 1), p16);
             }
             const float2 lsum = fadd2(ls[0], ls[1]);
             tmem_st_wait();
@@ -461,7 +478,7 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             tc_fence_before();
             mbar_arrive(&p_full[h]);
         }
-        if (ok && warp_wait(&pv_done[h], static_cast<uint32_t>(n_kv - 1) & 1, abort_flag, a.status)) {
+        if (ok && warp_wait(&o_full[h], 0, abort_flag, a.status)) {
             // epilogue: normalise, store bf16 rows and the log-sum-exp
             tc_fence_after();
             const int64_t grow = static_cast<int64_t>(m_tile) * kBM + row;
@@ -496,6 +513,21 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     }
 }
 
+// V [K, Hkv d_h] bf16 (token stride ld_v) -> dense fp16 [K, Hkv d_h], eight
+// elements per 16-byte load and store.
+__global__ void __launch_bounds__(128) v_to_f16_kernel(const uint4* __restrict__ v, int64_t ld_v8, int64_t K,
+                                                       int w8, uint4* __restrict__ v16) {
+    for (int64_t r = blockIdx.x; r < K; r += gridDim.x) {
+        for (int c = threadIdx.x; c < w8; c += blockDim.x) {
+            const uint4 x = v[r * ld_v8 + c];
+            uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w[e] = f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+            v16[r * w8 + c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
 template <int D, int NQ>
 static tg_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, Args a,
                         cudaStream_t st) {
@@ -520,17 +552,28 @@ extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg
                                         int32_t d_h, const float* s_kept, const float* gain, float tau,
                                         tg_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
                                         void* stream) {
-    if (K < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || !std::isfinite(tau)) return TG_ERR_INVALID_ARG;
+    if (K < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || !std::isfinite(tau) || !(tau > 0.0f))
+        return TG_ERR_INVALID_ARG;
     if (d_h != 64 && d_h != 128) return TG_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TG_ERR_INVALID_ARG;
     if (K == 0) return TG_OK;
     if (K > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
     if (!q || !k || !v || !out || !workspace || !aligned16(workspace)) return TG_ERR_INVALID_ARG;
-    if (workspace_bytes < tg_workspace_bytes(TG_OP_ATTENTION, K, 0, 0)) return TG_ERR_INVALID_ARG;
+    if (workspace_bytes < tg_workspace_bytes(TG_OP_ATTENTION, K, Hkv * d_h, 0)) return TG_ERR_INVALID_ARG;
     if (ld_q < static_cast<int64_t>(Hq) * d_h || ld_k < static_cast<int64_t>(Hkv) * d_h ||
         ld_v < static_cast<int64_t>(Hkv) * d_h || (ld_q % 8) || (ld_k % 8) || (ld_v % 8))
         return TG_ERR_INVALID_ARG;
 
+    // fp16 copy of V in the workspace, dense [K, Hkv, d_h]
+    void* v16 = static_cast<char*>(workspace) + ws_gate_offset();
+    cudaStream_t st = as_stream(stream);
+    {
+        const int w8 = Hkv * d_h / 8;
+        const int64_t grid = K < static_cast<int64_t>(num_sms()) * 16 ? K : static_cast<int64_t>(num_sms()) * 16;
+        attn::v_to_f16_kernel<<<static_cast<unsigned>(grid), 128, 0, st>>>(
+            reinterpret_cast<const uint4*>(v), ld_v / 8, K, w8, reinterpret_cast<uint4*>(v16));
+        if (launch_status() != TG_OK) return TG_ERR_CUDA;
+    }
     CUtensorMap mq, mk, mv;
     const uint32_t qbox[3] = {64, 1, 128};
     const uint32_t kvbox[3] = {64, 1, static_cast<uint32_t>(attn::kBN)};
@@ -542,8 +585,9 @@ extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg
     {
         const uint64_t dims[3] = {static_cast<uint64_t>(d_h), static_cast<uint64_t>(Hkv), static_cast<uint64_t>(K)};
         const uint64_t sk[2] = {static_cast<uint64_t>(d_h) * 2, static_cast<uint64_t>(ld_k) * 2};
-        const uint64_t sv[2] = {static_cast<uint64_t>(d_h) * 2, static_cast<uint64_t>(ld_v) * 2};
-        if (!make_tmap_bf16(&mk, k, 3, dims, sk, kvbox) || !make_tmap_bf16(&mv, v, 3, dims, sv, kvbox))
+        const uint64_t sv[2] = {static_cast<uint64_t>(d_h) * 2, static_cast<uint64_t>(Hkv) * d_h * 2};
+        // (the map's element type only matters for fills; the fp16 bits are copied as they are)
+        if (!make_tmap_bf16(&mk, k, 3, dims, sk, kvbox) || !make_tmap_bf16(&mv, v16, 3, dims, sv, kvbox))
             return TG_ERR_CUDA;
     }
     attn::Args a;
@@ -558,7 +602,6 @@ extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg
     a.out = reinterpret_cast<__nv_bfloat16*>(out);
     a.lse = lse;
     a.status = status_word(workspace);
-    cudaStream_t st = as_stream(stream);
     const bool pairs = ((Hq / Hkv) % 2) == 0;
     if (d_h == 128) return pairs ? attn::launch<128, 2>(mq, mk, mv, a, st) : attn::launch<128, 1>(mq, mk, mv, a, st);
     return pairs ? attn::launch<64, 2>(mq, mk, mv, a, st) : attn::launch<64, 1>(mq, mk, mv, a, st);

@@ -6,7 +6,9 @@
 //   [0, 256)                 status word (sticky TG_STATUS_* bits) + padding
 //   [256, 256 + S)           select scratch: grid-barrier counter, radix
 //                            histograms, per-block counts (self-cleaning)
-//   [256 + S', ...)          gate: bf16(rms_weight * W1) when rms_weight given
+//   [256 + S', ...)          gate: bf16(rms_weight * W1) when rms_weight given;
+//                            attention: fp16 copy of V (the two are rebuilt by
+//                            every call that uses them, so they may overlap)
 #include <cstdio>
 
 #include "tg_host.cuh"
@@ -38,13 +40,13 @@ extern "C" int64_t tg_kept_count(int64_t N, int64_t doc_begin, int64_t doc_end, 
 
 extern "C" size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g) {
     if (N < 0) return 0;
+    const size_t gate = (d > 0 && d_g > 0) ? static_cast<size_t>(d) * static_cast<size_t>(d_g) * 2 : 0;
+    const size_t attn = d > 0 ? static_cast<size_t>(N) * static_cast<size_t>(d) * 2 : 0;
     switch (op) {
         case TG_OP_SELECT: return kWsHeader + sizeof(SelectScratch);
-        case TG_OP_ATTENTION: return kWsHeader;
-        case TG_OP_GATE:
-        case TG_OP_ALL:
-            if (d <= 0 || d_g <= 0) return op == TG_OP_ALL ? ws_gate_offset() : 0;
-            return ws_gate_offset() + static_cast<size_t>(d) * static_cast<size_t>(d_g) * 2;
+        case TG_OP_ATTENTION: return d > 0 ? ws_gate_offset() + attn : 0;
+        case TG_OP_GATE: return gate ? ws_gate_offset() + gate : 0;
+        case TG_OP_ALL: return ws_gate_offset() + (gate > attn ? gate : attn);
     }
     return 0;
 }

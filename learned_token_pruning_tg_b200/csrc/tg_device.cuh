@@ -264,6 +264,13 @@ __device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t saddr, uint32_t lbo_b
     return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
 }
 
+// High word of a descriptor for the no-swizzle K-major layout: 8-row x 16-byte
+// core matrices stored whole (128 contiguous bytes), the next one along K at
+// LBO bytes (given in the low word), the next 8-row group at SBO bytes.
+__host__ __device__ constexpr uint32_t noswz_desc_hi(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulator.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),
 //   bit 15 A major (0 = K), bit 16 B major (0 = K, 1 = MN), bits 17-22 N >> 3,

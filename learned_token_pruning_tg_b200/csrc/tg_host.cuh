@@ -19,6 +19,10 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // Number of SMs of the current device (queried once per device).
+// Byte offset of the per-op region of a workspace (after the status header and
+// the select scratch); defined with the workspace sizing.
+size_t ws_gate_offset();
+
 inline int num_sms() {
     static int cache[64] = {0};
     int dev = 0;

@@ -49,7 +49,8 @@ class GatedPrefillLayer:
         self.WqkvT = Wqkv.to(dev, torch.bfloat16).t().contiguous()      # [d, (Hq + 2 Hkv) d_h]
         self.gain = gain.to(dev, torch.float32).contiguous()
         K, d = self.K, self.d
-        self.ws = tg.new_workspace(N, d, self.d_g, device=dev)
+        self.ws = tg.new_workspace(N, d, self.d_g, op=tg.TG_OP_GATE, device=dev)  # gate and select
+        self.ws_attn = tg.new_workspace(K, Hkv * d_h, op=tg.TG_OP_ATTENTION, device=dev)
         self.scores = torch.empty(N, dtype=torch.float32, device=dev)
         self.kept = torch.empty(max(K, 1), dtype=torch.int32, device=dev)
         self.h_kept = torch.empty(K, d, dtype=torch.bfloat16, device=dev)
@@ -79,8 +80,8 @@ class GatedPrefillLayer:
         m("rope")
         tg.tg_rope_apply(self.q, self.k, self.pos[:K], self.rope_base)
         m("attn")
-        tg.tg_gated_attention(self.q, self.k, self.v, self.out, self.ws, s_kept=self.s_kept[:K], gain=self.gain,
-                              tau=self.tau)
+        tg.tg_gated_attention(self.q, self.k, self.v, self.out, self.ws_attn, s_kept=self.s_kept[:K],
+                              gain=self.gain, tau=self.tau)
         m("end")
         return self.out, self.kept[:K]
 
@@ -95,5 +96,10 @@ class GatedPrefillLayer:
         return out_host, kept_host
 
     def launches_per_step(self) -> int:
-        """libtokengate kernels per run(): gate (+ the RMSNorm-weight fold), select, gather, rope, attention."""
-        return 5 + (1 if self.rms_weight is not None else 0)
+        """libtokengate kernels per run(): gate (+ the RMSNorm-weight fold), select, gather, rope, and the
+        attention's two (V to fp16, attention)."""
+        return 6 + (1 if self.rms_weight is not None else 0)
+
+    def device_status(self) -> int:
+        """OR of the status words of the layer's workspaces (synchronizes the stream); 0 = no timeout."""
+        return tg.tg_device_status(self.ws) | tg.tg_device_status(self.ws_attn)

@@ -55,6 +55,12 @@ def test_host_only_calls(lib):
     assert tg.tg_workspace_bytes(tg.TG_OP_GATE, 131072, 2048, 256) >= 2048 * 256 * 2
     assert tg.tg_workspace_bytes(tg.TG_OP_ALL, 131072, 2048, 256) >= tg.tg_workspace_bytes(tg.TG_OP_SELECT, 1)
     assert tg.tg_workspace_bytes(tg.TG_OP_GATE, -1, 2048, 256) == 0
+    # attention: N = K kept tokens, d = Hkv * d_h (an fp16 copy of V lives in the workspace)
+    attn = tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, 4608, 1024)
+    assert attn >= 4608 * 1024 * 2 and attn % 16 == 0
+    assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, 4608, 0) == 0
+    assert tg.tg_workspace_bytes(tg.TG_OP_ALL, 4608, 1024, 256) >= attn
+    assert tg.tg_workspace_bytes(tg.TG_OP_ALL, 4608, 1024, 256) >= tg.tg_workspace_bytes(tg.TG_OP_GATE, 4608, 1024, 256)
     assert tg.status_string(tg.TG_OK) == "ok"
     assert "timed out" in tg.status_string(tg.TG_ERR_TIMEOUT)
     assert tg.tg_version() >= 100
@@ -81,3 +87,8 @@ def test_argument_errors_before_launch(lib):
                                   vp(16), None, vp(256), 256, None) == tg.TG_ERR_UNSUPPORTED  # d_h = 96
     assert lib.tg_gated_attention(vp(17), 128, vp(16), 128, vp(16), 128, 5, 2, 2, 64, None, None, 1.0,
                                   vp(16), None, vp(256), 256, None) == tg.TG_ERR_INVALID_ARG  # misaligned
+    for tau in (0.0, -1.0, float("nan")):   # the temperature must be positive
+        assert lib.tg_gated_attention(vp(16), 128, vp(16), 128, vp(16), 128, 5, 2, 2, 64, None, None, tau,
+                                      vp(16), None, vp(256), 1 << 20, None) == tg.TG_ERR_INVALID_ARG
+    assert lib.tg_gated_attention(vp(16), 128, vp(16), 128, vp(16), 128, 5, 2, 2, 64, None, None, 1.0,
+                                  vp(16), None, vp(256), 256, None) == tg.TG_ERR_INVALID_ARG  # workspace too small
