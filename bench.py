@@ -359,6 +359,52 @@ def run_tokengate(args, rank, world, local_rank):
            "d2h_bytes_per_step": out_host.numel() * out_host.element_size() + kept_host.numel() * 4,
            "ms_per_step": e2e_ms}
 
+    # The same step captured once in a CUDA graph and replayed: no host launch cost in the timed
+    # region.  Every rank takes the same collective steps whether or not its capture works.
+    graph_ms, graph_err = -1.0, None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            layer.run(h)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            layer.run(h)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(K):
+            g.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        graph_ms = g0.elapsed_time(g1) / K
+        del g
+    except Exception as e:  # report, do not fail the run
+        graph_err = f"{type(e).__name__}: {e}"[:200]
+        torch.cuda.synchronize()
+    graph_failed = reduce_max(1.0 if graph_ms < 0 else 0.0, dev)
+    graph_ms = reduce_max(graph_ms, dev)
+    graph = ({"ms_per_step": graph_ms, "value": job_throughput(w.N, world, graph_ms), "unit": "tokens/s"}
+             if graph_failed == 0.0 else {"unavailable": graph_err or "capture failed on another rank"})
+
+    # The key bias's cost: the attention call with and without s' and g (the pages put it at <= 1.1x).
+    def time_attn(with_bias: bool, reps: int = 20) -> float:
+        kw = dict(s_kept=layer.s_kept[: layer.K], gain=layer.gain) if with_bias else {}
+        for _ in range(3):
+            tg.tg_gated_attention(layer.q, layer.k, layer.v, layer.out, layer.ws_attn, tau=layer.tau, **kw)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(reps):
+            tg.tg_gated_attention(layer.q, layer.k, layer.v, layer.out, layer.ws_attn, tau=layer.tau, **kw)
+        a1.record()
+        torch.cuda.synchronize()
+        return a0.elapsed_time(a1) / reps
+    t_bias, t_plain = time_attn(True), time_attn(False)
+
     if rank != 0:
         return None
 
@@ -389,6 +435,8 @@ def run_tokengate(args, rank, world, local_rank):
     t_path = sum(stage_ms[s] for s in path) * 1e-3
     path_roof = sum(lower_bound(s, tensor_peak) for s in path) / t_path
     path_roof_burst = sum(lower_bound(s, peaks["bf16_tflops"]) for s in path) / t_path
+    # against the nominal B200 figures (2.25 PFLOP/s dense bf16, 8 TB/s HBM3e), for context
+    path_roof_nominal = sum(max(work[s]["flops"] / 2.25e15, work[s]["bytes"] / 8.0e12) for s in path) / t_path
     kernels = {}
     for s in STAGES:
         sec_s = stage_ms[s] * 1e-3
@@ -410,6 +458,8 @@ def run_tokengate(args, rank, world, local_rank):
             "config": config_dict(w), "impl": "tokengate",
             "path_ms": t_path * 1e3, "path_tokens_per_s": w.N * world / t_path,
             "path_roofline_frac": path_roof, "path_roofline_frac_burst_peak": path_roof_burst,
+            "path_roofline_frac_nominal_peak": path_roof_nominal, "graph": graph,
+            "attention_bias_cost": {"with_bias_ms": t_bias, "without_bias_ms": t_plain, "ratio": t_bias / t_plain},
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": layer.launches_per_step() * K, "clocks": clk.summary(), "device_status": status,
             "peaks": peaks}

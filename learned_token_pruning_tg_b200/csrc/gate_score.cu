@@ -290,7 +290,8 @@ static tg_status launch(const CUtensorMap& mh, const CUtensorMap& mw, const Args
                         cudaStream_t st) {
     using C = Cfg<DG>;
     auto kern = gate_score_kernel<DG>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess)
+    static std::atomic<int> smem_set[64];  // zero before first use (static storage)
+    if (!set_max_dynamic_smem(kern, C::kSmem, smem_set))
         return TG_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(num_tiles, num_sms()));
     kern<<<grid, kThreads, C::kSmem, st>>>(mh, mw, a);

@@ -305,6 +305,7 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             const uint32_t ahi = noswz_desc_hi(256);
             const uint32_t aa_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffAugA), 128);
             const uint32_t ab_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffAugB), 128);
+            const bool bias = a.gain != nullptr && a.s_kept != nullptr;
             // K tile j and its bias operand B both in shared memory
             auto wait_k = [&](int j) -> bool {
                 const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
@@ -323,9 +324,10 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                     const uint32_t ko = static_cast<uint32_t>(((k >> 2) * (kBN * 128) + (k & 3) * 32) >> 4);
                     mma_ss_lo(tmem + C::col_s(h), q_lo + qo, k_lo + ko, dhi, idesc_s, k > 0);
                 }
-                // + A_h B^T: the key bias g_h s_c / c, one more K step
-                mma_ss_lo(tmem + C::col_s(h), aa_lo0 + static_cast<uint32_t>(h * (C::kAugTile >> 4)),
-                          ab_lo0 + static_cast<uint32_t>((j % kStages) * (C::kAugTile >> 4)), ahi, idesc_s, 1u);
+                // + A_h B^T: the key bias g_h s_c / c, one more K step (none without a bias)
+                if (bias)
+                    mma_ss_lo(tmem + C::col_s(h), aa_lo0 + static_cast<uint32_t>(h * (C::kAugTile >> 4)),
+                              ab_lo0 + static_cast<uint32_t>((j % kStages) * (C::kAugTile >> 4)), ahi, idesc_s, 1u);
                 mma_commit(&s_full[h]);
             };
             bool ok = mbar_wait(q_full, 0, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
@@ -533,7 +535,8 @@ static tg_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
                         cudaStream_t st) {
     using C = Cfg<D, NQ>;
     auto kern = gated_attention_kernel<D, NQ>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess)
+    static std::atomic<int> smem_set[64];  // zero before first use (static storage)
+    if (!set_max_dynamic_smem(kern, C::kSmem, smem_set))
         return TG_ERR_CUDA;
     a.pairs_per_group = (a.Hq / a.Hkv) / NQ;
     const int64_t grid = static_cast<int64_t>(a.num_q_tiles) * a.Hkv * a.pairs_per_group;

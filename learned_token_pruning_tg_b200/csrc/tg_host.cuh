@@ -3,6 +3,7 @@
 // encoding through the driver entry point (no link-time libcuda dependency).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <cuda.h>
@@ -18,15 +19,20 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-// Number of SMs of the current device (queried once per device).
 // Byte offset of the per-op region of a workspace (after the status header and
 // the select scratch); defined with the workspace sizing.
 size_t ws_gate_offset();
 
+inline int current_device() {
+    int dev = 0;
+    return (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) ? dev : -1;
+}
+
+// Number of SMs of the current device (queried once per device).
 inline int num_sms() {
     static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    const int dev = current_device();
+    if (dev < 0) return 148;
     if (cache[dev] == 0) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
@@ -47,11 +53,44 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// A tensor map is a pure function of its arguments, and encoding one costs
+// microseconds of host time per call; each host thread keeps its last few.
+struct TmapKey {
+    const void* base;
+    uint64_t dims[5], strides[4];
+    uint32_t box[5];
+    int32_t rank, promo;
+};
+struct TmapCache {
+    static constexpr int kEntries = 16;
+    TmapKey key[kEntries];
+    CUtensorMap map[kEntries];
+    bool used[kEntries] = {};
+    int next = 0;
+};
+
 // Tensor map over a bf16 tensor of `rank` dims (dims[0] innermost, in elements;
 // strides[i] in bytes for dims 1..rank-1), box `box` (elements), 128-byte swizzle.
 inline bool make_tmap_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                            const uint64_t* strides_bytes, const uint32_t* box,
                            CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
+    if (rank < 1 || rank > 5) return false;
+    TmapKey k;
+    std::memset(&k, 0, sizeof(k));  // padding too, so keys compare bytewise
+    k.base = base;
+    k.rank = rank;
+    k.promo = static_cast<int32_t>(promo);
+    for (int i = 0; i < rank; ++i) {
+        k.dims[i] = dims[i];
+        k.box[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides_bytes[i];
+    thread_local TmapCache cache;
+    for (int i = 0; i < TmapCache::kEntries; ++i)
+        if (cache.used[i] && std::memcmp(&cache.key[i], &k, sizeof(k)) == 0) {
+            *m = cache.map[i];
+            return true;
+        }
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t gdim[5];
@@ -67,7 +106,25 @@ inline bool make_tmap_bf16(CUtensorMap* m, const void* base, int rank, const uin
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
                     gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) return false;
+    const int slot = cache.next;
+    cache.next = (slot + 1) % TmapCache::kEntries;
+    cache.key[slot] = k;
+    cache.map[slot] = *m;
+    cache.used[slot] = true;
+    return true;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device;
+// `done` is a per-kernel array of 64 flags owned by the caller (a static in the
+// kernel's own launch function).
+template <typename Kernel>
+inline bool set_max_dynamic_smem(Kernel* kern, int bytes, std::atomic<int>* done) {
+    const int dev = current_device();
+    if (dev >= 0 && done[dev].load(std::memory_order_acquire) == bytes) return true;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    if (dev >= 0) done[dev].store(bytes, std::memory_order_release);
+    return true;
 }
 
 inline tg_status launch_status() {
