@@ -478,6 +478,59 @@ def run_tokengate(args, rank, world, local_rank):
             "peaks": peaks}
 
 
+def run_stack(args, rank, world, local_rank):
+    """The pruned prefill through a 28-layer stack at 64k (gate after layer 13, 8192 document tokens
+    kept) against the same stack with every token kept: device time per prefill and peak memory."""
+    from learned_token_pruning_tg_b200 import stack as stk
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = stk.STACK64K
+    wts = stk.random_weights(cfg, dev)
+    x = stk.random_embeddings(cfg, dev)
+    s = stk.PrunedPrefillStack(cfg, wts, device=dev)
+    reps = max(1, min(args.steps, 5))
+
+    def timed(prune: bool):
+        for _ in range(max(1, min(args.warmup, 2))):
+            s.run(x, prune=prune, keep_kv=True)
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            s.run(x, prune=prune, keep_kv=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        return reduce_max(e0.elapsed_time(e1) / reps, dev), peak, s.kv_bytes()
+
+    with ClockSampler(dev.index) as clk:
+        ms_pruned, mem_pruned, kv_pruned = timed(True)
+        ms_dense, mem_dense, kv_dense = timed(False)
+    status = s.device_status()
+    if rank != 0:
+        return None
+    return {"metric": f"prefill latency, {cfg.n_layers}-layer stack at {cfg.N // 1024}k (gate after layer "
+                      f"{cfg.gate_layer}, {cfg.k_doc} document tokens kept)",
+            "value": ms_pruned, "unit": "ms", "n_gpus": world, "steps": reps, "warmup": args.warmup,
+            "ms_per_step": ms_pruned, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded random weights and embeddings)",
+            "config": {"workload": cfg.name, "N": cfg.N, "doc_span": [cfg.doc_begin, cfg.doc_end],
+                       "k_doc": cfg.k_doc, "K": cfg.K, "layers": cfg.n_layers, "gate_layer": cfg.gate_layer,
+                       "d": cfg.d, "d_ff": cfg.d_ff, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d_h": cfg.d_h},
+            "impl": "tokengate",
+            "dense_ms": ms_dense, "speedup": ms_dense / ms_pruned,
+            "kv_cache_gb": {"pruned": kv_pruned / 1e9, "dense": kv_dense / 1e9},
+            "peak_memory_gb": {"pruned": mem_pruned / 1e9, "dense": mem_dense / 1e9,
+                               "note": "above the weights and inputs, KV cache included"},
+            "clocks": clk.summary(), "device_status": status}
+
+
 def main():
     faulthandler.enable()
     ap = argparse.ArgumentParser()
@@ -487,6 +540,8 @@ def main():
     ap.add_argument("--impl", choices=["tokengate", "reference"], default="tokengate")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--stack", action="store_true",
+                    help="time the pruned prefill through a 28-layer stack (and the unpruned one) instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -504,7 +559,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        res = run_tokengate(args, rank, world, local_rank)
+        res = (run_stack if args.stack else run_tokengate)(args, rank, world, local_rank)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:
