@@ -531,6 +531,95 @@ def run_stack(args, rank, world, local_rank):
             "clocks": clk.summary(), "device_status": status}
 
 
+def run_decode(args, rank, world, local_rank):
+    """One decoding step's attention over the KV cache a 28-layer 64k pruned prefill leaves (layers
+    up to the gate layer hold all N keys, the layers above the K kept keys with their scores; plus
+    the new token's own key), against the cache of the unpruned stack (N + 1 keys in every layer).
+    Each layer's cache is its own buffer (4.3 GB and 7.5 GB in all, far above L2), so every step
+    reads it from HBM; the 28 launches of a step are captured in one CUDA graph."""
+    from learned_token_pruning_tg_b200 import stack as stk
+    from learned_token_pruning_tg_b200 import tokengate as tg
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = stk.STACK64K
+    Hq, Hkv, d_h, L = cfg.Hq, cfg.Hkv, cfg.d_h, cfg.gate_layer
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(cfg.seed + 7 + rank)
+
+    def cache(T):
+        return (torch.randn(T, Hkv, d_h, generator=gen, device=dev, dtype=torch.bfloat16),
+                torch.randn(T, Hkv, d_h, generator=gen, device=dev, dtype=torch.bfloat16),
+                torch.randn(T, generator=gen, device=dev))
+
+    T_all, T_kept = cfg.N + 1, cfg.K + 1
+    pruned = [cache(T_all if li <= L else T_kept) for li in range(cfg.n_layers)]
+    dense = [cache(T_all) for _ in range(cfg.n_layers)]
+    q = torch.randn(Hq, d_h, generator=gen, device=dev, dtype=torch.bfloat16)
+    gain = 2.0 * torch.rand(Hq, generator=gen, device=dev)
+    out = torch.empty(Hq, d_h, dtype=torch.bfloat16, device=dev)
+    ws = tg.new_workspace(0, Hq, op=tg.TG_OP_DECODE, device=dev)
+
+    def step(layers, prune):
+        for li, (k, v, sc) in enumerate(layers):
+            if prune and li > L:
+                tg.tg_gated_decode(q, k, v, out, ws, s_cache=sc, gain=gain, tau=1.1)
+            else:
+                tg.tg_gated_decode(q, k, v, out, ws, tau=1.0)
+
+    def cache_bytes(layers, prune):
+        return sum(k.numel() * 2 * 2 + (sc.numel() * 4 if prune and li > L else 0)
+                   for li, (k, v, sc) in enumerate(layers))
+
+    reps = max(10, min(args.steps, 200))
+
+    def timed(layers, prune):
+        for _ in range(3):
+            step(layers, prune)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(layers, prune)
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        del g
+        return reduce_max(e0.elapsed_time(e1) / reps, dev)
+
+    with ClockSampler(dev.index) as clk:
+        ms_pruned = timed(pruned, True)
+        ms_dense = timed(dense, False)
+    status = tg.tg_device_status(ws)
+    if rank != 0:
+        return None
+    peaks = load_peaks()
+    b_pruned, b_dense = cache_bytes(pruned, True), cache_bytes(dense, False)
+    achieved = b_pruned / (ms_pruned * 1e-3) / 1e9
+    return {"metric": f"decode-step attention latency over the KV cache of a {cfg.n_layers}-layer {cfg.N // 1024}k "
+                      f"pruned prefill (gate after layer {cfg.gate_layer}, {cfg.k_doc} document tokens kept)",
+            "value": ms_pruned, "unit": "ms", "n_gpus": world, "steps": reps, "warmup": args.warmup,
+            "ms_per_step": ms_pruned, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded random caches)",
+            "config": {"workload": f"{cfg.name} decode", "layers": cfg.n_layers, "gate_layer": L,
+                       "keys_per_layer": {"up_to_gate": T_all, "above_gate": T_kept}, "Hq": Hq, "Hkv": Hkv,
+                       "d_h": d_h, "timing": "one CUDA graph of the 28 launches per step, replayed"},
+            "impl": "tokengate", "dense_ms": ms_dense, "speedup": ms_dense / ms_pruned,
+            "bytes_per_step": {"pruned": b_pruned, "dense": b_dense},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "gated_decode_kernel",
+                         "dense_frac": b_dense / (ms_dense * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "gpu_launches": cfg.n_layers * reps, "clocks": clk.summary(), "device_status": status}
+
+
 def main():
     faulthandler.enable()
     ap = argparse.ArgumentParser()
@@ -540,6 +629,8 @@ def main():
     ap.add_argument("--impl", choices=["tokengate", "reference"], default="tokengate")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--decode", action="store_true",
+                    help="time one decoding step's attention over a pruned 28-layer cache (and an unpruned one)")
     ap.add_argument("--stack", action="store_true",
                     help="time the pruned prefill through a 28-layer stack (and the unpruned one) instead")
     args = ap.parse_args()
@@ -559,7 +650,8 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        res = (run_stack if args.stack else run_tokengate)(args, rank, world, local_rank)
+        res = (run_stack if args.stack else run_decode if args.decode else run_tokengate)(args, rank, world,
+                                                                                        local_rank)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

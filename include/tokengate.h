@@ -69,7 +69,8 @@ typedef enum {
     TG_OP_GATE = 0,
     TG_OP_SELECT = 1,
     TG_OP_ATTENTION = 2,
-    TG_OP_ALL = 3 /* one buffer usable by every call */
+    TG_OP_ALL = 3, /* one buffer usable by every call above */
+    TG_OP_DECODE = 4
 } tg_op;
 
 /* Bits of the device status word (first 4 bytes of the workspace). */
@@ -95,6 +96,7 @@ int64_t tg_kept_count(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_d
  *                    token's V row; the workspace holds an fp16 copy of V)
  *   TG_OP_ALL        every op above with these N, d, d_g (attention over at
  *                    most N tokens whose V rows are at most d wide)
+ *   TG_OP_DECODE     tg_gated_decode with d = Hq query heads (N, d_g unused)
  * Returns 0 for bad arguments. */
 size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g);
 
@@ -199,6 +201,27 @@ tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, i
                              int32_t Hkv, int32_t d_h, const float* s_kept,
                              const float* gain, float tau, tg_bf16* out, float* lse,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* One decoding step of token-gated attention over a KV cache (the layers
+ * above the gate layer keep only the kept tokens' keys, each with its gate
+ * score as a logit bias; a new token's key carries its own score):
+ *   l_c = tau * (q_h . k_{c,kv(h)}) / sqrt(d_h) + gain_h * s_c,   c < T
+ *   out_h = sum_c softmax_c(l_c) v_{c,kv(h)},  kv(h) = h / (Hq / Hkv)
+ * The query attends to all T keys in the cache (the new token's own key is
+ * the last one), so there is no mask.
+ * q: [Hq, d_h] bf16 (one token, heads contiguous).  k_cache, v_cache:
+ * [T, Hkv, d_h] bf16 with token strides ld_k, ld_v (elements, multiples of
+ * d_h / 32).  s_cache: [T] fp32 or NULL (no bias); gain: [Hq] fp32 or NULL.
+ * out: [Hq, d_h] bf16.  lse: [Hq] fp32 natural-log sum of exp, or NULL.
+ * workspace: tg_workspace_bytes(TG_OP_DECODE, 0, Hq, 0) bytes, zero-filled
+ * once; concurrent calls must not share one.
+ * Supported: d_h in {64, 128}, Hq / Hkv in {1, 2, 4, 8}, Hkv <= 64, 1 <= T <
+ * 2^31; q, k_cache, v_cache aligned to d_h / 16 bytes.  One launch; every
+ * cache row is read once (HBM-bound), fp32 softmax and accumulation. */
+tg_status tg_gated_decode(const tg_bf16* q, const tg_bf16* k_cache, int64_t ld_k, const tg_bf16* v_cache,
+                          int64_t ld_v, int64_t T, int32_t Hq, int32_t Hkv, int32_t d_h,
+                          const float* s_cache, const float* gain, float tau, tg_bf16* out, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* Reads the workspace's status word after synchronizing `stream`.
  * *status_word receives the raw TG_STATUS_* bits (may be NULL).

@@ -15,6 +15,7 @@
 
 namespace tg {
 size_t ws_gate_offset() { return kWsHeader + ((sizeof(SelectScratch) + 255) / 256) * 256; }
+size_t ws_decode_bytes(int32_t Hq);  // gated_decode.cu
 }  // namespace tg
 
 using namespace tg;
@@ -47,6 +48,7 @@ extern "C" size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g
         case TG_OP_ATTENTION: return d > 0 ? ws_gate_offset() + attn : 0;
         case TG_OP_GATE: return gate ? ws_gate_offset() + gate : 0;
         case TG_OP_ALL: return ws_gate_offset() + (gate > attn ? gate : attn);
+        case TG_OP_DECODE: return (d > 0 && d <= 512) ? ws_decode_bytes(d) : 0;
     }
     return 0;
 }

@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtokengate.so")
 
 TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_CUDA, TG_ERR_TIMEOUT = range(5)
-TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL = range(4)
+TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL, TG_OP_DECODE = range(5)
 
 _lib = None
 
@@ -52,9 +52,10 @@ def lib() -> ctypes.CDLL:
         L.tg_rope_apply.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, f64, vp]
         L.tg_gated_attention.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp,
                                          vp, sz, vp]
+        L.tg_gated_decode.argtypes = [vp, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp, vp, sz, vp]
         L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
         for fn in ("tg_gate_score", "tg_topk_select", "tg_topk_select_noalloc", "tg_gather_compact", "tg_rope_apply",
-                   "tg_gated_attention", "tg_device_status"):
+                   "tg_gated_attention", "tg_gated_decode", "tg_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -218,6 +219,30 @@ def tg_gated_attention(q, k, v, out, workspace, s_kept=None, gain=None, tau: flo
     _check("tg_gated_attention", lib().tg_gated_attention(
         _ptr(q), _row_stride(q, "q"), _ptr(k), _row_stride(k, "k"), _ptr(v), _row_stride(v, "v"), K, Hq, Hkv,
         d_h, _ptr(s_kept), _ptr(gain), tau, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return out
+
+
+def tg_gated_decode(q, k_cache, v_cache, out, workspace, s_cache=None, gain=None, tau: float = 1.0, lse=None,
+                    stream=None):
+    """One decoding step: q [Hq, d_h] over the T rows of k_cache, v_cache [T, Hkv, d_h] (token stride
+    may be padded); out [Hq, d_h]."""
+    _req(q, "q", torch.bfloat16, 2)
+    _req(k_cache, "k_cache", torch.bfloat16, 3)
+    _req(v_cache, "v_cache", torch.bfloat16, 3)
+    _req(out, "out", torch.bfloat16, 2)
+    _req(s_cache, "s_cache", torch.float32, 1)
+    _req(gain, "gain", torch.float32, 1)
+    _req(lse, "lse", torch.float32, 1)
+    Hq, d_h = q.shape
+    T, Hkv = k_cache.shape[0], k_cache.shape[1]
+    if not q.is_contiguous() or not out.is_contiguous() or out.shape != q.shape:
+        raise ValueError("q and out must be contiguous [Hq, d_h] tensors")
+    if v_cache.shape != k_cache.shape or (s_cache is not None and s_cache.shape[0] < T):
+        raise ValueError("shape mismatch")
+    _check("tg_gated_decode", lib().tg_gated_decode(
+        _ptr(q), _ptr(k_cache), _row_stride(k_cache, "k_cache"), _ptr(v_cache), _row_stride(v_cache, "v_cache"), T,
+        Hq, Hkv, d_h, _ptr(s_cache), _ptr(gain), tau, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)))
     return out
 

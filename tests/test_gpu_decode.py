@@ -1,0 +1,97 @@
+"""GPU parity of tg_gated_decode (one decoding step over a KV cache) against the oracle.
+
+The decoding query is the last row of a sequence whose first T rows are the
+cache, so the oracle's gated attention of row T-1 (which sees every key c <= T-1)
+is the exact answer.  The decode kernel keeps P in fp32 (no rounding before the
+P V product), so besides the specification's 1e-2 (over the output's own bf16
+rounding) the tests hold a derived 1e-3: fp32 accumulation over T <= 65537 keys
+and ex2.approx (relative error ~2^-22) stay far below it.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from learned_token_pruning_tg_b200 import synth
+from learned_token_pruning_tg_b200 import tokengate as tg
+
+pytestmark = pytest.mark.gpu
+
+SPEC_TOL = 1e-2
+DERIVED_TOL = 1e-3
+LSE_TOL = 1e-4
+
+
+def half_ulp_bf16(x):
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - 8), 0.0)
+
+
+def run_decode(d, strided=False, use_bias=True):
+    T, Hq, d_h = d.q.shape
+    Hkv = d.k.shape[1]
+    q = d.q[T - 1].contiguous().cuda()
+    if strided:
+        buf = torch.cat([d.k.reshape(T, -1), d.v.reshape(T, -1), torch.zeros(T, 8, dtype=torch.bfloat16)], 1).cuda()
+        k = buf[:, : Hkv * d_h].view(T, Hkv, d_h)
+        v = buf[:, Hkv * d_h: 2 * Hkv * d_h].view(T, Hkv, d_h)
+    else:
+        k, v = d.k.cuda(), d.v.cuda()
+    out = torch.full((Hq, d_h), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((Hq,), float("nan"), device="cuda")
+    ws = tg.new_workspace(0, Hq, op=tg.TG_OP_DECODE)
+    tg.tg_gated_decode(q, k, v, out, ws, s_cache=d.s.cuda() if use_bias else None,
+                       gain=d.gain.cuda() if use_bias else None, tau=d.tau, lse=lse)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def check(d, strided=False, use_bias=True):
+    T = d.q.shape[0]
+    got, lse = run_decode(d, strided, use_bias)
+    q, k, v = (t.float().numpy() for t in (d.q, d.k, d.v))
+    s = d.s.numpy() if use_bias else None
+    g = d.gain.numpy() if use_bias else None
+    want, want_lse = oracle.gated_attention(q, k, v, s=s, g=g, tau=d.tau, rows=[T - 1], want_lse=True)
+    want, want_lse = want[0], want_lse[0]
+    assert np.all(np.isfinite(got))
+    excess = np.abs(got - want) - half_ulp_bf16(want)
+    assert np.max(excess) <= SPEC_TOL
+    assert np.max(excess) <= DERIVED_TOL, np.max(excess)
+    assert np.max(np.abs(lse - want_lse)) <= LSE_TOL
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,d_h", [
+    (1, 2, 1, 128),          # a single key: out = v_0
+    (5, 16, 8, 128),
+    (300, 8, 8, 64),         # G = 1
+    (777, 16, 8, 128),       # G = 2, ragged splits
+    (1031, 16, 4, 64),       # G = 4
+    (2049, 32, 4, 128),      # G = 8
+    (8705, 16, 8, 128),      # the pruned stack's cache above the gate layer (+ the new token)
+    (65537, 16, 8, 128),     # the dense cache at 64k (+ the new token)
+])
+def test_decode_parity(T, Hq, Hkv, d_h):
+    check(synth.qkv(T, Hq, Hkv, d_h, seed=T + 31 * Hq + d_h))
+
+
+def test_decode_strided_cache_and_no_bias():
+    d = synth.qkv(1500, 16, 8, 128, seed=7)
+    check(d, strided=True)
+    check(d, use_bias=False)
+
+
+def test_decode_single_key_is_v0():
+    d = synth.qkv(1, 4, 2, 64, seed=3)
+    got, _ = run_decode(d)
+    want = np.repeat(d.v[0].float().numpy(), 2, axis=0)
+    assert np.array_equal(got, want)
+
+
+def test_decode_repeatable_bit_exact():
+    d = synth.qkv(8705, 16, 8, 128, seed=99)
+    a, la = run_decode(d)
+    for _ in range(3):
+        b, lb = run_decode(d)
+        assert np.array_equal(a, b) and np.array_equal(la, lb)
