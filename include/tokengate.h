@@ -211,13 +211,13 @@ tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, i
  * the last one), so there is no mask.
  * q: [Hq, d_h] bf16 (one token, heads contiguous).  k_cache, v_cache:
  * [T, Hkv, d_h] bf16 with token strides ld_k, ld_v (elements, multiples of
- * d_h / 32).  s_cache: [T] fp32 or NULL (no bias); gain: [Hq] fp32 or NULL.
+ * 8).  s_cache: [T] fp32 or NULL (no bias); gain: [Hq] fp32 or NULL.
  * out: [Hq, d_h] bf16.  lse: [Hq] fp32 natural-log sum of exp, or NULL.
  * workspace: tg_workspace_bytes(TG_OP_DECODE, 0, Hq, 0) bytes, zero-filled
  * once; concurrent calls must not share one.
  * Supported: d_h in {64, 128}, Hq / Hkv in {1, 2, 4, 8}, Hkv <= 64, 1 <= T <
- * 2^31; q, k_cache, v_cache aligned to d_h / 16 bytes.  One launch; every
- * cache row is read once (HBM-bound), fp32 softmax and accumulation. */
+ * 2^31; k_cache, v_cache 16-byte aligned, q 8-byte aligned.  One launch;
+ * every cache row is read once (HBM-bound), fp32 softmax and accumulation. */
 tg_status tg_gated_decode(const tg_bf16* q, const tg_bf16* k_cache, int64_t ld_k, const tg_bf16* v_cache,
                           int64_t ld_v, int64_t T, int32_t Hq, int32_t Hkv, int32_t d_h,
                           const float* s_cache, const float* gain, float tau, tg_bf16* out, float* lse,

@@ -13,13 +13,16 @@
 // Kernel: grid (Hkv, splits), 8 warps per CTA.  A CTA owns one KV head (and
 // the G = Hq / Hkv query heads that read it) and one contiguous range of keys.
 // Its key range streams through a 4-stage ring in shared memory (64 keys' K
-// and V rows a stage, copied with cp.async by all threads: 128 KB in flight
-// per CTA for d_h = 128, as HBM latency needs; one wave of CTAs).  Lane l
-// holds elements [E l, E l + E) of every query head (E = d_h / 32, scaled by
-// tau / sqrt(d_h) log2(e)); warp w takes 8 of a stage's keys, reads each K and
-// V row from shared memory (one conflict-free line), reduces the G partial
-// dot products with xor shuffles, and keeps an fp32 online softmax (running
-// max, sum, and E output elements per lane and head).  The warps' states
+// and V rows a stage, copied with cp.async by all threads, each thread always
+// the same row pieces: 128 KB in flight per CTA for d_h = 128, as HBM latency
+// needs; one wave of CTAs).  A key is handled by a group of LPK lanes (8 for
+// G <= 2, 16 for G = 4, 32 for G = 8, which keeps the registers per lane
+// about the same): each lane holds d_h / LPK elements of every query head
+// (scaled by tau / sqrt(d_h) log2(e)) and of the output, reads its piece of the
+// K and V rows from shared memory, and the group reduces the G partial dot
+// products with log2(LPK) xor shuffles.  Every lane group keeps its own fp32
+// online softmax (running max, sum, output piece) over the keys it sees; the
+// groups of a warp merge by shuffles at the end, then the warps' states
 // are merged in shared memory, the CTA writes (m, l, o) to the workspace, and
 // the last CTA of the KV head (a counter in the workspace, reset by that CTA)
 // merges all splits and writes out (bf16) and the log-sum-exp.  No thread
@@ -96,56 +99,76 @@ __device__ __forceinline__ void widen(const typename Piece<E>::T& u, float (&f)[
     }
 }
 
+// Lanes that share one key: fewer lanes (fewer shuffles per key) when few query
+// heads read the KV head, at most d_h / 4 so that a lane holds whole 8-byte pieces.
+template <int D, int G>
+struct Lanes {
+    static constexpr int kByG = G <= 2 ? 8 : (G == 4 ? 16 : 32);
+    static constexpr int kPerKey = kByG < D / 4 ? kByG : D / 4;
+};
+
 template <int D, int G>
 __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a) {
-    constexpr int E = D / 32;
+    constexpr int LPK = Lanes<D, G>::kPerKey;
+    constexpr int ED = D / LPK;          // elements per lane (multiple of 4)
+    static_assert(ED % 4 == 0, "a lane holds whole 8-byte pieces");
+    constexpr int KPS = 32 / LPK;        // keys a warp handles at once
     __shared__ float s_m[kWarps][G], s_l[kWarps][G];
     __shared__ float s_o[kWarps][G][D];
     __shared__ bool s_last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = lane / LPK, sub = lane % LPK;
     const int kvh = blockIdx.x, split = blockIdx.y;
     const int64_t c_begin = static_cast<int64_t>(split) * a.split_len;
     const int64_t c_end = min(c_begin + a.split_len, a.T);
 
-    float qr[G][E], gl2[G];
+    float qr[G][ED], gl2[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         const int head = kvh * G + g;
-        float f[E];
-        load_row<E>(a.q + static_cast<int64_t>(head) * D + lane * E, f);
 #pragma unroll
-        for (int e = 0; e < E; ++e) qr[g][e] = f[e] * a.scale_log2;
+        for (int e = 0; e < ED; e += 4) {
+            float f[4];
+            load_row<4>(a.q + static_cast<int64_t>(head) * D + sub * ED + e, f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) qr[g][e + i] = f[i] * a.scale_log2;
+        }
         gl2[g] = a.gain ? a.gain[head] * kLog2e : 0.0f;
     }
-    float m[G], l[G], o[G][E];
+    float m[G], l[G], o[G][ED];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         m[g] = -INFINITY;
         l[g] = 0.0f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[g][e] = 0.0f;
+        for (int e = 0; e < ED; ++e) o[g][e] = 0.0f;
     }
 
-    using PT = typename Piece<E>::T;
     constexpr int kRow = D * 2;                        // bytes of one key's row (one head)
     constexpr int kStageBytes = kStageKeys * kRow * 2;  // K rows, then V rows
-    constexpr int kPieces = kStageKeys * kRow / 16;     // 16-byte copies per matrix and stage
+    constexpr int kPiecesPerRow = kRow / 16;
+    constexpr int kRowsPerPass = kWarps * 32 / kPiecesPerRow;
+    constexpr int kPasses = kStageKeys / kRowsPerPass;
     extern __shared__ __align__(16) uint8_t ring[];
-    const char* kg = reinterpret_cast<const char*>(a.k + static_cast<int64_t>(kvh) * D);
-    const char* vg = reinterpret_cast<const char*>(a.v + static_cast<int64_t>(kvh) * D);
-    const int64_t n_keys = c_end - c_begin;
-    const int n_stages = static_cast<int>((n_keys + kStageKeys - 1) / kStageKeys);
-    // copy stage t's rows into ring slot t mod kRing (keys past the range are not copied)
+    const int n_keys = static_cast<int>(c_end - c_begin);
+    const int n_stages = (n_keys + kStageKeys - 1) / kStageKeys;
+    // this thread always copies piece `cp_piece` of rows cp_row + kRowsPerPass j of K and of V
+    const int cp_piece = threadIdx.x % kPiecesPerRow, cp_row = threadIdx.x / kPiecesPerRow;
+    const char* kg = reinterpret_cast<const char*>(a.k + static_cast<int64_t>(kvh) * D) + cp_piece * 16;
+    const char* vg = reinterpret_cast<const char*>(a.v + static_cast<int64_t>(kvh) * D) + cp_piece * 16;
+    const int64_t ldk2 = a.ld_k * 2, ldv2 = a.ld_v * 2;
     auto issue = [&](int t) {
-        uint8_t* slot = ring + (t % kRing) * kStageBytes;
-        for (int i = threadIdx.x; i < 2 * kPieces; i += kWarps * 32) {
-            const int mat = i / kPieces, rem = i % kPieces;
-            const int r = rem / (kRow / 16), piece = rem % (kRow / 16);
+        uint8_t* slot = ring + (t % kRing) * kStageBytes + cp_row * kRow + cp_piece * 16;
+#pragma unroll
+        for (int j = 0; j < kPasses; ++j) {
+            const int r = cp_row + j * kRowsPerPass;
             const int64_t c = c_begin + static_cast<int64_t>(t) * kStageKeys + r;
             if (c < c_end) {
-                const char* src = (mat ? vg + c * a.ld_v * 2 : kg + c * a.ld_k * 2) + piece * 16;
-                const uint32_t dst = smem_u32(slot + mat * (kStageKeys * kRow) + r * kRow + piece * 16);
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+                const uint32_t dk = smem_u32(slot + j * kRowsPerPass * kRow);
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dk), "l"(kg + c * ldk2) : "memory");
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dk + kStageKeys * kRow),
+                             "l"(vg + c * ldv2)
+                             : "memory");
             }
         }
     };
@@ -159,54 +182,71 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
         asm volatile("cp.async.wait_group %0;" ::"n"(kRing - 1) : "memory");  // stage t has landed (own copies)
         __syncthreads();                                                      // ... and everyone's
         const uint8_t* slot = ring + (t % kRing) * kStageBytes;
-        const int64_t c0 = c_begin + static_cast<int64_t>(t) * kStageKeys + warp * kUnroll;
-        float kf[kUnroll][E], vf[kUnroll][E], sr[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int r = warp * kUnroll + u;
-            if (c0 + u < c_end) {
-                widen<E>(*reinterpret_cast<const PT*>(slot + r * kRow + lane * E * 2), kf[u]);
-                widen<E>(*reinterpret_cast<const PT*>(slot + kStageKeys * kRow + r * kRow + lane * E * 2), vf[u]);
-                sr[u] = a.s ? __ldg(a.s + c0 + u) : 0.0f;
-            } else {  // past the range: the slot holds no row here (weight 0, and no NaN from stale bits)
+        for (int step = 0; step < kUnroll / KPS; ++step) {
+            // this lane group's key of the step
+            const int r = warp * kUnroll + step * KPS + grp;
+            const int64_t c = c_begin + static_cast<int64_t>(t) * kStageKeys + r;
+            const bool valid = c < c_end;
+            float kf[ED], vf[ED];
 #pragma unroll
-                for (int e = 0; e < E; ++e) kf[u][e] = vf[u][e] = 0.0f;
-                sr[u] = 0.0f;
+            for (int e = 0; e < ED; e += 4) {
+                if (valid) {
+                    widen<4>(*reinterpret_cast<const uint2*>(slot + r * kRow + (sub * ED + e) * 2),
+                             *reinterpret_cast<float(*)[4]>(kf + e));
+                    widen<4>(*reinterpret_cast<const uint2*>(slot + kStageKeys * kRow + r * kRow + (sub * ED + e) * 2),
+                             *reinterpret_cast<float(*)[4]>(vf + e));
+                } else {  // past the range: no row here (weight 0, and no NaN from stale bits)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) kf[e + i] = vf[e + i] = 0.0f;
+                }
             }
-        }
+            const float sb = (valid && a.s) ? __ldg(a.s + c) : 0.0f;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float x[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
+            for (int g = 0; g < G; ++g) {
                 float d = 0.0f;
 #pragma unroll
-                for (int e = 0; e < E; ++e) d = fmaf(qr[g][e], kf[u][e], d);
+                for (int e = 0; e < ED; ++e) d = fmaf(qr[g][e], kf[e], d);
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-                x[u] = (c0 + u < c_end) ? d + gl2[g] * sr[u] : -INFINITY;
-            }
-            float mx = m[g];
+                for (int off = LPK / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+                if (!valid) continue;  // uniform over the lane group
+                const float x = d + gl2[g] * sb;
+                if (x > m[g]) {        // new running max for this group (rescale its state)
+                    const float alpha = ex2(m[g] - x);
+                    m[g] = x;
+                    l[g] *= alpha;
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) mx = fmaxf(mx, x[u]);
-            if (mx == -INFINITY) continue;  // no key in this warp's share (uniform over the warp)
-            const float alpha = ex2(m[g] - mx);
-            m[g] = mx;
-            l[g] *= alpha;
-#pragma unroll
-            for (int e = 0; e < E; ++e) o[g][e] *= alpha;
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const float p = ex2(x[u] - mx);
+                    for (int e = 0; e < ED; ++e) o[g][e] *= alpha;
+                }
+                const float p = ex2(x - m[g]);
                 l[g] += p;
 #pragma unroll
-                for (int e = 0; e < E; ++e) o[g][e] = fmaf(p, vf[u][e], o[g][e]);
+                for (int e = 0; e < ED; ++e) o[g][e] = fmaf(p, vf[e], o[g][e]);
             }
         }
         __syncthreads();  // the slot is refilled by the next iteration's copies
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
+    // merge the lane groups of each warp (lanes sub, sub + LPK, ... hold the same output piece)
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int off = LPK; off < 32; off <<= 1) {
+            const float mo = __shfl_xor_sync(0xffffffffu, m[g], off);
+            const float lo = __shfl_xor_sync(0xffffffffu, l[g], off);
+            const float mx = fmaxf(m[g], mo);
+            const float fa = m[g] == -INFINITY ? 0.0f : ex2(m[g] - mx);
+            const float fb = mo == -INFINITY ? 0.0f : ex2(mo - mx);
+            l[g] = l[g] * fa + lo * fb;
+#pragma unroll
+            for (int e = 0; e < ED; ++e) {
+                const float oo = __shfl_xor_sync(0xffffffffu, o[g][e], off);
+                o[g][e] = o[g][e] * fa + oo * fb;
+            }
+            m[g] = mx;
+        }
+    }
     // merge the warps' states
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -214,8 +254,10 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
             s_m[warp][g] = m[g];
             s_l[warp][g] = l[g];
         }
+        if (grp == 0) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) s_o[warp][g][lane * E + e] = o[g][e];
+            for (int e = 0; e < ED; ++e) s_o[warp][g][sub * ED + e] = o[g][e];
+        }
     }
     __syncthreads();
     for (int i = threadIdx.x; i < G * D; i += kWarps * 32) {
@@ -334,9 +376,9 @@ extern "C" tg_status tg_gated_decode(const tg_bf16* q, const tg_bf16* k_cache, i
     if (G != 1 && G != 2 && G != 4 && G != 8) return TG_ERR_UNSUPPORTED;
     if (Hkv > 64 || T > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
     if (!aligned16(workspace) || workspace_bytes < ws_decode_bytes(Hq)) return TG_ERR_INVALID_ARG;
-    // 16-byte copies of cache rows; q read in d_h / 16-byte pieces
+    // 16-byte copies of cache rows; q read in 8-byte pieces
     if (!aligned16(k_cache) || !aligned16(v_cache) || (ld_k % 8) != 0 || (ld_v % 8) != 0 ||
-        reinterpret_cast<uintptr_t>(q) % (d_h / 16) != 0)
+        reinterpret_cast<uintptr_t>(q) % 8 != 0)
         return TG_ERR_INVALID_ARG;
     if (ld_k < static_cast<int64_t>(Hkv) * d_h || ld_v < static_cast<int64_t>(Hkv) * d_h) return TG_ERR_INVALID_ARG;
 
