@@ -620,6 +620,52 @@ def run_decode(args, rank, world, local_rank):
             "gpu_launches": cfg.n_layers * reps, "clocks": clk.summary(), "device_status": status}
 
 
+def run_decode_layer(args, rank, world, local_rank):
+    """One layer's decoding-step attention over a 64k cache (65,537 keys x 8 KV heads x 128, K and V
+    268 MB, above L2): the single launch the decode kernel's ncu summary captures."""
+    from learned_token_pruning_tg_b200 import stack as stk
+    from learned_token_pruning_tg_b200 import tokengate as tg
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = stk.STACK64K
+    T = cfg.N + 1
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(cfg.seed + 11 + rank)
+    k = torch.randn(T, cfg.Hkv, cfg.d_h, generator=gen, device=dev, dtype=torch.bfloat16)
+    v = torch.randn(T, cfg.Hkv, cfg.d_h, generator=gen, device=dev, dtype=torch.bfloat16)
+    s = torch.randn(T, generator=gen, device=dev)
+    q = torch.randn(cfg.Hq, cfg.d_h, generator=gen, device=dev, dtype=torch.bfloat16)
+    gain = 2.0 * torch.rand(cfg.Hq, generator=gen, device=dev)
+    out = torch.empty(cfg.Hq, cfg.d_h, dtype=torch.bfloat16, device=dev)
+    ws = tg.new_workspace(0, cfg.Hq, op=tg.TG_OP_DECODE, device=dev)
+    for _ in range(max(3, args.warmup)):
+        tg.tg_gated_decode(q, k, v, out, ws, s_cache=s, gain=gain, tau=1.1)
+    torch.cuda.synchronize()
+    reps = max(3, min(args.steps, 100))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        tg.tg_gated_decode(q, k, v, out, ws, s_cache=s, gain=gain, tau=1.1)
+    e1.record()
+    torch.cuda.synchronize()
+    us = reduce_max(e0.elapsed_time(e1) / reps * 1e3, dev)
+    if rank != 0:
+        return None
+    nbytes = 2 * k.numel() * 2 + s.numel() * 4
+    peaks = load_peaks()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"metric": "one layer's decoding-step attention over a 64k KV cache", "value": us, "unit": "us",
+            "n_gpus": world, "steps": reps, "warmup": args.warmup, "ms_per_step": us / 1e3,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random cache)",
+            "config": {"workload": "qwen3-1.7b 64k layer cache", "T": T, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d_h": cfg.d_h,
+                       "l2": "cache 268 MB > L2, no flush"},
+            "impl": "tokengate",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "gated_decode_kernel"},
+            "gpu_launches": reps, "device_status": tg.tg_device_status(ws)}
+
+
 def main():
     faulthandler.enable()
     ap = argparse.ArgumentParser()
@@ -629,6 +675,8 @@ def main():
     ap.add_argument("--impl", choices=["tokengate", "reference"], default="tokengate")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--decode-layer", action="store_true",
+                    help="time one layer's decoding step over a 64k cache (the decode kernel alone)")
     ap.add_argument("--decode", action="store_true",
                     help="time one decoding step's attention over a pruned 28-layer cache (and an unpruned one)")
     ap.add_argument("--stack", action="store_true",
@@ -650,8 +698,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        res = (run_stack if args.stack else run_decode if args.decode else run_tokengate)(args, rank, world,
-                                                                                        local_rank)
+        run = (run_stack if args.stack else run_decode if args.decode else
+               run_decode_layer if args.decode_layer else run_tokengate)
+        res = run(args, rank, world, local_rank)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

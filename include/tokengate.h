@@ -77,6 +77,7 @@ typedef enum {
 #define TG_STATUS_SELECT_TIMEOUT 0x1u
 #define TG_STATUS_GATE_TIMEOUT 0x2u
 #define TG_STATUS_ATTENTION_TIMEOUT 0x4u
+#define TG_STATUS_DECODE_TIMEOUT 0x8u
 
 /* Static description of a status code.  Never NULL. */
 const char* tg_status_string(tg_status status);
@@ -216,8 +217,10 @@ tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, i
  * workspace: tg_workspace_bytes(TG_OP_DECODE, 0, Hq, 0) bytes, zero-filled
  * once; concurrent calls must not share one.
  * Supported: d_h in {64, 128}, Hq / Hkv in {1, 2, 4, 8}, Hkv <= 64, 1 <= T <
- * 2^31; k_cache, v_cache 16-byte aligned, q 8-byte aligned.  One launch;
- * every cache row is read once (HBM-bound), fp32 softmax and accumulation. */
+ * 2^31; q, k_cache, v_cache, s_cache 16-byte aligned.  One launch;
+ * every cache row is read once (HBM-bound), fp32 softmax and accumulation.
+ * Waits on copies are bounded (TG_STATUS_DECODE_TIMEOUT in the workspace's
+ * status word; re-zero the workspace after a timeout). */
 tg_status tg_gated_decode(const tg_bf16* q, const tg_bf16* k_cache, int64_t ld_k, const tg_bf16* v_cache,
                           int64_t ld_v, int64_t T, int32_t Hq, int32_t Hkv, int32_t d_h,
                           const float* s_cache, const float* gain, float tau, tg_bf16* out, float* lse,

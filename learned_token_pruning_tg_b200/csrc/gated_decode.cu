@@ -10,34 +10,37 @@
 // The step reads the whole cache once, so it is bound by HBM bandwidth:
 // T * Hkv * d_h * 2 bytes of K and as many of V (+ 4T of scores).
 //
-// Kernel: grid (Hkv, splits), 8 warps per CTA.  A CTA owns one KV head (and
+// Kernel: grid (Hkv, splits), 16 warps per CTA.  A CTA owns one KV head (and
 // the G = Hq / Hkv query heads that read it) and one contiguous range of keys.
-// Its key range streams through a 4-stage ring in shared memory (64 keys' K
-// and V rows a stage, copied with cp.async by all threads, each thread always
-// the same row pieces: 128 KB in flight per CTA for d_h = 128, as HBM latency
-// needs; one wave of CTAs).  A key is handled by a group of LPK lanes (8 for
+// Its key range (a multiple of 64 keys long) streams through a 4-stage ring in
+// shared memory (64 keys' K and V rows and scores a stage, one TMA box per
+// matrix (d_h x 1 head x 64 keys, no swizzle, keys past T read as zeros) and
+// one for the scores, issued by one thread and completing on the stage's
+// mbarrier: 128 KB in flight per CTA for d_h = 128, as HBM latency needs; one
+// wave of CTAs).  A key is handled by a group of LPK lanes (8 for
 // G <= 2, 16 for G = 4, 32 for G = 8, which keeps the registers per lane
 // about the same): each lane holds d_h / LPK elements of every query head
-// (scaled by tau / sqrt(d_h) log2(e)) and of the output, reads its piece of the
-// K and V rows from shared memory, and the group reduces the G partial dot
-// products with log2(LPK) xor shuffles.  Every lane group keeps its own fp32
+// (scaled by tau / sqrt(d_h) log2(e)) and of the output, as 16-byte units
+// j LPK + sub of the row (8-byte units when it holds only 4 elements), so a
+// quarter-warp -- one lane group or half of one -- reads 128 contiguous bytes of
+// one row from shared memory (no bank conflicts); the group reduces the G
+// partial dot products with log2(LPK) xor shuffles.  Every lane group keeps its own fp32
 // online softmax (running max, sum, output piece) over the keys it sees; the
 // groups of a warp merge by shuffles at the end, then the warps' states
 // are merged in shared memory, the CTA writes (m, l, o) to the workspace, and
 // the last CTA of the KV head (a counter in the workspace, reset by that CTA)
-// merges all splits and writes out (bf16) and the log-sum-exp.  No thread
-// waits on another.
+// merges all splits and writes out (bf16) and the log-sum-exp.  Waits on the
+// copies are bounded (TG_STATUS_DECODE_TIMEOUT); no thread waits on another.
 #include <cmath>
-#include <type_traits>
 
 #include "tg_host.cuh"
 
 namespace tg {
 namespace dec {
 
-constexpr int kWarps = 8;
-constexpr int kUnroll = 8;                  // keys per warp per stage
-constexpr int kStageKeys = kWarps * kUnroll;  // 64
+constexpr int kWarps = 16;
+constexpr int kStageKeys = 64;
+constexpr int kUnroll = kStageKeys / kWarps;  // keys per warp per stage
 constexpr int kRing = 4;                    // stages in flight
 constexpr int kMaxSplits = 64;
 constexpr int kMaxD = 128;
@@ -57,6 +60,7 @@ struct Args {
     float* lse;               // [Hq] or NULL
     float* part;              // [Hq][kMaxSplits][2 + d_h]: m, l (log2 units), o
     unsigned int* counter;    // [Hkv]
+    unsigned int* status;     // the workspace's status word
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -65,37 +69,32 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// E consecutive bf16 elements (E = 2 or 4) widened to fp32.
-template <int E>
-__device__ __forceinline__ void load_row(const __nv_bfloat16* p, float (&f)[E]) {
-    if constexpr (E == 4) {
+// One-dimensional tiled TMA load (coordinate c0 in elements) completing on `bar`.
+__device__ __forceinline__ void tma_load_1d(void* dst, const void* tmap, uint64_t* bar, int c0, uint64_t cache_hint) {
+    asm volatile(
+        "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2}], [%3], %4;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(c0), "r"(smem_u32(bar)), "l"(cache_hint)
+        : "memory");
+}
+
+// EW consecutive bf16 elements (4 or 8: one 8- or 16-byte load) widened to fp32.
+template <int EW>
+__device__ __forceinline__ void load_unit(const __nv_bfloat16* p, float (&f)[EW]) {
+    if constexpr (EW == 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(p);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    } else {
         const uint2 u = *reinterpret_cast<const uint2*>(p);
         f[0] = __uint_as_float(u.x << 16);
         f[1] = __uint_as_float(u.x & 0xffff0000u);
         f[2] = __uint_as_float(u.y << 16);
         f[3] = __uint_as_float(u.y & 0xffff0000u);
-    } else {
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
-        f[0] = __uint_as_float(u << 16);
-        f[1] = __uint_as_float(u & 0xffff0000u);
-    }
-}
-
-// Raw row pieces: E bf16 (E = 2 or 4) in one 4- or 8-byte load.
-template <int E>
-struct Piece {
-    using T = typename std::conditional<E == 4, uint2, uint32_t>::type;
-};
-template <int E>
-__device__ __forceinline__ void widen(const typename Piece<E>::T& u, float (&f)[E]) {
-    if constexpr (E == 4) {
-        f[0] = __uint_as_float(u.x << 16);
-        f[1] = __uint_as_float(u.x & 0xffff0000u);
-        f[2] = __uint_as_float(u.y << 16);
-        f[3] = __uint_as_float(u.y & 0xffff0000u);
-    } else {
-        f[0] = __uint_as_float(u << 16);
-        f[1] = __uint_as_float(u & 0xffff0000u);
     }
 }
 
@@ -108,13 +107,16 @@ struct Lanes {
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a) {
+__global__ void __launch_bounds__(kWarps * 32)
+gated_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                    const __grid_constant__ CUtensorMap tmap_s, const Args a) {
     constexpr int LPK = Lanes<D, G>::kPerKey;
     constexpr int ED = D / LPK;          // elements per lane (multiple of 4)
     static_assert(ED % 4 == 0, "a lane holds whole 8-byte pieces");
+    constexpr int EW = ED >= 8 ? 8 : 4;  // elements per unit: a 16-byte (or 8-byte) load
+    constexpr int NU = ED / EW;          // units per lane; unit j of lane `sub` is unit j LPK + sub of the row
     constexpr int KPS = 32 / LPK;        // keys a warp handles at once
     __shared__ float s_m[kWarps][G], s_l[kWarps][G];
-    __shared__ float s_o[kWarps][G][D];
     __shared__ bool s_last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int grp = lane / LPK, sub = lane % LPK;
@@ -127,11 +129,11 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
     for (int g = 0; g < G; ++g) {
         const int head = kvh * G + g;
 #pragma unroll
-        for (int e = 0; e < ED; e += 4) {
-            float f[4];
-            load_row<4>(a.q + static_cast<int64_t>(head) * D + sub * ED + e, f);
+        for (int j = 0; j < NU; ++j) {
+            float f[EW];
+            load_unit<EW>(a.q + static_cast<int64_t>(head) * D + (j * LPK + sub) * EW, f);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) qr[g][e + i] = f[i] * a.scale_log2;
+            for (int i = 0; i < EW; ++i) qr[g][j * EW + i] = f[i] * a.scale_log2;
         }
         gl2[g] = a.gain ? a.gain[head] * kLog2e : 0.0f;
     }
@@ -145,42 +147,42 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
     }
 
     constexpr int kRow = D * 2;                        // bytes of one key's row (one head)
-    constexpr int kStageBytes = kStageKeys * kRow * 2;  // K rows, then V rows
-    constexpr int kPiecesPerRow = kRow / 16;
-    constexpr int kRowsPerPass = kWarps * 32 / kPiecesPerRow;
-    constexpr int kPasses = kStageKeys / kRowsPerPass;
-    extern __shared__ __align__(16) uint8_t ring[];
+    constexpr int kScoreOff = kStageKeys * kRow * 2;    // K rows, then V rows, then the 64 scores
+    constexpr int kStageBytes = kScoreOff + kStageKeys * 4;
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ __align__(8) uint64_t full[kRing];
+    __shared__ int abort_flag;
     const int n_keys = static_cast<int>(c_end - c_begin);
     const int n_stages = (n_keys + kStageKeys - 1) / kStageKeys;
-    // this thread always copies piece `cp_piece` of rows cp_row + kRowsPerPass j of K and of V
-    const int cp_piece = threadIdx.x % kPiecesPerRow, cp_row = threadIdx.x / kPiecesPerRow;
-    const char* kg = reinterpret_cast<const char*>(a.k + static_cast<int64_t>(kvh) * D) + cp_piece * 16;
-    const char* vg = reinterpret_cast<const char*>(a.v + static_cast<int64_t>(kvh) * D) + cp_piece * 16;
-    const int64_t ldk2 = a.ld_k * 2, ldv2 = a.ld_v * 2;
-    auto issue = [&](int t) {
-        uint8_t* slot = ring + (t % kRing) * kStageBytes + cp_row * kRow + cp_piece * 16;
-#pragma unroll
-        for (int j = 0; j < kPasses; ++j) {
-            const int r = cp_row + j * kRowsPerPass;
-            const int64_t c = c_begin + static_cast<int64_t>(t) * kStageKeys + r;
-            if (c < c_end) {
-                const uint32_t dk = smem_u32(slot + j * kRowsPerPass * kRow);
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dk), "l"(kg + c * ldk2) : "memory");
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dk + kStageKeys * kRow),
-                             "l"(vg + c * ldv2)
-                             : "memory");
-            }
-        }
-    };
-    for (int t = 0; t < kRing - 1; ++t) {
-        if (t < n_stages) issue(t);
-        asm volatile("cp.async.commit_group;" ::: "memory");
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kRing; ++i) mbar_init(&full[i], 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_v);
+        if (a.s) tma_prefetch_desc(&tmap_s);
     }
-    for (int t = 0; t < n_stages; ++t) {
-        if (t + kRing - 1 < n_stages) issue(t + kRing - 1);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_group %0;" ::"n"(kRing - 1) : "memory");  // stage t has landed (own copies)
-        __syncthreads();                                                      // ... and everyone's
+    __syncthreads();
+    // one thread: stage t's K and V boxes into slot t mod kRing
+    auto issue = [&](int t) {
+        if (lane != 0) return;
+        uint8_t* slot = ring + (t % kRing) * kStageBytes;
+        uint64_t* bar = &full[t % kRing];
+        const int c_first = static_cast<int>(c_begin) + t * kStageKeys;
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(a.s ? kStageBytes : kScoreOff));
+        tma_load_3d(slot, &tmap_k, bar, 0, kvh, c_first, kEvictFirst);
+        tma_load_3d(slot + kStageKeys * kRow, &tmap_v, bar, 0, kvh, c_first, kEvictFirst);
+        if (a.s) tma_load_1d(slot + kScoreOff, &tmap_s, bar, c_first, kEvictFirst);
+    };
+    if (warp == 0)
+        for (int t = 0; t < kRing - 1 && t < n_stages; ++t) issue(t);
+    bool ok = true;
+    int t = 0;
+    for (; t < n_stages; ++t) {
+        if (warp == 0 && t + kRing - 1 < n_stages) issue(t + kRing - 1);
+        ok = mbar_wait(&full[t % kRing], static_cast<uint32_t>(t / kRing) & 1, &abort_flag, a.status,
+                       TG_STATUS_DECODE_TIMEOUT);
+        if (!__syncthreads_and(ok)) break;  // every thread leaves together
         const uint8_t* slot = ring + (t % kRing) * kStageBytes;
 #pragma unroll
         for (int step = 0; step < kUnroll / KPS; ++step) {
@@ -190,18 +192,19 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
             const bool valid = c < c_end;
             float kf[ED], vf[ED];
 #pragma unroll
-            for (int e = 0; e < ED; e += 4) {
+            for (int j = 0; j < NU; ++j) {
+                const int off = (j * LPK + sub) * EW * 2;
                 if (valid) {
-                    widen<4>(*reinterpret_cast<const uint2*>(slot + r * kRow + (sub * ED + e) * 2),
-                             *reinterpret_cast<float(*)[4]>(kf + e));
-                    widen<4>(*reinterpret_cast<const uint2*>(slot + kStageKeys * kRow + r * kRow + (sub * ED + e) * 2),
-                             *reinterpret_cast<float(*)[4]>(vf + e));
-                } else {  // past the range: no row here (weight 0, and no NaN from stale bits)
+                    load_unit<EW>(reinterpret_cast<const __nv_bfloat16*>(slot + r * kRow + off),
+                                  *reinterpret_cast<float(*)[EW]>(kf + j * EW));
+                    load_unit<EW>(reinterpret_cast<const __nv_bfloat16*>(slot + kStageKeys * kRow + r * kRow + off),
+                                  *reinterpret_cast<float(*)[EW]>(vf + j * EW));
+                } else {  // past the range: the slot holds another key or zeros here (weight 0)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) kf[e + i] = vf[e + i] = 0.0f;
+                    for (int i = 0; i < EW; ++i) kf[j * EW + i] = vf[j * EW + i] = 0.0f;
                 }
             }
-            const float sb = (valid && a.s) ? __ldg(a.s + c) : 0.0f;
+            const float sb = (valid && a.s) ? reinterpret_cast<const float*>(slot + kScoreOff)[r] : 0.0f;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 float d = 0.0f;
@@ -224,9 +227,22 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
                 for (int e = 0; e < ED; ++e) o[g][e] = fmaf(p, vf[e], o[g][e]);
             }
         }
-        __syncthreads();  // the slot is refilled by the next iteration's copies
+        // these generic-proxy reads of the slot come before the bulk copies (async proxy) that
+        // refill it once every thread is past the barrier
+        fence_proxy_async_smem();
+        __syncthreads();
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (t < n_stages) {
+        // gave up: let the copies already issued land before the CTA's shared memory goes away
+        if (threadIdx.x == 0) {
+            volatile int no_abort = 0;
+            for (int u = t; u < n_stages && u < t + kRing; ++u)
+                mbar_wait(&full[u % kRing], static_cast<uint32_t>(u / kRing) & 1, &no_abort, a.status,
+                          TG_STATUS_DECODE_TIMEOUT);
+        }
+        __syncthreads();
+        return;
+    }
 
     // merge the lane groups of each warp (lanes sub, sub + LPK, ... hold the same output piece)
 #pragma unroll
@@ -247,7 +263,9 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
             m[g] = mx;
         }
     }
-    // merge the warps' states
+    // merge the warps' states (through the ring, idle now: every stage has landed and been read)
+    float (*s_o)[G][D] = reinterpret_cast<float (*)[G][D]>(ring);
+    static_assert(kWarps * G * D * 4 <= kRing * (kStageKeys * D * 2 * 2), "the merge fits in the ring");
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         if (lane == 0) {
@@ -256,7 +274,9 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
         }
         if (grp == 0) {
 #pragma unroll
-            for (int e = 0; e < ED; ++e) s_o[warp][g][sub * ED + e] = o[g][e];
+            for (int j = 0; j < NU; ++j)
+#pragma unroll
+                for (int i = 0; i < EW; ++i) s_o[warp][g][(j * LPK + sub) * EW + i] = o[g][j * EW + i];
         }
     }
     __syncthreads();
@@ -315,15 +335,16 @@ __global__ void __launch_bounds__(kWarps * 32) gated_decode_kernel(const Args a)
 // from the occupancy calculator, cached per kernel and device), at least 64
 // keys per split.
 template <int D, int G>
-static tg_status launch(Args a, int64_t T, cudaStream_t st) {
+static tg_status launch(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& ms, Args a, int64_t T,
+                        cudaStream_t st) {
     static std::atomic<int> occ_cache[64];
     static std::atomic<int> smem_set0[64];
     const int dev = current_device();
     int occ = dev >= 0 ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
     if (occ <= 0) {
-        if (!set_max_dynamic_smem(gated_decode_kernel<D, G>, kRing * kStageKeys * D * 2 * 2, smem_set0) ||
+        if (!set_max_dynamic_smem(gated_decode_kernel<D, G>, kRing * (kStageKeys * D * 2 * 2 + kStageKeys * 4), smem_set0) ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gated_decode_kernel<D, G>, kWarps * 32,
-                                                          kRing * kStageKeys * D * 2 * 2) !=
+                                                          kRing * (kStageKeys * D * 2 * 2 + kStageKeys * 4)) !=
                 cudaSuccess ||
             occ <= 0)
             occ = 1;
@@ -333,23 +354,25 @@ static tg_status launch(Args a, int64_t T, cudaStream_t st) {
     if (nsplit > (T + 63) / 64) nsplit = (T + 63) / 64;
     if (nsplit > kMaxSplits) nsplit = kMaxSplits;
     if (nsplit < 1) nsplit = 1;
-    a.split_len = static_cast<int>((T + nsplit - 1) / nsplit);
+    // split lengths are multiples of the 64-key stage (the scores' TMA coordinate must be a multiple of 4)
+    a.split_len = static_cast<int>(((T + nsplit - 1) / nsplit + kStageKeys - 1) / kStageKeys * kStageKeys);
     nsplit = (T + a.split_len - 1) / a.split_len;
-    constexpr int kSmem = kRing * kStageKeys * D * 2 * 2;
+    constexpr int kSmem = kRing * (kStageKeys * D * 2 * 2 + kStageKeys * 4);  // the ring
     static std::atomic<int> smem_set[64];
     if (!set_max_dynamic_smem(gated_decode_kernel<D, G>, kSmem, smem_set)) return TG_ERR_CUDA;
     gated_decode_kernel<D, G><<<dim3(static_cast<unsigned>(a.Hkv), static_cast<unsigned>(nsplit)), kWarps * 32,
-                                kSmem, st>>>(a);
+                                kSmem, st>>>(mk, mv, ms, a);
     return launch_status();
 }
 
 template <int D>
-static tg_status launch_g(const Args& a, int G, int64_t T, cudaStream_t st) {
+static tg_status launch_g(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& ms, const Args& a, int G,
+                          int64_t T, cudaStream_t st) {
     switch (G) {
-        case 1: return launch<D, 1>(a, T, st);
-        case 2: return launch<D, 2>(a, T, st);
-        case 4: return launch<D, 4>(a, T, st);
-        case 8: return launch<D, 8>(a, T, st);
+        case 1: return launch<D, 1>(mk, mv, ms, a, T, st);
+        case 2: return launch<D, 2>(mk, mv, ms, a, T, st);
+        case 4: return launch<D, 4>(mk, mv, ms, a, T, st);
+        case 8: return launch<D, 8>(mk, mv, ms, a, T, st);
     }
     return TG_ERR_UNSUPPORTED;
 }
@@ -376,9 +399,8 @@ extern "C" tg_status tg_gated_decode(const tg_bf16* q, const tg_bf16* k_cache, i
     if (G != 1 && G != 2 && G != 4 && G != 8) return TG_ERR_UNSUPPORTED;
     if (Hkv > 64 || T > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
     if (!aligned16(workspace) || workspace_bytes < ws_decode_bytes(Hq)) return TG_ERR_INVALID_ARG;
-    // 16-byte copies of cache rows; q read in 8-byte pieces
-    if (!aligned16(k_cache) || !aligned16(v_cache) || (ld_k % 8) != 0 || (ld_v % 8) != 0 ||
-        reinterpret_cast<uintptr_t>(q) % 8 != 0)
+    // TMA boxes of cache rows (16-byte aligned bases and strides); q read in 16-byte units
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q) || (ld_k % 8) != 0 || (ld_v % 8) != 0)
         return TG_ERR_INVALID_ARG;
     if (ld_k < static_cast<int64_t>(Hkv) * d_h || ld_v < static_cast<int64_t>(Hkv) * d_h) return TG_ERR_INVALID_ARG;
 
@@ -396,8 +418,30 @@ extern "C" tg_status tg_gated_decode(const tg_bf16* q, const tg_bf16* k_cache, i
     a.out = reinterpret_cast<__nv_bfloat16*>(out);
     a.lse = lse;
     a.counter = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + kWsHeader);
+    a.status = status_word(workspace);
     a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeader + 256);
     a.split_len = 0;
+    // K and V as [T, Hkv, d_h] boxes of d_h x 1 x 64 keys, rows kept in order (no swizzle)
+    CUtensorMap mk, mv;
+    const uint64_t dims[3] = {static_cast<uint64_t>(d_h), static_cast<uint64_t>(Hkv), static_cast<uint64_t>(T)};
+    const uint64_t sk[2] = {static_cast<uint64_t>(d_h) * 2, static_cast<uint64_t>(ld_k) * 2};
+    const uint64_t sv[2] = {static_cast<uint64_t>(d_h) * 2, static_cast<uint64_t>(ld_v) * 2};
+    const uint32_t box[3] = {static_cast<uint32_t>(d_h), 1, static_cast<uint32_t>(dec::kStageKeys)};
+    if (!make_tmap_bf16(&mk, k_cache, 3, dims, sk, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tmap_bf16(&mv, v_cache, 3, dims, sv, box, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_SWIZZLE_NONE))
+        return TG_ERR_CUDA;
+    // the scores as [T] fp32 boxes of 64 (unused without scores: the K map stands in)
+    CUtensorMap ms = mk;
+    if (s_cache) {
+        if (!aligned16(s_cache)) return TG_ERR_INVALID_ARG;
+        const uint64_t sdims[1] = {static_cast<uint64_t>(T)};
+        const uint32_t sbox[1] = {static_cast<uint32_t>(dec::kStageKeys)};
+        if (!make_tmap_bf16(&ms, s_cache, 1, sdims, nullptr, sbox, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+            return TG_ERR_CUDA;
+    }
     cudaStream_t st = as_stream(stream);
-    return d_h == 128 ? dec::launch_g<128>(a, G, T, st) : dec::launch_g<64>(a, G, T, st);
+    return d_h == 128 ? dec::launch_g<128>(mk, mv, ms, a, G, T, st) : dec::launch_g<64>(mk, mv, ms, a, G, T, st);
 }

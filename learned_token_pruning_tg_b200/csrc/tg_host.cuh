@@ -59,7 +59,7 @@ struct TmapKey {
     const void* base;
     uint64_t dims[5], strides[4];
     uint32_t box[5];
-    int32_t rank, promo;
+    int32_t rank, promo, swizzle, dtype;
 };
 struct TmapCache {
     static constexpr int kEntries = 16;
@@ -70,16 +70,21 @@ struct TmapCache {
 };
 
 // Tensor map over a bf16 tensor of `rank` dims (dims[0] innermost, in elements;
-// strides[i] in bytes for dims 1..rank-1), box `box` (elements), 128-byte swizzle.
+// strides[i] in bytes for dims 1..rank-1), box `box` (elements), 128-byte swizzle
+// unless `swizzle` says otherwise (and bf16 unless `dtype` does).
 inline bool make_tmap_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                            const uint64_t* strides_bytes, const uint32_t* box,
-                           CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
+                           CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B,
+                           CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     if (rank < 1 || rank > 5) return false;
     TmapKey k;
     std::memset(&k, 0, sizeof(k));  // padding too, so keys compare bytewise
     k.base = base;
     k.rank = rank;
     k.promo = static_cast<int32_t>(promo);
+    k.swizzle = static_cast<int32_t>(swizzle);
+    k.dtype = static_cast<int32_t>(dtype);
     for (int i = 0; i < rank; ++i) {
         k.dims[i] = dims[i];
         k.box[i] = box[i];
@@ -103,8 +108,8 @@ inline bool make_tmap_bf16(CUtensorMap* m, const void* base, int rank, const uin
         estride[i] = 1;
     }
     for (int i = 0; i + 1 < rank; ++i) gstride[i] = strides_bytes[i];
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
-                    gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+    CUresult r = fn(m, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+                    gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
     const int slot = cache.next;
