@@ -37,6 +37,10 @@ def lib():
         L.tgo_rope.restype = i32
         L.tgo_gated_attention.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, dbl, vp, i64, vp, vp]
         L.tgo_gated_attention.restype = i32
+        L.tgo_random_select.argtypes = [i64, i64, i64, i64, ctypes.c_uint64, vp]
+        L.tgo_random_select.restype = i64
+        L.tgo_splitmix64_stream.argtypes = [ctypes.c_uint64, i64, vp]
+        L.tgo_splitmix64_stream.restype = i32
         L.tgo_round_bf16.argtypes = [ctypes.c_float]
         L.tgo_round_bf16.restype = ctypes.c_float
         _lib = L
@@ -88,6 +92,27 @@ def topk_select(scores, doc_begin, doc_end, k_doc):
     n = lib().tgo_topk_select(_p(s), N, doc_begin, doc_end, k_doc, _p(out))
     if n != K:
         raise ValueError("tgo_topk_select failed")
+    return out[:K]
+
+
+def splitmix64_stream(state, n):
+    """n successive SplitMix64 outputs from `state` (uint64)."""
+    out = np.empty(max(n, 1), dtype=np.uint64)
+    if lib().tgo_splitmix64_stream(ctypes.c_uint64(state), n, _p(out)) != 0:
+        raise ValueError("tgo_splitmix64_stream failed")
+    return out[:n]
+
+
+def random_select(N, doc_begin, doc_end, k_doc, seed):
+    """Random-K kept indices (int32, ascending): the k_doc document tokens with the largest
+    SplitMix64 keys drawn from `seed`, plus every token outside the span."""
+    K = kept_count(N, doc_begin, doc_end, k_doc)
+    if K < 0:
+        raise ValueError("bad span or budget")
+    out = np.empty(max(K, 1), dtype=np.int32)
+    n = lib().tgo_random_select(N, doc_begin, doc_end, k_doc, ctypes.c_uint64(seed), _p(out))
+    if n != K:
+        raise ValueError("tgo_random_select failed")
     return out[:K]
 
 

@@ -166,6 +166,83 @@ int64_t tgo_topk_select(const float* scores, int64_t N, int64_t doc_begin,
     return n;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Random-K selector.  The pages compare TokenGate with keeping K document
+ * tokens chosen at random (a budget-matched random baseline).  The draw is
+ * SplitMix64 (Steele, Lea and Flood; the constants of Vigna's reference code):
+ * the state advances by 0x9E3779B97F4A7C15 per output, and an output is the
+ * new state through z ^= z >> 30; z *= 0xBF58476D1CE4E5B9; z ^= z >> 27;
+ * z *= 0x94D049BB133111EB; z ^= z >> 31.  Token i draws the (i + 1)-th output
+ * of the stream started at state `seed`; a document token's key is that
+ * output's top 32 bits, and the k_doc largest keys are kept (the lower index
+ * first on equal keys), with every token outside the span. */
+uint64_t tgo_splitmix64_next(uint64_t* state)
+{
+    *state += 0x9E3779B97F4A7C15ull;
+    uint64_t z = *state;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+int tgo_splitmix64_stream(uint64_t state, int64_t n, uint64_t* out)
+{
+    if (n < 0 || (n > 0 && !out))
+        return -1;
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = tgo_splitmix64_next(&state);
+    return 0;
+}
+
+static const uint32_t* g_rkeys; /* comparator context (single-threaded oracle) */
+
+static int cmp_rkey(const void* a, const void* b)
+{
+    int32_t i = *(const int32_t*)a, j = *(const int32_t*)b;
+    if (g_rkeys[i] != g_rkeys[j])
+        return g_rkeys[i] > g_rkeys[j] ? -1 : 1; /* larger key first */
+    return i < j ? -1 : (i > j);                 /* then lower index */
+}
+
+int64_t tgo_random_select(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_doc,
+                          uint64_t seed, int32_t* kept)
+{
+    int64_t K = tgo_kept_count(N, doc_begin, doc_end, k_doc);
+    if (K < 0 || !kept || N > 2147483647)
+        return -1;
+    uint32_t* keys = (uint32_t*)malloc((size_t)(N > 0 ? N : 1) * sizeof(uint32_t));
+    int32_t* order = (int32_t*)malloc((size_t)(N > 0 ? N : 1) * sizeof(int32_t));
+    unsigned char* keep = (unsigned char*)calloc((size_t)(N > 0 ? N : 1), 1);
+    if (!keys || !order || !keep) {
+        free(keys);
+        free(order);
+        free(keep);
+        return -1;
+    }
+    uint64_t state = seed;
+    for (int64_t i = 0; i < N; ++i)
+        keys[i] = (uint32_t)(tgo_splitmix64_next(&state) >> 32);
+    int64_t n_doc = doc_end - doc_begin;
+    for (int64_t r = 0; r < n_doc; ++r)
+        order[r] = (int32_t)(doc_begin + r);
+    g_rkeys = keys;
+    qsort(order, (size_t)n_doc, sizeof(int32_t), cmp_rkey);
+    int64_t keep_doc = k_doc < n_doc ? k_doc : n_doc;
+    for (int64_t i = 0; i < N; ++i)
+        if (i < doc_begin || i >= doc_end)
+            keep[i] = 1;
+    for (int64_t r = 0; r < keep_doc; ++r)
+        keep[order[r]] = 1;
+    int64_t n = 0;
+    for (int64_t i = 0; i < N; ++i)
+        if (keep[i])
+            kept[n++] = (int32_t)i;
+    free(keys);
+    free(order);
+    free(keep);
+    return n;
+}
+
 double tgo_topk_threshold(const float* scores, int64_t N, int64_t doc_begin,
                           int64_t doc_end, int64_t k_doc)
 {

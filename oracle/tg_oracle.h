@@ -73,6 +73,15 @@ int64_t tgo_topk_select(const float* scores, int64_t N, int64_t doc_begin,
 /* The k_doc-th document score in the selection order (the threshold), as
  * fp64; NaN if k_doc == 0 or the span is empty.  Used to express the
  * "within 1e-4 of the K-th threshold" acceptance rule. */
+/* Random-K selector: the k_doc document tokens with the largest keys, key of
+ * token i = top 32 bits of the (i + 1)-th SplitMix64 output from state `seed`
+ * (lower index first on equal keys), plus every token outside the span,
+ * ascending.  Returns the count written or -1. */
+int64_t tgo_random_select(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_doc,
+                          uint64_t seed, int32_t* kept);
+/* n successive SplitMix64 outputs from `state` (the generator itself). */
+int tgo_splitmix64_stream(uint64_t state, int64_t n, uint64_t* out);
+
 double tgo_topk_threshold(const float* scores, int64_t N, int64_t doc_begin,
                           int64_t doc_end, int64_t k_doc);
 
