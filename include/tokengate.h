@@ -159,6 +159,19 @@ tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int64_t doc_beg
                                  int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
                                  void* stream);
 
+/* Random-K selector (the pages' budget-matched random baseline): keeps
+ * min(k_doc, doc_end - doc_begin) document tokens chosen at random, plus every
+ * token outside [doc_begin, doc_end), as ascending indices (the same output as
+ * tg_topk_select).  Token i's key is the top 32 bits of the (i + 1)-th output
+ * of a SplitMix64 stream started at state `seed` (state += 0x9E3779B97F4A7C15;
+ * z ^= z >> 30; z *= 0xBF58476D1CE4E5B9; z ^= z >> 27; z *= 0x94D049BB133111EB;
+ * z ^= z >> 31); the largest keys are kept, the lower index first on equal
+ * keys, so the result is a deterministic function of the seed.  Workspace,
+ * sizes, errors and limits as tg_topk_select (the same kernel, keys drawn in
+ * registers instead of read from scores). */
+tg_status tg_random_select(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_doc, uint64_t seed,
+                           int32_t* kept_idx, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Compaction (step 3: layers above the gate see only the K kept tokens):
  *   h_out[r, :] = h[kept_idx[r], :]           (bit-exact copy)
  *   pos_out[r]  = pos_in ? pos_in[kept_idx[r]] : kept_idx[r]

@@ -22,11 +22,26 @@
 //     counts after one more grid barrier, in-block prefixes from ballots.
 // The grid barrier is a sense-reversing counter in the workspace that resets
 // itself; each wait is bounded and reports TG_STATUS_SELECT_TIMEOUT.
+//
+// The same kernel is the random-K selector (the pages' budget-matched random
+// baseline) when it is given no scores: token i's key is then the top 32 bits
+// of the (i + 1)-th output of a SplitMix64 stream started at `seed` (Steele,
+// Lea and Flood; the state advances by 0x9E3779B97F4A7C15 and each output is
+// the state through the published finalizer), drawn in registers.
 #include <mutex>
 
 #include "tg_host.cuh"
 
 namespace tg {
+
+// Token i's random key: the top 32 bits of SplitMix64 output i + 1 from `seed`
+// (the state after i + 1 steps is seed + (i + 1) * 0x9E3779B97F4A7C15 mod 2^64).
+__device__ __forceinline__ uint32_t random_key(uint64_t seed, int64_t i) {
+    uint64_t z = seed + static_cast<uint64_t>(i + 1) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return static_cast<uint32_t>((z ^ (z >> 31)) >> 32);
+}
 
 __device__ __forceinline__ uint32_t radix_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -95,7 +110,8 @@ __device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* s_warp
 }
 
 struct SelectArgs {
-    const float* scores;
+    const float* scores;   // NULL: random keys from `seed`
+    uint64_t seed;
     int64_t N, D0, D1;
     unsigned int kd;   // document tokens kept, 0 < kd < n_doc
     int32_t* out;
@@ -120,7 +136,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const Se
 #pragma unroll
     for (int j = 0; j < EPT; ++j) {
         const int64_t i = base + static_cast<int64_t>(j) * kSelectThreads + tid;
-        key[j] = (j < a.ept && i < end) ? radix_key(__ldg(a.scores + i)) : 0u;
+        key[j] = (j < a.ept && i < end) ? (a.scores ? radix_key(__ldg(a.scores + i)) : random_key(a.seed, i)) : 0u;
     }
 
     uint32_t prefix = 0, pmask = 0;
@@ -262,14 +278,15 @@ static cudaError_t launch_select(const SelectArgs& a, int grid, cudaStream_t st)
 
 using namespace tg;
 
-extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_begin, int64_t doc_end,
-                                    int64_t k_doc, int32_t* kept_idx, void* workspace, size_t workspace_bytes,
-                                    void* stream) {
+// The select with keys from `scores`, or random keys from `seed` when scores is NULL.
+static tg_status select_impl(const float* scores, uint64_t seed, int64_t N, int64_t doc_begin, int64_t doc_end,
+                             int64_t k_doc, int32_t* kept_idx, void* workspace, size_t workspace_bytes,
+                             void* stream) {
     const int64_t K = tg_kept_count(N, doc_begin, doc_end, k_doc);
     if (K < 0) return TG_ERR_INVALID_ARG;
     if (N > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
     if (K == 0) return TG_OK;
-    if (!scores || !kept_idx) return TG_ERR_INVALID_ARG;
+    if (!kept_idx) return TG_ERR_INVALID_ARG;
     const int64_t n_doc = doc_end - doc_begin;
     const int64_t kd = k_doc < n_doc ? k_doc : n_doc;
     cudaStream_t st = as_stream(stream);
@@ -292,6 +309,7 @@ extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_
 
     SelectArgs a;
     a.scores = scores;
+    a.seed = seed;
     a.N = N;
     a.D0 = doc_begin;
     a.D1 = doc_end;
@@ -312,6 +330,18 @@ extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_
     else
         e = launch_select<16>(a, grid, st);
     return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;
+}
+
+extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_begin, int64_t doc_end,
+                                    int64_t k_doc, int32_t* kept_idx, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+    if (!scores && tg_kept_count(N, doc_begin, doc_end, k_doc) > 0) return TG_ERR_INVALID_ARG;
+    return select_impl(scores, 0, N, doc_begin, doc_end, k_doc, kept_idx, workspace, workspace_bytes, stream);
+}
+
+extern "C" tg_status tg_random_select(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_doc, uint64_t seed,
+                                      int32_t* kept_idx, void* workspace, size_t workspace_bytes, void* stream) {
+    return select_impl(nullptr, seed, N, doc_begin, doc_end, k_doc, kept_idx, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- allocation-free entry point
@@ -388,6 +418,7 @@ extern "C" tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int6
 
     SelectArgs a;
     a.scores = scores;
+    a.seed = 0;
     a.N = N;
     a.D0 = doc_begin;
     a.D1 = doc_end;

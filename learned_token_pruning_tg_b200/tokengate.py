@@ -48,13 +48,15 @@ def lib() -> ctypes.CDLL:
         L.tg_gate_score.argtypes = [vp, i64, i32, i64, vp, f32, vp, vp, vp, f32, i32, vp, vp, sz, vp]
         L.tg_topk_select.argtypes = [vp, i64, i64, i64, i64, vp, vp, sz, vp]
         L.tg_topk_select_noalloc.argtypes = [vp, i64, i64, i64, i64, vp, vp]
+        L.tg_random_select.argtypes = [i64, i64, i64, i64, ctypes.c_uint64, vp, vp, sz, vp]
         L.tg_gather_compact.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, vp, vp, vp]
         L.tg_rope_apply.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, f64, vp]
         L.tg_gated_attention.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp,
                                          vp, sz, vp]
         L.tg_gated_decode.argtypes = [vp, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp, vp, sz, vp]
         L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
-        for fn in ("tg_gate_score", "tg_topk_select", "tg_topk_select_noalloc", "tg_gather_compact", "tg_rope_apply",
+        for fn in ("tg_gate_score", "tg_topk_select", "tg_topk_select_noalloc", "tg_random_select", "tg_gather_compact",
+                   "tg_rope_apply",
                    "tg_gated_attention", "tg_gated_decode", "tg_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
@@ -168,6 +170,21 @@ def tg_topk_select_noalloc(scores, doc_begin: int, doc_end: int, k_doc: int, kep
         raise ValueError("kept_idx too small or not contiguous")
     _check("tg_topk_select_noalloc", lib().tg_topk_select_noalloc(
         _ptr(scores), N, doc_begin, doc_end, k_doc, _ptr(kept_idx), _stream(stream)))
+    return kept_idx
+
+
+def tg_random_select(N: int, doc_begin: int, doc_end: int, k_doc: int, seed: int, kept_idx, workspace, stream=None):
+    """The random-K selector: k_doc document tokens drawn from SplitMix64(seed), plus every token outside
+    the span, ascending (same output layout as tg_topk_select)."""
+    _req(kept_idx, "kept_idx", torch.int32, 1)
+    K = tg_kept_count(N, doc_begin, doc_end, k_doc)
+    if K < 0:
+        raise TokenGateError("tg_random_select", TG_ERR_INVALID_ARG)
+    if kept_idx.numel() < K or not kept_idx.is_contiguous():
+        raise ValueError("kept_idx too small or not contiguous")
+    _check("tg_random_select", lib().tg_random_select(
+        N, doc_begin, doc_end, k_doc, ctypes.c_uint64(seed & ((1 << 64) - 1)), _ptr(kept_idx), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
     return kept_idx
 
 

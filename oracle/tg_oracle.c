@@ -228,14 +228,11 @@ int64_t tgo_random_select(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t
     g_rkeys = keys;
     qsort(order, (size_t)n_doc, sizeof(int32_t), cmp_rkey);
     int64_t keep_doc = k_doc < n_doc ? k_doc : n_doc;
-    for (int64_t i = 0; i < N; ++i)
-        if (i < doc_begin || i >= doc_end)
-            keep[i] = 1;
     for (int64_t r = 0; r < keep_doc; ++r)
         keep[order[r]] = 1;
     int64_t n = 0;
     for (int64_t i = 0; i < N; ++i)
-        if (keep[i])
+        if (keep[i] || i < doc_begin || i >= doc_end) /* every token outside the span is kept */
             kept[n++] = (int32_t)i;
     free(keys);
     free(order);
