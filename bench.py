@@ -281,7 +281,7 @@ def run_reference(args, rank, world):
 
 def run_tokengate(args, rank, world, local_rank):
     from learned_token_pruning_tg_b200 import tokengate as tg
-    from learned_token_pruning_tg_b200.path import STAGES, GatedPrefillLayer
+    from learned_token_pruning_tg_b200.path import STAGES, GatedPrefillLayer, nvtx_marks
 
     if not os.path.exists(tg.LIB_PATH):
         from learned_token_pruning_tg_b200 import build as tg_build
@@ -296,7 +296,8 @@ def run_tokengate(args, rank, world, local_rank):
                               ap.gain, ap.tau, eps=w.eps, rope_base=w.rope_base, device=dev)
     h = gi.h.to(dev)
     for _ in range(args.warmup):
-        layer.run(h)
+        # warm-up steps carry NVTX ranges per step when asked (for a profiler's NVTX filter)
+        layer.run(h, mark=nvtx_marks() if args.nvtx else None)
     torch.cuda.synchronize()
     assert layer.device_status() == 0, "device wait timed out during warm-up"
 
@@ -674,6 +675,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["tokengate", "reference"], default="tokengate")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nvtx", action="store_true", help="NVTX range tg:<step> around each warm-up step")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--decode-layer", action="store_true",
                     help="time one layer's decoding step over a 64k cache (the decode kernel alone)")

@@ -239,6 +239,17 @@ tg_status tg_gated_decode(const tg_bf16* q, const tg_bf16* k_cache, int64_t ld_k
                           const float* s_cache, const float* gain, float tau, tg_bf16* out, float* lse,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Test hook (fault injection without a fault): sets the time limit of the
+ * grid barrier inside tg_topk_select, tg_topk_select_noalloc and
+ * tg_random_select on the current device to `ns` nanoseconds of %globaltimer
+ * (0 restores the default of about one second).  With a limit of a few
+ * nanoseconds a call's blocks stop waiting for one another, set
+ * TG_STATUS_SELECT_TIMEOUT and return before writing any result; the
+ * workspace must then be zero-filled again.  No other wait in the library is
+ * affected (the others also guard asynchronous copies in flight).
+ * Synchronous; not for use while a select may be running. */
+tg_status tg_debug_set_select_wait_limit(uint64_t ns);
+
 /* Reads the workspace's status word after synchronizing `stream`.
  * *status_word receives the raw TG_STATUS_* bits (may be NULL).
  * Returns TG_ERR_TIMEOUT if any bit is set, TG_OK otherwise. */

@@ -50,6 +50,11 @@ __device__ __forceinline__ uint32_t radix_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Time limit of the grid barrier's wait (ns of %globaltimer), per device.
+// tg_debug_set_select_wait_limit shrinks it so that tests can make the barrier
+// give up (fault injection without a fault); no other wait reads it.
+__device__ unsigned long long g_select_wait_limit_ns = kWaitLimitNs;
+
 // Grid-wide barrier.  Returns false (block-uniformly) if the wait timed out.
 __device__ __forceinline__ bool grid_sync(SelectScratch* sc, unsigned nblocks, unsigned int* status, int* s_ok) {
     __syncthreads();
@@ -66,7 +71,7 @@ __device__ __forceinline__ bool grid_sync(SelectScratch* sc, unsigned nblocks, u
         } else {
             const unsigned long long t0 = globaltimer_ns();
             while (*vgen == g) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                if (globaltimer_ns() - t0 > g_select_wait_limit_ns) {
                     atomicOr(status, TG_STATUS_SELECT_TIMEOUT);
                     ok = 0;
                     break;
@@ -337,6 +342,11 @@ extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_
                                     void* stream) {
     if (!scores && tg_kept_count(N, doc_begin, doc_end, k_doc) > 0) return TG_ERR_INVALID_ARG;
     return select_impl(scores, 0, N, doc_begin, doc_end, k_doc, kept_idx, workspace, workspace_bytes, stream);
+}
+
+extern "C" tg_status tg_debug_set_select_wait_limit(uint64_t ns) {
+    const unsigned long long v = ns ? static_cast<unsigned long long>(ns) : kWaitLimitNs;
+    return cudaMemcpyToSymbol(g_select_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? TG_OK : TG_ERR_CUDA;
 }
 
 extern "C" tg_status tg_random_select(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_doc, uint64_t seed,

@@ -28,6 +28,21 @@ from . import tokengate as tg
 STAGES = ("gate", "select", "gather", "qkv", "rope", "attn")
 
 
+def nvtx_marks() -> Callable[[str], None]:
+    """A `mark` hook for GatedPrefillLayer.run that wraps each step in an NVTX range named
+    "tg:<step>" (so a profiler can select one step, e.g. ncu --nvtx --nvtx-include "tg:attn/")."""
+    open_range = [False]
+
+    def mark(name: str) -> None:
+        if open_range[0]:
+            torch.cuda.nvtx.range_pop()
+        open_range[0] = name != "end"
+        if open_range[0]:
+            torch.cuda.nvtx.range_push("tg:" + name)
+
+    return mark
+
+
 class GatedPrefillLayer:
     def __init__(self, N: int, doc_begin: int, doc_end: int, k_doc: int, W1: torch.Tensor, w2: torch.Tensor,
                  Wqkv: torch.Tensor, Hq: int, Hkv: int, d_h: int, gain: torch.Tensor, tau: float,

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libtokengate.so")
 
 TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_CUDA, TG_ERR_TIMEOUT = range(5)
 TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL, TG_OP_DECODE = range(5)
+TG_STATUS_SELECT_TIMEOUT, TG_STATUS_GATE_TIMEOUT, TG_STATUS_ATTENTION_TIMEOUT, TG_STATUS_DECODE_TIMEOUT = 1, 2, 4, 8
 
 _lib = None
 
@@ -54,10 +55,11 @@ def lib() -> ctypes.CDLL:
         L.tg_gated_attention.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp,
                                          vp, sz, vp]
         L.tg_gated_decode.argtypes = [vp, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp, vp, sz, vp]
+        L.tg_debug_set_select_wait_limit.argtypes = [ctypes.c_uint64]
         L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
         for fn in ("tg_gate_score", "tg_topk_select", "tg_topk_select_noalloc", "tg_random_select", "tg_gather_compact",
                    "tg_rope_apply",
-                   "tg_gated_attention", "tg_gated_decode", "tg_device_status"):
+                   "tg_gated_attention", "tg_gated_decode", "tg_debug_set_select_wait_limit", "tg_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -262,6 +264,11 @@ def tg_gated_decode(q, k_cache, v_cache, out, workspace, s_cache=None, gain=None
         Hq, Hkv, d_h, _ptr(s_cache), _ptr(gain), tau, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)))
     return out
+
+
+def tg_debug_set_select_wait_limit(ns: int) -> None:
+    """Test hook: the select's grid-barrier time limit on the current device (0 = the default)."""
+    _check("tg_debug_set_select_wait_limit", lib().tg_debug_set_select_wait_limit(ctypes.c_uint64(ns)))
 
 
 def tg_device_status(workspace, stream=None) -> int:

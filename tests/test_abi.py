@@ -92,3 +92,33 @@ def test_argument_errors_before_launch(lib):
                                       vp(16), None, vp(256), 1 << 20, None) == tg.TG_ERR_INVALID_ARG
     assert lib.tg_gated_attention(vp(16), 128, vp(16), 128, vp(16), 128, 5, 2, 2, 64, None, None, 1.0,
                                   vp(16), None, vp(256), 256, None) == tg.TG_ERR_INVALID_ARG  # workspace too small
+
+
+def test_decode_and_random_select_argument_errors(lib):
+    vp = ctypes.c_void_p
+    INV, UNS = tg.TG_ERR_INVALID_ARG, tg.TG_ERR_UNSUPPORTED
+    big = tg.tg_workspace_bytes(tg.TG_OP_DECODE, 0, 64, 0)
+    assert big > 0
+
+    def dec(q=16, ldk=1024, ldv=1024, T=100, Hq=16, Hkv=8, d_h=128, tau=1.0, ws_bytes=big, out=16):
+        return lib.tg_gated_decode(vp(q), vp(4096), ldk, vp(8192), ldv, T, Hq, Hkv, d_h, None, None, tau,
+                                   vp(out) if out else None, None, vp(256), ws_bytes, None)
+
+    assert dec(T=0) == INV
+    assert dec(Hq=12, Hkv=8) == INV                 # Hq % Hkv
+    assert dec(tau=float("nan")) == INV
+    assert dec(out=0) == INV                        # no output
+    assert dec(d_h=96) == UNS
+    assert dec(Hq=16, Hkv=1, ldk=128, ldv=128) == UNS   # 16 query heads per KV head
+    assert dec(Hq=128, Hkv=128, ldk=128 * 128, ldv=128 * 128, ws_bytes=1 << 30) == UNS   # Hkv > 64
+    assert dec(q=24) == INV                         # q not 16-byte aligned
+    assert dec(ldk=1028) == INV                     # stride not a multiple of 8 elements
+    assert dec(ldv=512) == INV                      # stride shorter than a row
+    assert dec(ws_bytes=tg.tg_workspace_bytes(tg.TG_OP_DECODE, 0, 16, 0) - 16) == INV
+    rs = lib.tg_random_select
+    assert rs(10, 2, 11, 1, 7, vp(16), vp(256), 1 << 20, None) == INV      # span past N
+    assert rs(10, 2, 8, -1, 7, vp(16), vp(256), 1 << 20, None) == INV      # negative budget
+    assert rs(10, 2, 8, 3, 7, None, vp(256), 1 << 20, None) == INV         # no output
+    assert rs(1000, 0, 900, 10, 7, vp(16), vp(256), 16, None) == INV       # workspace too small
+    assert rs(1000, 0, 900, 10, 7, vp(16), None, 1 << 20, None) == INV     # no workspace
+    assert rs(0, 0, 0, 5, 7, None, None, 0, None) == tg.TG_OK              # nothing to keep

@@ -17,6 +17,7 @@ import torch
 from learned_token_pruning_tg_b200 import synth
 from learned_token_pruning_tg_b200 import tokengate as tg
 from tests import oracle_pool
+from tests.guards import guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -41,12 +42,14 @@ def run_gpu(d, fused=False, want_lse=True, use_bias=True):
         v = buf[:, (Hq + Hkv) * d_h:].view(K, Hkv, d_h)
     else:
         q, k, v = d.q.cuda(), d.k.cuda(), d.v.cuda()
-    out = torch.full((K, Hq, d_h), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out, check = guarded((K, Hq, d_h), torch.bfloat16)   # guard bands around the output
+    out.fill_(float("nan"))                                # and every element must be written
     lse = torch.full((Hq, K), float("nan"), device="cuda") if want_lse else None
     ws = tg.new_workspace(K, Hkv * d_h, op=tg.TG_OP_ATTENTION)
     tg.tg_gated_attention(q, k, v, out, ws, s_kept=d.s.cuda() if use_bias else None,
                           gain=d.gain.cuda() if use_bias else None, tau=d.tau, lse=lse)
     torch.cuda.synchronize()
+    check()
     assert tg.tg_device_status(ws) == 0
     return out.float().cpu().numpy(), (lse.cpu().numpy() if want_lse else None)
 

@@ -14,6 +14,7 @@ import torch
 import oracle
 from learned_token_pruning_tg_b200 import synth
 from learned_token_pruning_tg_b200 import tokengate as tg
+from tests.guards import guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -38,12 +39,15 @@ def run_decode(d, strided=False, use_bias=True):
         v = buf[:, Hkv * d_h: 2 * Hkv * d_h].view(T, Hkv, d_h)
     else:
         k, v = d.k.cuda(), d.v.cuda()
-    out = torch.full((Hq, d_h), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out, check = guarded((Hq, d_h), torch.bfloat16)      # guard bands around the output
+    out.fill_(float("nan"))
     lse = torch.full((Hq,), float("nan"), device="cuda")
     ws = tg.new_workspace(0, Hq, op=tg.TG_OP_DECODE)
     tg.tg_gated_decode(q, k, v, out, ws, s_cache=d.s.cuda() if use_bias else None,
                        gain=d.gain.cuda() if use_bias else None, tau=d.tau, lse=lse)
     torch.cuda.synchronize()
+    check()
+    assert tg.tg_device_status(ws) == 0
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
 

@@ -10,6 +10,7 @@ import torch
 import oracle
 from learned_token_pruning_tg_b200 import synth
 from learned_token_pruning_tg_b200 import tokengate as tg
+from tests.guards import guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -76,11 +77,12 @@ def test_gather_bit_exact(N, d, K, ld_pad):
     pos_in = (torch.arange(N, dtype=torch.int32) * 3 + 1)
     s = torch.randn(N, generator=g)
     hd = h_full.cuda()[:, :d]
-    h_out = torch.empty(K, d, dtype=torch.bfloat16, device="cuda")
-    pos_out = torch.empty(K, dtype=torch.int32, device="cuda")
-    s_out = torch.empty(K, dtype=torch.float32, device="cuda")
+    h_out, check_h = guarded((K, d), torch.bfloat16)      # guard bands around every output
+    pos_out, check_p = guarded((K,), torch.int32)
+    s_out, check_s = guarded((K,), torch.float32)
     tg.tg_gather_compact(hd, idx.cuda(), h_out, pos_out, pos_in=pos_in.cuda(), scores=s.cuda(), s_out=s_out)
     torch.cuda.synchronize()
+    check_h(), check_p(), check_s()
     bits = h_full[:, :d].contiguous().view(torch.int16).numpy().view(np.uint16)
     want_h, want_pos, want_s = oracle.gather_compact(bits, idx.numpy(), pos_in=pos_in.numpy(), scores=s.numpy())
     assert np.array_equal(h_out.cpu().view(torch.int16).numpy().view(np.uint16), want_h)
