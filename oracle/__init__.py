@@ -37,6 +37,9 @@ def lib():
         L.tgo_rope.restype = i32
         L.tgo_gated_attention.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, dbl, vp, i64, vp, vp]
         L.tgo_gated_attention.restype = i32
+        L.tgo_gated_attention_backward.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, dbl, vp,
+                                                   vp, vp, vp, vp, vp, vp]
+        L.tgo_gated_attention_backward.restype = i32
         L.tgo_random_select.argtypes = [i64, i64, i64, i64, ctypes.c_uint64, vp]
         L.tgo_random_select.restype = i64
         L.tgo_splitmix64_stream.argtypes = [ctypes.c_uint64, i64, vp]
@@ -173,5 +176,28 @@ def gated_attention(q, k, v, s=None, g=None, tau=1.0, pos=None, rows=None, want_
     return out
 
 
+def gated_attention_backward(q, k, v, dout, s=None, g=None, tau=1.0, pos=None):
+    """Gradients of sum(dout * out) of gated_attention with respect to every input.
+    q [K,Hq,d_h], k/v [K,Hkv,d_h], dout [K,Hq,d_h] fp32 values; returns a dict of fp64 arrays
+    dq [K,Hq,d_h], dk, dv [K,Hkv,d_h], ds [K], dg [Hq] and the float dtau."""
+    q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+    K, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    s, g = _f32(s), _f32(g)
+    pos = None if pos is None else np.ascontiguousarray(pos, dtype=np.int32)
+    dq = np.empty((max(K, 1), Hq, d_h), dtype=np.float64)
+    dk = np.empty((max(K, 1), Hkv, d_h), dtype=np.float64)
+    dv = np.empty((max(K, 1), Hkv, d_h), dtype=np.float64)
+    ds = np.empty(max(K, 1), dtype=np.float64)
+    dg = np.empty(Hq, dtype=np.float64)
+    dtau = np.empty(1, dtype=np.float64)
+    rc = lib().tgo_gated_attention_backward(_p(q), _p(k), _p(v), K, Hq, Hkv, d_h, _p(pos), _p(s), _p(g),
+                                            float(tau), _p(dout), _p(dq), _p(dk), _p(dv), _p(ds), _p(dg),
+                                            _p(dtau))
+    if rc != 0:
+        raise ValueError("tgo_gated_attention_backward: bad arguments")
+    return {"dq": dq[:K], "dk": dk[:K], "dv": dv[:K], "ds": ds[:K], "dg": dg, "dtau": float(dtau[0])}
+
+
 __all__ = ["lib", "kept_count", "round_bf16", "gate_score", "topk_select", "topk_threshold",
-           "gather_compact", "rope", "gated_attention"]
+           "gather_compact", "rope", "gated_attention", "gated_attention_backward"]

@@ -385,3 +385,121 @@ int tgo_gated_attention(const float* q, const float* k, const float* v,
     free(logit);
     return 0;
 }
+
+/* Backward of the token-gated logit and the softmax-weighted sum, one query
+ * row and head at a time, straight from the chain rule:
+ *   P_c   = exp(l_c - lse)                      (softmax over visible keys)
+ *   out   = sum_c P_c v_c
+ *   dP_c  = dout . v_c                          (d loss / d P_c)
+ *   dl_c  = P_c (dP_c - sum_c' P_c' dP_c')      (softmax Jacobian)
+ *   l_c   = tau (q . k_c) / sqrt(d_h) + g_h s_c, so
+ *   dq   += dl_c tau / sqrt(d_h) k_c,   dk_c += dl_c tau / sqrt(d_h) q,
+ *   dv_c += P_c dout,                    ds_c += dl_c g_h,
+ *   dg_h += dl_c s_c,                    dtau += dl_c (q . k_c) / sqrt(d_h). */
+int tgo_gated_attention_backward(const float* q, const float* k, const float* v,
+                                 int64_t K, int Hq, int Hkv, int d_h,
+                                 const int32_t* pos, const float* s, const float* g,
+                                 double tau, const float* dout,
+                                 double* dq, double* dk, double* dv,
+                                 double* ds, double* dg, double* dtau)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || K < 0 || Hq <= 0 || Hkv <= 0 || d_h <= 0 ||
+        (Hq % Hkv))
+        return -1;
+    int group = Hq / Hkv;
+    double inv_sqrt_d = 1.0 / sqrt((double)d_h);
+    double scale = tau * inv_sqrt_d;
+    memset(dq, 0, sizeof(double) * (size_t)K * Hq * d_h);
+    memset(dk, 0, sizeof(double) * (size_t)K * Hkv * d_h);
+    memset(dv, 0, sizeof(double) * (size_t)K * Hkv * d_h);
+    if (ds)
+        memset(ds, 0, sizeof(double) * (size_t)K);
+    if (dg)
+        memset(dg, 0, sizeof(double) * (size_t)Hq);
+    double dtau_sum = 0.0;
+    size_t n = (size_t)(K > 0 ? K : 1);
+    double* dot = (double*)malloc(sizeof(double) * n);   /* q . k_c */
+    double* prob = (double*)malloc(sizeof(double) * n);  /* logit, then P_c */
+    double* dprob = (double*)malloc(sizeof(double) * n); /* dP_c */
+    if (!dot || !prob || !dprob) {
+        free(dot);
+        free(prob);
+        free(dprob);
+        return -1;
+    }
+
+    for (int h = 0; h < Hq; ++h) {
+        int kv_head = h / group;
+        double gain = g ? (double)g[h] : 0.0;
+        for (int64_t r = 0; r < K; ++r) {
+            const float* qr = q + (r * Hq + h) * (int64_t)d_h;
+            const float* dor = dout + (r * Hq + h) * (int64_t)d_h;
+            /* keys 0..last are the candidates; key c is visible iff VISIBLE(c) */
+#define VISIBLE(c) (pos ? (pos[(c)] <= pos[r]) : ((c) <= r))
+
+            /* forward again: logits of the visible keys, their maximum, the softmax */
+            double m = -INFINITY;
+            for (int64_t c = 0; c < K; ++c) {
+                if (!VISIBLE(c))
+                    continue;
+                const float* kc = k + (c * Hkv + kv_head) * (int64_t)d_h;
+                double d = 0.0;
+                for (int t = 0; t < d_h; ++t)
+                    d += (double)qr[t] * (double)kc[t];
+                dot[c] = d;
+                prob[c] = scale * d + gain * (s ? (double)s[c] : 0.0);
+                if (prob[c] > m)
+                    m = prob[c];
+            }
+            double denom = 0.0;
+            for (int64_t c = 0; c < K; ++c) {
+                if (!VISIBLE(c))
+                    continue;
+                prob[c] = exp(prob[c] - m);
+                denom += prob[c];
+            }
+
+            /* P_c, d loss / d P_c, and the P-weighted mean of the latter */
+            double mean = 0.0;
+            for (int64_t c = 0; c < K; ++c) {
+                if (!VISIBLE(c))
+                    continue;
+                prob[c] /= denom;
+                const float* vc = v + (c * Hkv + kv_head) * (int64_t)d_h;
+                double d = 0.0;
+                for (int t = 0; t < d_h; ++t)
+                    d += (double)dor[t] * (double)vc[t];
+                dprob[c] = d;
+                mean += prob[c] * d;
+            }
+
+            /* through the softmax and the logit to every input */
+            double* dqr = dq + (r * Hq + h) * (int64_t)d_h;
+            for (int64_t c = 0; c < K; ++c) {
+                if (!VISIBLE(c))
+                    continue;
+                double dl = prob[c] * (dprob[c] - mean);
+                const float* kc = k + (c * Hkv + kv_head) * (int64_t)d_h;
+                double* dkc = dk + (c * Hkv + kv_head) * (int64_t)d_h;
+                double* dvc = dv + (c * Hkv + kv_head) * (int64_t)d_h;
+                for (int t = 0; t < d_h; ++t) {
+                    dqr[t] += dl * scale * (double)kc[t];
+                    dkc[t] += dl * scale * (double)qr[t];
+                    dvc[t] += prob[c] * (double)dor[t];
+                }
+                if (ds)
+                    ds[c] += dl * gain;
+                if (dg)
+                    dg[h] += dl * (s ? (double)s[c] : 0.0);
+                dtau_sum += dl * dot[c] * inv_sqrt_d;
+            }
+#undef VISIBLE
+        }
+    }
+    if (dtau)
+        *dtau = dtau_sum;
+    free(dot);
+    free(prob);
+    free(dprob);
+    return 0;
+}

@@ -113,6 +113,26 @@ int tgo_gated_attention(const float* q, const float* k, const float* v,
                         double tau, const int64_t* rows, int64_t n_rows,
                         double* out, double* lse);
 
+/* Gradients of token-gated attention, fp64, over all K rows (test
+ * infrastructure for the backward kernels).  The pages give the reason the
+ * bias exists -- it is the scorer's gradient path, and the per-head gain and
+ * the temperature are learned (aiproducthub.cn article, paragraph 事件详情;
+ * aisight.pl article, section Jak to działa; chathome.org article, section
+ * トークンゲート付きアテンションとは) -- so the quantities are the derivatives
+ * of the loss sum_{r,h,t} dout[r,h,t] * out[r,h,t] with respect to q, k, v,
+ * the kept scores s, the gains g and tau, by the chain rule through the
+ * forward of tgo_gated_attention (same arguments, same visibility rule).
+ * dout: [K, Hq, d_h].  Outputs: dq [K, Hq, d_h], dk and dv [K, Hkv, d_h],
+ * ds [K], dg [Hq], dtau [1]; ds, dg, dtau may be NULL.  s NULL or g NULL
+ * means 0 (their gradients are still defined and returned).
+ * Returns 0, or -1 on bad arguments. */
+int tgo_gated_attention_backward(const float* q, const float* k, const float* v,
+                                 int64_t K, int Hq, int Hkv, int d_h,
+                                 const int32_t* pos, const float* s, const float* g,
+                                 double tau, const float* dout,
+                                 double* dq, double* dk, double* dv,
+                                 double* ds, double* dg, double* dtau);
+
 /* Round an fp32 value to the nearest bf16 (ties to even), returned widened to
  * fp32.  NaN stays NaN.  Exposed so tests can state bf16 inputs exactly. */
 float tgo_round_bf16(float x);

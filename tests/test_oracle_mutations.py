@@ -29,6 +29,13 @@ MUTATIONS = {
     "attn_scale_no_sqrt": ("tau / sqrt((double)d_h)", "tau / (double)d_h"),
     "rope_sign": ("o[t] = x1 * c - x2 * s;", "o[t] = x1 * c + x2 * s;"),
     "rope_pairing": ("double x1 = xr[t], x2 = xr[t + half];", "double x1 = xr[2 * t], x2 = xr[2 * t + 1];"),
+    "bwd_drop_softmax_mean": ("double dl = prob[c] * (dprob[c] - mean);", "double dl = prob[c] * dprob[c];"),
+    "bwd_dk_wrong_operand": ("dkc[t] += dl * scale * (double)qr[t];", "dkc[t] += dl * scale * (double)kc[t];"),
+    "bwd_dv_uses_dl": ("dvc[t] += prob[c] * (double)dor[t];", "dvc[t] += dl * (double)dor[t];"),
+    "bwd_dtau_no_sqrt": ("dtau_sum += dl * dot[c] * inv_sqrt_d;", "dtau_sum += dl * dot[c];"),
+    "bwd_ds_no_gain": ("ds[c] += dl * gain;", "ds[c] += dl;"),
+    "bwd_kv_head": ("int kv_head = h / group;", "int kv_head = h % Hkv;"),
+    "bwd_unnormalised_p": ("prob[c] /= denom;", "(void)denom;"),
     "gather_pos_index": ("pos_out[r] = pos_in ? pos_in[i] : (int32_t)i;",
                          "pos_out[r] = pos_in ? pos_in[r] : (int32_t)i;"),
 }
@@ -48,6 +55,6 @@ def test_pins_catch_mutation(name, tmp_path):
     env = dict(os.environ, TG_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         "tests/test_oracle_gate.py", "tests/test_oracle_select.py",
-                        "tests/test_oracle_attention.py"],
+                        "tests/test_oracle_attention.py", "tests/test_oracle_attention_backward.py"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"no pin caught mutation {name}:\n{r.stdout[-2000:]}"
