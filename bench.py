@@ -667,6 +667,66 @@ def run_decode_layer(args, rank, world, local_rank):
             "gpu_launches": reps, "device_status": tg.tg_device_status(ws)}
 
 
+def run_backward(args, rank, world, local_rank):
+    """The gradients of the gated attention above the gate at the 128k workload's kept set (K = 4608,
+    16 query / 8 KV heads of 128): one tg_gated_attention_backward call (four launches) per step, after
+    one forward that provides the output and log-sum-exp.  The inputs (75 MB) fit in L2, so a 512 MB
+    buffer is written between timed calls; each call is timed alone with its own events."""
+    from learned_token_pruning_tg_b200 import tokengate as tg
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    K, Hq, Hkv, d_h = WORKLOAD.K, WORKLOAD.Hq, WORKLOAD.Hkv, WORKLOAD.d_h
+    d = synth.qkv(K, Hq, Hkv, d_h, seed=4608 + rank, heavy_frac=0.03)
+    dout = synth.grad_out(K, Hq, d_h, seed=4609 + rank).to(dev)
+    q, k, v, s, g = d.q.to(dev), d.k.to(dev), d.v.to(dev), d.s.to(dev), d.gain.to(dev)
+    out = torch.empty(K, Hq, d_h, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(Hq, K, dtype=torch.float32, device=dev)
+    ws_f = tg.new_workspace(K, Hkv * d_h, op=tg.TG_OP_ATTENTION, device=dev)
+    tg.tg_gated_attention(q, k, v, out, ws_f, s_kept=s, gain=g, tau=d.tau, lse=lse)
+    ws = tg.new_workspace(K, Hq, Hkv, op=tg.TG_OP_ATTENTION_BACKWARD, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ds = torch.empty(K, dtype=torch.float32, device=dev)
+    dg = torch.empty(Hq, dtype=torch.float32, device=dev)
+    dtau = torch.empty(1, dtype=torch.float32, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def call():
+        tg.tg_gated_attention_backward(q, k, v, out, dout, lse, dq, dk, dv, ws, s_kept=s, gain=g, tau=d.tau,
+                                       ds=ds, dg=dg, dtau=dtau)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    reps = max(3, min(args.steps, 50))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with ClockSampler(dev.index) as clk:
+        for e0, e1 in ev:
+            flush.fill_(1)
+            e0.record()
+            call()
+            e1.record()
+        torch.cuda.synchronize()
+    us = reduce_max(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps * 1e3, dev)
+    if rank != 0:
+        return None
+    pairs = K * (K + 1) / 2
+    flop = 5 * 2 * pairs * d_h * Hq     # S, dP, dV, dK, dQ over the causal pairs (S and dP recomputed: 7)
+    peaks = load_peaks()
+    tf = flop / (us * 1e-6) / 1e12
+    return {"metric": "gated attention backward (dq, dk, dv, ds, dg, dtau), 128k workload's kept set",
+            "value": us, "unit": "us", "n_gpus": world, "steps": reps, "warmup": args.warmup,
+            "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded q, k, v, dO; 3% heavy rows)",
+            "config": {"workload": "qwen3-1.7b-128k kept set", "K": K, "Hq": Hq, "Hkv": Hkv, "d_h": d_h,
+                       "l2": "inputs 75 MB < L2: 512 MB written between timed calls"},
+            "impl": "tokengate",
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "whole backward (prep, dq, dkdv, finish)",
+                         "algorithmic_flop": flop},
+            "clocks": clk.summary(), "gpu_launches": 4 * reps, "device_status": tg.tg_device_status(ws)}
+
+
 def main():
     faulthandler.enable()
     ap = argparse.ArgumentParser()
@@ -681,6 +741,8 @@ def main():
                     help="time one layer's decoding step over a 64k cache (the decode kernel alone)")
     ap.add_argument("--decode", action="store_true",
                     help="time one decoding step's attention over a pruned 28-layer cache (and an unpruned one)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the gated attention backward at the 128k workload's kept set")
     ap.add_argument("--stack", action="store_true",
                     help="time the pruned prefill through a 28-layer stack (and the unpruned one) instead")
     args = ap.parse_args()
@@ -700,7 +762,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        run = (run_stack if args.stack else run_decode if args.decode else
+        run = (run_stack if args.stack else run_decode if args.decode else run_backward if args.backward else
                run_decode_layer if args.decode_layer else run_tokengate)
         res = run(args, rank, world, local_rank)
         if res is not None:

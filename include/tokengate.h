@@ -70,7 +70,8 @@ typedef enum {
     TG_OP_SELECT = 1,
     TG_OP_ATTENTION = 2,
     TG_OP_ALL = 3, /* one buffer usable by every call above */
-    TG_OP_DECODE = 4
+    TG_OP_DECODE = 4,
+    TG_OP_ATTENTION_BACKWARD = 5
 } tg_op;
 
 /* Bits of the device status word (first 4 bytes of the workspace). */
@@ -78,6 +79,7 @@ typedef enum {
 #define TG_STATUS_GATE_TIMEOUT 0x2u
 #define TG_STATUS_ATTENTION_TIMEOUT 0x4u
 #define TG_STATUS_DECODE_TIMEOUT 0x8u
+#define TG_STATUS_BACKWARD_TIMEOUT 0x10u
 
 /* Static description of a status code.  Never NULL. */
 const char* tg_status_string(tg_status status);
@@ -98,6 +100,8 @@ int64_t tg_kept_count(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_d
  *   TG_OP_ALL        every op above with these N, d, d_g (attention over at
  *                    most N tokens whose V rows are at most d wide)
  *   TG_OP_DECODE     tg_gated_decode with d = Hq query heads (N, d_g unused)
+ *   TG_OP_ATTENTION_BACKWARD  tg_gated_attention_backward with N = K kept
+ *                    tokens, d = Hq query heads, d_g = Hkv KV heads
  * Returns 0 for bad arguments. */
 size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g);
 
@@ -238,6 +242,41 @@ tg_status tg_gated_decode(const tg_bf16* q, const tg_bf16* k_cache, int64_t ld_k
                           int64_t ld_v, int64_t T, int32_t Hq, int32_t Hkv, int32_t d_h,
                           const float* s_cache, const float* gain, float tau, tg_bf16* out, float* lse,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Gradients of tg_gated_attention (the gradient path the key bias gives the
+ * scorer, with the learned per-head gain and temperature: aiproducthub.cn
+ * article, paragraph 事件详情; aisight.pl article, section Jak to działa;
+ * chathome.org article, section トークンゲート付きアテンションとは).  With
+ * l_{r,c} = tau q_r.k_c / sqrt(d_h) + g_h s_c (c <= r), P = softmax_c(l),
+ * O = P V, an upstream gradient dO and D_r = dO_r . O_r:
+ *   dl = P (dO V^T - D)
+ *   dq = tau / sqrt(d_h) dl K,   dk = tau / sqrt(d_h) dl^T Q,   dv = P^T dO
+ *   ds_c = sum_h g_h sum_r dl_{h,r,c},   dg_h = sum_{r,c} dl_{h,r,c} s_c,
+ *   dtau = sum_{h,r,c} dl_{h,r,c} q_r.k_c / sqrt(d_h)
+ * (GQA: dk and dv sum over the query heads of each KV head).
+ * q, k, v, K, Hq, Hkv, d_h, s_kept, gain, tau: as given to the forward call.
+ * out: the forward's output, dout: the gradient of the loss with respect to
+ * it, both [K, Hq, d_h] bf16 dense; lse: the forward's [Hq, K] fp32
+ * log-sum-exp (required).  Outputs: dq [K, Hq, d_h], dk and dv [K, Hkv, d_h]
+ * bf16 dense; ds [K], dg [Hq], dtau [1] fp32, each may be NULL.  Without a
+ * bias (s_kept or gain NULL) the missing one counts as 0: ds is then 0 and dg
+ * is still defined.
+ * workspace: tg_workspace_bytes(TG_OP_ATTENTION_BACKWARD, K, Hq, Hkv) bytes,
+ * 16-byte aligned; every part of it is rewritten by each call (no zeroing).
+ * Supported: d_h in {64, 128}, Hq / Hkv <= 8, tau > 0; every bf16 tensor
+ * 16-byte aligned, strides multiples of 8 elements.  Four launches: D and the
+ * log2 lse; the dq kernel (per query tile and head); the dk/dv kernel (per key
+ * tile and KV head, which also sums ds and dg); the final fixed-order sums.
+ * Both main kernels recompute S on the tensor cores (tcgen05, TMEM
+ * accumulators, TMA-staged tiles) with P and dS in bf16.  Deterministic: the
+ * same inputs give the same bits.  Waits are bounded
+ * (TG_STATUS_BACKWARD_TIMEOUT in the workspace's status word). */
+tg_status tg_gated_attention_backward(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
+                                      const tg_bf16* v, int64_t ld_v, int64_t K, int32_t Hq, int32_t Hkv,
+                                      int32_t d_h, const float* s_kept, const float* gain, float tau,
+                                      const tg_bf16* out, const tg_bf16* dout, const float* lse,
+                                      tg_bf16* dq, tg_bf16* dk, tg_bf16* dv, float* ds, float* dg,
+                                      float* dtau, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Test hook (fault injection without a fault): sets the time limit of the
  * grid barrier inside tg_topk_select, tg_topk_select_noalloc and

@@ -182,6 +182,12 @@ def qkv(K: int, Hq: int, Hkv: int, d_h: int, seed: int, score_std=0.6, tau_range
                gain=gain, tau=tau, pos=pos)
 
 
+def grad_out(K: int, Hq: int, d_h: int, seed: int, std: float = 1.0) -> torch.Tensor:
+    """An upstream gradient for the attention output: [K, Hq, d_h] bf16 ~ N(0, std^2)."""
+    g = _gen(seed)
+    return (torch.randn(K, Hq, d_h, generator=g) * std).to(torch.bfloat16)
+
+
 def score_vector(N: int, seed: int, kind: str = "normal") -> torch.Tensor:
     """fp32 score vectors for select-only stress cases.
 

@@ -18,8 +18,9 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtokengate.so")
 
 TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_CUDA, TG_ERR_TIMEOUT = range(5)
-TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL, TG_OP_DECODE = range(5)
+TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL, TG_OP_DECODE, TG_OP_ATTENTION_BACKWARD = range(6)
 TG_STATUS_SELECT_TIMEOUT, TG_STATUS_GATE_TIMEOUT, TG_STATUS_ATTENTION_TIMEOUT, TG_STATUS_DECODE_TIMEOUT = 1, 2, 4, 8
+TG_STATUS_BACKWARD_TIMEOUT = 16
 
 _lib = None
 
@@ -55,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.tg_gated_attention.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp,
                                          vp, sz, vp]
         L.tg_gated_decode.argtypes = [vp, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp, vp, sz, vp]
+        L.tg_gated_attention_backward.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp,
+                                                  vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.tg_debug_set_select_wait_limit.argtypes = [ctypes.c_uint64]
         L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
         for fn in ("tg_gate_score", "tg_topk_select", "tg_topk_select_noalloc", "tg_random_select", "tg_gather_compact",
@@ -240,6 +243,32 @@ def tg_gated_attention(q, k, v, out, workspace, s_kept=None, gain=None, tau: flo
         d_h, _ptr(s_kept), _ptr(gain), tau, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)))
     return out
+
+
+def tg_gated_attention_backward(q, k, v, out, dout, lse, dq, dk, dv, workspace, s_kept=None, gain=None,
+                                tau: float = 1.0, ds=None, dg=None, dtau=None, stream=None):
+    """Gradients of tg_gated_attention: out, dout [K, Hq, d_h] and lse [Hq, K] from the forward call;
+    writes dq [K, Hq, d_h], dk and dv [K, Hkv, d_h] (bf16) and, when given, ds [K], dg [Hq], dtau [1]
+    (fp32)."""
+    for t, n, r in ((q, "q", 3), (k, "k", 3), (v, "v", 3), (out, "out", 3), (dout, "dout", 3), (dq, "dq", 3),
+                    (dk, "dk", 3), (dv, "dv", 3)):
+        _req(t, n, torch.bfloat16, r)
+    for t, n, r in ((lse, "lse", 2), (s_kept, "s_kept", 1), (gain, "gain", 1), (ds, "ds", 1), (dg, "dg", 1),
+                    (dtau, "dtau", 1)):
+        _req(t, n, torch.float32, r)
+    if lse is None:
+        raise ValueError("lse (the forward's log-sum-exp) is required")
+    K, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    for t, n, shape in ((out, "out", (K, Hq, d_h)), (dout, "dout", (K, Hq, d_h)), (dq, "dq", (K, Hq, d_h)),
+                        (dk, "dk", (K, Hkv, d_h)), (dv, "dv", (K, Hkv, d_h)), (lse, "lse", (Hq, K))):
+        if not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError(f"{n} must be a contiguous {list(shape)} tensor")
+    _check("tg_gated_attention_backward", lib().tg_gated_attention_backward(
+        _ptr(q), _row_stride(q, "q"), _ptr(k), _row_stride(k, "k"), _ptr(v), _row_stride(v, "v"), K, Hq, Hkv,
+        d_h, _ptr(s_kept), _ptr(gain), tau, _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(ds), _ptr(dg), _ptr(dtau), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 def tg_gated_decode(q, k_cache, v_cache, out, workspace, s_cache=None, gain=None, tau: float = 1.0, lse=None,

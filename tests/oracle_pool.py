@@ -45,3 +45,28 @@ def gated_attention(q, k, v, s=None, g=None, tau=1.0, pos=None, rows=None, n_chu
     parts = np.array_split(rows, n)
     futs = [pool().submit(_attn_chunk, q, k, v, s, g, tau, pos, p) for p in parts if len(p)]
     return np.concatenate([f.result() for f in futs])
+
+
+def _bwd_group(q, k, v, dout, s, g, tau):
+    import oracle
+    return oracle.gated_attention_backward(q, k, v, dout, s=s, g=g, tau=tau)
+
+
+def gated_attention_backward(q, k, v, dout, s=None, g=None, tau=1.0):
+    """Oracle backward split by KV head: each worker runs one KV head and its query heads (an
+    independent problem), and the parts are put back together (ds and dtau summed)."""
+    K, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    futs = [pool().submit(_bwd_group, np.ascontiguousarray(q[:, j * G:(j + 1) * G]),
+                          np.ascontiguousarray(k[:, j:j + 1]), np.ascontiguousarray(v[:, j:j + 1]),
+                          np.ascontiguousarray(dout[:, j * G:(j + 1) * G]), s,
+                          None if g is None else np.ascontiguousarray(g[j * G:(j + 1) * G]), tau)
+            for j in range(Hkv)]
+    parts = [f.result() for f in futs]
+    return {"dq": np.concatenate([p["dq"] for p in parts], axis=1),
+            "dk": np.concatenate([p["dk"] for p in parts], axis=1),
+            "dv": np.concatenate([p["dv"] for p in parts], axis=1),
+            "ds": np.sum([p["ds"] for p in parts], axis=0),
+            "dg": np.concatenate([p["dg"] for p in parts]),
+            "dtau": float(np.sum([p["dtau"] for p in parts]))}

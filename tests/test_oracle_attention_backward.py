@@ -121,3 +121,15 @@ def test_backward_grouped_heads_equal_duplicated_kv_heads():
     np.testing.assert_allclose(d["dv"].reshape(K, Hkv, G, d_h).sum(axis=2), b["dv"], rtol=1e-12, atol=1e-13)
     for key in ("dq", "ds", "dg"):
         np.testing.assert_allclose(d[key], b[key], rtol=1e-12, atol=1e-13)
+
+
+def test_backward_split_by_kv_head_equals_whole():
+    from tests import oracle_pool
+    rng = np.random.default_rng(13)
+    K, Hq, Hkv, d_h, tau = 30, 6, 3, 8, 0.8
+    x = grid_inputs(rng, K, Hq, Hkv, d_h)
+    whole = oracle.gated_attention_backward(x["q"], x["k"], x["v"], x["dout"], s=x["s"], g=x["g"], tau=tau)
+    split = oracle_pool.gated_attention_backward(x["q"], x["k"], x["v"], x["dout"], s=x["s"], g=x["g"], tau=tau)
+    for key in ("dq", "dk", "dv", "ds", "dg"):
+        np.testing.assert_allclose(split[key], whole[key], rtol=1e-12, atol=1e-14)
+    assert abs(split["dtau"] - whole["dtau"]) <= 1e-12 * max(1.0, abs(whole["dtau"]))
