@@ -34,8 +34,11 @@
 //   bwd_finish_kernel ds over the KV heads, dg over the key tiles, dtau over the
 //                     dq CTAs, in a fixed order (deterministic)
 // Warps of both big kernels: 0 TMA, 1 TMEM allocation and the single MMA-issuing
-// thread, 2 the bias operands, 3-10 two warpgroups that split each tile's 128
-// columns (one row per thread, 64 columns each).  P and dS are bf16 because dO,
+// thread, 2 the bias operands, 3-10 two softmax warpgroups (one row per thread).
+// The dq kernel's warpgroups split each tile's 128 keys (64 each); the dk/dv kernel
+// takes each step's 128 queries in two 64-query halves with their own S^T / dP^T
+// columns, so one half's products overlap the other half's softmax (32 queries of
+// a half per warpgroup).  P and dS are bf16 because dO,
 // Q and K are (kind::f16 multiplies operands of one type).  Every wait is bounded
 // (TG_STATUS_BACKWARD_TIMEOUT).
 #include <algorithm>
@@ -50,6 +53,11 @@ constexpr int kB = 128;  // rows of every tile (queries or keys)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kAugTile = 4096;   // 128 rows x 16 bf16, no-swizzle K-major
 constexpr int kMaxGroup = 8;     // query heads per KV head
+constexpr int kHalf = 64;        // the dk/dv kernel takes each step's 128 query columns in two halves
+constexpr int kWG = 2;           // softmax warpgroups; each takes kWGCols of a half's 64 columns
+constexpr int kWGCols = kHalf / kWG;
+constexpr int kSoftWarps = 4 * kWG;
+constexpr int kThreads = 32 * (3 + kSoftWarps);
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -105,50 +113,56 @@ __device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, volatile i
 __device__ __forceinline__ uint32_t kstep_off(int k) {
     return static_cast<uint32_t>(((k >> 2) * (kB * 128) + (k & 3) * 32) >> 4);
 }
-// TMEM column of the A operand for K-step k of a bf16 P / dS tile that the two softmax warpgroups
-// wrote at the start of their own 64-column halves (keys or queries 0-63 at columns 0-31, 64-127 at 64-95).
-__device__ __forceinline__ uint32_t a_col(int k) { return static_cast<uint32_t>(k < 4 ? 8 * k : 64 + 8 * (k - 4)); }
+// TMEM column of the A operand for K-step k (16 elements) of a bf16 P / dS tile that each softmax
+// warpgroup wrote, packed two to a column, at the start of its own kWGCols-column range.
+// The dq kernel's whole-tile variant: two warpgroups of 64 keys, keys 0-63 at columns 0-31, 64-127 at 64-95.
+__device__ __forceinline__ uint32_t a_col_full(int k) { return static_cast<uint32_t>(k < 4 ? 8 * k : 64 + 8 * (k - 4)); }
+__device__ __forceinline__ uint32_t a_col(int k) {
+    constexpr int steps = kWGCols / 16;  // K-steps per warpgroup
+    return static_cast<uint32_t>((k / steps) * kWGCols + (k % steps) * 8);
+}
 
 // ============================================================== prep: D and lse in log2 units
+// One thread per (row, head), rows padded to Kp: D = dO . O from 16-byte loads of both rows.
+template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ out,
                                                        const __nv_bfloat16* __restrict__ dout,
                                                        const float* __restrict__ lse, int64_t K, int64_t Kp, int Hq,
-                                                       int D, float* __restrict__ lse2, float* __restrict__ dvec) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+                                                       float* __restrict__ lse2, float* __restrict__ dvec) {
     const int64_t total = Kp * Hq;
-    for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < total; w += warps) {
-        const int h = static_cast<int>(w / Kp);
-        const int64_t r = w - static_cast<int64_t>(h) * Kp;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < total;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = w / Hq;
+        const int h = static_cast<int>(w - r * Hq);
         float acc = 0.0f;
         if (r < K) {
-            const __nv_bfloat16* o = out + (r * Hq + h) * D;
-            const __nv_bfloat16* g = dout + (r * Hq + h) * D;
-            for (int t = lane * 4; t < D; t += 128) {
-                const uint2 a = *reinterpret_cast<const uint2*>(o + t);
-                const uint2 b = *reinterpret_cast<const uint2*>(g + t);
-                acc = fmaf(__uint_as_float(a.x << 16), __uint_as_float(b.x << 16), acc);
-                acc = fmaf(__uint_as_float(a.x & 0xffff0000u), __uint_as_float(b.x & 0xffff0000u), acc);
-                acc = fmaf(__uint_as_float(a.y << 16), __uint_as_float(b.y << 16), acc);
-                acc = fmaf(__uint_as_float(a.y & 0xffff0000u), __uint_as_float(b.y & 0xffff0000u), acc);
+            const uint4* o = reinterpret_cast<const uint4*>(out + w * D);   // row r, head h: w = r Hq + h
+            const uint4* g = reinterpret_cast<const uint4*>(dout + w * D);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                const uint4 a = o[i], b = g[i];
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), acc);
+                    acc = fmaf(__uint_as_float(aw[e] & 0xffff0000u), __uint_as_float(bw[e] & 0xffff0000u), acc);
+                }
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) {
-            lse2[h * Kp + r] = r < K ? lse[h * K + r] * kLog2e : INFINITY;
-            dvec[h * Kp + r] = acc;
-        }
+        lse2[h * Kp + r] = r < K ? lse[h * K + r] * kLog2e : INFINITY;
+        dvec[h * Kp + r] = acc;
     }
 }
 
 // ============================================================== dQ
+// Whole 128-key tiles: S and dP of one tile, then dQ += dS K_j.  (Taking the tile in 64-key halves
+// to overlap the softmax with the products made S and dP N = 64 MMAs, which read the full Q / dO
+// tile from shared memory for half the work each, and measured slower.)
 template <int D>
 struct CfgQ {
     static constexpr int kStages = (D == 64) ? 4 : 2;
     static constexpr int kTile = kB * D * 2;
     static constexpr int kChunks = D / 64;
-    static constexpr int kThreads = 352;
     static constexpr int kOffQ = 0;
     static constexpr int kOffDO = kTile;
     static constexpr int kOffK = 2 * kTile;
@@ -158,7 +172,7 @@ struct CfgQ {
     static constexpr int kOffBar = kOffAugB + kStages * kAugTile;
     static constexpr int kNumBars = 1 + 3 * kStages + 4;
     static constexpr int kOffRed = kOffBar + kNumBars * 8;
-    static constexpr int kOffMisc = kOffRed + 8 * 4;
+    static constexpr int kOffMisc = kOffRed + kSoftWarps * 4;
     static constexpr int kSmem = kOffMisc + 16 + 1024;
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
 };
@@ -180,7 +194,7 @@ struct ArgsQ {
 };
 
 template <int D>
-__global__ void __launch_bounds__(CfgQ<D>::kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_do,
               const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v, const ArgsQ a) {
     using C = CfgQ<D>;
@@ -214,10 +228,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant_
             mbar_init(&aug_full[s], 32);
         }
         mbar_init(s_full, 1);
-        mbar_init(ds_full, 256);
+        mbar_init(ds_full, 32 * kSoftWarps);
         mbar_init(o_full, 1);
         mbar_init(drain, 1);
-        for (int w = 0; w < 8; ++w) red[w] = 0.0f;
+        for (int w = 0; w < kSoftWarps; ++w) red[w] = 0.0f;
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmap_q);
@@ -321,7 +335,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant_
                 const uint32_t ko = kmn_lo0 + static_cast<uint32_t>(st * (C::kTile >> 4));
 #pragma unroll
                 for (int k = 0; k < kB / 16; ++k)
-                    mma_ts_lo(tmem + C::kColDQ, tmem + C::kColS + a_col(k), ko + static_cast<uint32_t>(k * (2048 >> 4)),
+                    mma_ts_lo(tmem + C::kColDQ, tmem + C::kColS + a_col_full(k), ko + static_cast<uint32_t>(k * (2048 >> 4)),
                               dhi, idesc_q, (j > 0 || k > 0) ? 1u : 0u);
                 mma_commit(&kv_empty[st]);
                 if (j + 1 < n_kv) {
@@ -436,18 +450,22 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant_
     }
     if (threadIdx.x == 0) {
         float t = 0.0f;
-        for (int w = 0; w < 8; ++w) t += red[w];
+        for (int w = 0; w < kSoftWarps; ++w) t += red[w];
         a.dtau_part[blockIdx.x] = t;
     }
 }
 
+__device__ __forceinline__ uint32_t col_s(int x) { return static_cast<uint32_t>(128 * x); }
+__device__ __forceinline__ uint32_t col_dp(int x) { return static_cast<uint32_t>(128 * x + kHalf); }
+
 // ============================================================== dK, dV, column sums
+// Each step's 128 query columns are taken in two 64-query halves with their own S^T / dP^T
+// columns, so one half's products overlap the other half's softmax.
 template <int D>
 struct CfgKV {
     static constexpr int kStages = (D == 64) ? 3 : 2;
     static constexpr int kTile = kB * D * 2;
     static constexpr int kChunks = D / 64;
-    static constexpr int kThreads = 352;
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kTile;
     static constexpr int kOffQ = 2 * kTile;                      // [S]
@@ -456,12 +474,12 @@ struct CfgKV {
     static constexpr int kOffAugA = kOffVec + kStages * 1024;    // s_c of the CTA's keys
     static constexpr int kOffAugB = kOffAugA + kAugTile;         // [S] gamma_h of the step's head
     static constexpr int kOffBar = kOffAugB + kStages * kAugTile;
-    static constexpr int kNumBars = 1 + 3 * kStages + 4;
-    static constexpr int kOffDs = kOffBar + kNumBars * 8;        // [2][128] per-warpgroup ds
-    static constexpr int kOffDg = kOffDs + 2 * kB * 4;           // [8 warps][kMaxGroup]
-    static constexpr int kOffMisc = kOffDg + 8 * kMaxGroup * 4;
+    static constexpr int kNumBars = 1 + 3 * kStages + 6;
+    static constexpr int kOffDs = kOffBar + kNumBars * 8;        // [kWG][128] per-warpgroup ds
+    static constexpr int kOffDg = kOffDs + kWG * kB * 4;         // [kSoftWarps][kMaxGroup]
+    static constexpr int kOffMisc = kOffDg + kSoftWarps * kMaxGroup * 4;
     static constexpr int kSmem = kOffMisc + 16 + 1024;
-    static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+    static constexpr uint32_t kColDV = 256, kColDK = 256 + D;
 };
 
 struct ArgsKV {
@@ -480,7 +498,7 @@ struct ArgsKV {
 };
 
 template <int D>
-__global__ void __launch_bounds__(CfgKV<D>::kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_do,
                 const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                 const ArgsKV a) {
@@ -491,11 +509,11 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* kv_full = bars;             // K and V tiles of the CTA landed
     uint64_t* st_full = bars + 1;         // [S] Q_i, dO_i, lse2 and D slices landed
-    uint64_t* st_empty = st_full + S;     // [S] commit after dV and dK of the step
+    uint64_t* st_empty = st_full + S;     // [S] commit after the second half's dV and dK
     uint64_t* aug_full = st_empty + S;    // [S] gamma operand of the step written (32 lanes)
-    uint64_t* s_full = aug_full + S;      // commit after S^T and dP^T
-    uint64_t* p_full = s_full + 1;        // 256 softmax threads wrote P^T and dS^T
-    uint64_t* o_full = p_full + 1;        // commit after the last dV / dK MMA
+    uint64_t* s_full = aug_full + S;      // [2] commit after a half's S^T and dP^T
+    uint64_t* p_full = s_full + 2;        // [2] the softmax threads wrote that half's P^T and dS^T
+    uint64_t* o_full = p_full + 2;        // commit after the last dV / dK MMA
     uint64_t* drain = o_full + 1;
     float* dsw = reinterpret_cast<float*>(smem + C::kOffDs);
     float* dgw = reinterpret_cast<float*>(smem + C::kOffDg);
@@ -507,6 +525,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const int kvh = static_cast<int>(blockIdx.x % a.Hkv);
     const int nq = a.num_q_tiles - n_tile;                    // query tiles n_tile .. last
     const int T = nq * a.G;                                   // steps: (head of the group, query tile)
+    const int U = 2 * T;                                      // halves: u = 2 t + (0 | 1)
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -515,12 +534,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
             mbar_init(&st_empty[s], 1);
             mbar_init(&aug_full[s], 32);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 256);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 32 * kSoftWarps);
+        }
         mbar_init(o_full, 1);
         mbar_init(drain, 1);
-        for (int i = 0; i < 8 * kMaxGroup; ++i) dgw[i] = 0.0f;
-        for (int i = 0; i < 2 * kB; ++i) dsw[i] = 0.0f;
+        for (int i = 0; i < kSoftWarps * kMaxGroup; ++i) dgw[i] = 0.0f;
+        for (int i = 0; i < kWG * kB; ++i) dsw[i] = 0.0f;
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmap_q);
@@ -584,7 +605,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(kB, kB, false);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(kB, kHalf, false);  // 128 keys x 64 queries
             constexpr uint32_t idesc_o = idesc_bf16_f32(kB, D, true);
             const uint32_t dhi = sw128_desc_hi(1024);
             const uint32_t k_lo = sw128_desc_lo(smem_u32(smem + C::kOffK), 16);
@@ -602,46 +623,50 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
                 return wait1(&st_full[t % S], ph, abort_flag, a.status) &&
                        wait1(&aug_full[t % S], ph, abort_flag, a.status);
             };
-            // S^T = K Q_i^T (+ bias) and dP^T = V dO_i^T
-            auto issue_sdp = [&](int t) {
-                const uint32_t so = static_cast<uint32_t>((t % S) * (C::kTile >> 4));
+            // half u (queries 64 (u & 1) .. of step u / 2): S^T = K Q^T (+ bias), dP^T = V dO^T
+            auto issue_sdp = [&](int u) {
+                const int t = u >> 1, hf = u & 1;
+                const uint32_t so = static_cast<uint32_t>((t % S) * (C::kTile >> 4) + ((hf * kHalf * 128) >> 4));
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k)
-                    mma_ss_lo(tmem + C::kColS, k_lo + kstep_off(k), q_lo0 + so + kstep_off(k), dhi, idesc_s, k > 0);
+                    mma_ss_lo(tmem + col_s(hf), k_lo + kstep_off(k), q_lo0 + so + kstep_off(k), dhi, idesc_s, k > 0);
                 if (bias)
-                    mma_ss_lo(tmem + C::kColS, aa_lo, ab_lo0 + static_cast<uint32_t>((t % S) * (kAugTile >> 4)), ahi,
+                    mma_ss_lo(tmem + col_s(hf), aa_lo,
+                              ab_lo0 + static_cast<uint32_t>((t % S) * (kAugTile >> 4) + ((hf * 2048) >> 4)), ahi,
                               idesc_s, 1u);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k)
-                    mma_ss_lo(tmem + C::kColDP, v_lo + kstep_off(k), do_lo0 + so + kstep_off(k), dhi, idesc_s, k > 0);
-                mma_commit(s_full);
+                    mma_ss_lo(tmem + col_dp(hf), v_lo + kstep_off(k), do_lo0 + so + kstep_off(k), dhi, idesc_s, k > 0);
+                mma_commit(&s_full[hf]);
             };
             bool ok = wait1(kv_full, 0, abort_flag, a.status) && ready(0);
             if (ok) {
                 tc_fence_after();
                 issue_sdp(0);
+                issue_sdp(1);
             }
-            for (int t = 0; t < T && ok; ++t) {
+            for (int u = 0; u < U && ok; ++u) {
+                const int t = u >> 1, hf = u & 1;
                 const int st = t % S;
-                if (!(ok = wait1(p_full, static_cast<uint32_t>(t) & 1, abort_flag, a.status))) break;
+                if (!(ok = wait1(&p_full[hf], static_cast<uint32_t>(t) & 1, abort_flag, a.status))) break;
                 tc_fence_after();
-                const uint32_t so = static_cast<uint32_t>(st * (C::kTile >> 4));
-                // dV += P^T dO_i and dK += dS^T Q_i: 16 queries per step
+                // dV += P^T dO and dK += dS^T Q over the half's 64 queries (16 rows of the MN-major tiles per step)
+                const uint32_t so = static_cast<uint32_t>(st * (C::kTile >> 4) + ((hf * kHalf * 128) >> 4));
 #pragma unroll
-                for (int k = 0; k < kB / 16; ++k)
-                    mma_ts_lo(tmem + C::kColDV, tmem + C::kColS + a_col(k),
+                for (int k = 0; k < kHalf / 16; ++k)
+                    mma_ts_lo(tmem + C::kColDV, tmem + col_s(hf) + a_col(k),
                               domn_lo0 + so + static_cast<uint32_t>(k * (2048 >> 4)), dhi, idesc_o,
-                              (t > 0 || k > 0) ? 1u : 0u);
+                              (u > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
-                for (int k = 0; k < kB / 16; ++k)
-                    mma_ts_lo(tmem + C::kColDK, tmem + C::kColDP + a_col(k),
+                for (int k = 0; k < kHalf / 16; ++k)
+                    mma_ts_lo(tmem + C::kColDK, tmem + col_dp(hf) + a_col(k),
                               qmn_lo0 + so + static_cast<uint32_t>(k * (2048 >> 4)), dhi, idesc_o,
-                              (t > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&st_empty[st]);
-                if (t + 1 < T) {
-                    if (!(ok = ready(t + 1))) break;
-                    issue_sdp(t + 1);
-                } else {
+                              (u > 0 || k > 0) ? 1u : 0u);
+                if (hf == 1) mma_commit(&st_empty[st]);  // both halves of the step consumed
+                if (u + 2 < U) {
+                    if (hf == 0 && !(ok = ready(t + 1))) break;
+                    issue_sdp(u + 2);
+                } else if (u == U - 1) {
                     mma_commit(o_full);
                 }
             }
@@ -668,7 +693,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     } else {
         // ------------------------------------------------------------ P^T, dS^T, column sums; dk/dv epilogue
         const int sw = warp - 3;
-        const int wg = sw >> 2;              // which 64 queries of the tile
+        const int wg = sw >> 2;              // which kWGCols queries of each half
         const int qd = warp & 3;
         const int row = qd * 32 + lane;      // key in the tile == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
@@ -686,50 +711,49 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
             cs = 0.0f;
         };
         bool ok = true;
-        for (int t = 0; t < T && ok; ++t) {
+        for (int u = 0; u < U && ok; ++u) {
+            const int t = u >> 1, hf = u & 1;
             const int st = t % S;
             const int hh = t / nq;
             const int i = n_tile + t % nq;
-            if (t > 0 && t % nq == 0) flush(hh - 1);
-            if (!(ok = warp_wait(s_full, static_cast<uint32_t>(t) & 1, abort_flag, a.status))) break;
+            if (hf == 0 && t > 0 && t % nq == 0) flush(hh - 1);
+            if (!(ok = warp_wait(&s_full[hf], static_cast<uint32_t>(t) & 1, abort_flag, a.status))) break;
             tc_fence_after();
             const float* lse2s = reinterpret_cast<const float*>(smem + C::kOffVec + st * 1024);
             const float* dvs = lse2s + kB;
             const bool diag = i == n_tile;
+            const int c0 = kWGCols * wg;          // first query of this warpgroup in the half
+            const int q0 = hf * kHalf + c0;       // ... and in the tile
+            uint32_t sv[32], pv[32];
+            tmem_ld32(tmem + lane_off + col_s(hf) + c0, sv);
+            tmem_ld32(tmem + lane_off + col_dp(hf) + c0, pv);
+            tmem_ld_wait();
+            uint32_t p16[16], d16[16];
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                const int c0 = 64 * wg + 32 * ch;  // first query column of the chunk
-                uint32_t sv[32], pv[32];
-                tmem_ld32(tmem + lane_off + C::kColS + c0, sv);
-                tmem_ld32(tmem + lane_off + C::kColDP + c0, pv);
-                tmem_ld_wait();
-                uint32_t p16[16], d16[16];
+            for (int e = 0; e < 32; e += 4) {
+                const float4 L = *reinterpret_cast<const float4*>(lse2s + q0 + e);
+                const float4 Dd = *reinterpret_cast<const float4*>(dvs + q0 + e);
+                const float lv[4] = {L.x, L.y, L.z, L.w};
+                const float dv4[4] = {Dd.x, Dd.y, Dd.z, Dd.w};
+                float p[4], ds[4];
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    const float4 L = *reinterpret_cast<const float4*>(lse2s + c0 + e);
-                    const float4 Dd = *reinterpret_cast<const float4*>(dvs + c0 + e);
-                    const float lv[4] = {L.x, L.y, L.z, L.w};
-                    const float dv4[4] = {Dd.x, Dd.y, Dd.z, Dd.w};
-                    float p[4], ds[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        p[u] = ex2(fmaf(__uint_as_float(sv[e + u]), a.scale_log2, -lv[u]));
-                        if (diag && c0 + e + u < row) p[u] = 0.0f;  // query before the key
-                        ds[u] = p[u] * (__uint_as_float(pv[e + u]) - dv4[u]);
-                        cs += ds[u];
-                    }
-                    p16[e >> 1] = pack_bf16x2(p[0], p[1]);
-                    p16[(e >> 1) + 1] = pack_bf16x2(p[2], p[3]);
-                    d16[e >> 1] = pack_bf16x2(ds[0], ds[1]);
-                    d16[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
+                for (int w = 0; w < 4; ++w) {
+                    p[w] = ex2(fmaf(__uint_as_float(sv[e + w]), a.scale_log2, -lv[w]));
+                    if (diag && q0 + e + w < row) p[w] = 0.0f;  // query before the key
+                    ds[w] = p[w] * (__uint_as_float(pv[e + w]) - dv4[w]);
+                    cs += ds[w];
                 }
-                tmem_st16(tmem + lane_off + C::kColS + 64 * wg + 16 * ch, p16);
-                tmem_st16(tmem + lane_off + C::kColDP + 64 * wg + 16 * ch, d16);
+                p16[e >> 1] = pack_bf16x2(p[0], p[1]);
+                p16[(e >> 1) + 1] = pack_bf16x2(p[2], p[3]);
+                d16[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+                d16[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
             }
+            tmem_st16(tmem + lane_off + col_s(hf) + c0, p16);
+            tmem_st16(tmem + lane_off + col_dp(hf) + c0, d16);
             tmem_st_wait();
             fence_proxy_async_smem();  // the lse2 / D reads come before the stage is refilled by TMA
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[hf]);
         }
         if (ok) {
             flush(a.G - 1);
@@ -743,18 +767,18 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
                 const float f = pass == 0 ? 1.0f : a.scale;
                 __nv_bfloat16* dst_row = (pass == 0 ? a.dv : a.dk) + (key * a.Hkv + kvh) * D;
 #pragma unroll
-                for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_off + col0 + c0, v);
+                for (int c0 = wg * (D / kWG); c0 < (wg + 1) * (D / kWG); c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + lane_off + col0 + c0, v);
                     tmem_ld_wait();
                     if (key < a.K) {
-                        uint32_t o[16];
+                        uint32_t o[8];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
+                        for (int e = 0; e < 8; ++e)
                             o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * f, __uint_as_float(v[2 * e + 1]) * f);
                         uint4* dst = reinterpret_cast<uint4*>(dst_row + c0);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+                        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
                     }
                 }
             }
@@ -767,11 +791,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-    if (threadIdx.x < kB)
-        a.ds_part[kvh * a.Kp + static_cast<int64_t>(n_tile) * kB + threadIdx.x] = dsw[threadIdx.x] + dsw[kB + threadIdx.x];
+    if (threadIdx.x < kB) {
+        float t = 0.0f;
+        for (int w = 0; w < kWG; ++w) t += dsw[w * kB + threadIdx.x];
+        a.ds_part[kvh * a.Kp + static_cast<int64_t>(n_tile) * kB + threadIdx.x] = t;
+    }
     if (threadIdx.x < a.G) {
         float t = 0.0f;
-        for (int w = 0; w < 8; ++w) t += dgw[w * kMaxGroup + threadIdx.x];
+        for (int w = 0; w < kSoftWarps; ++w) t += dgw[w * kMaxGroup + threadIdx.x];
         a.dg_part[static_cast<int64_t>(kvh * a.G + threadIdx.x) * a.num_k_tiles + n_tile] = t;
     }
 }
@@ -782,6 +809,7 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const float* __restrict
                                                          const float* __restrict__ dtau_part, int64_t K, int64_t Kp,
                                                          int Hq, int Hkv, int num_k_tiles, int n_dq_ctas,
                                                          float inv_sqrt_d, float* ds, float* dg, float* dtau) {
+    __shared__ float red[256];
     if (ds) {
         for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < K;
              c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -797,11 +825,16 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const float* __restrict
                 for (int n = 0; n < num_k_tiles; ++n) t += dg_part[static_cast<int64_t>(h) * num_k_tiles + n];
                 dg[h] = t;
             }
-        if (dtau && threadIdx.x == 0) {
-            float t = 0.0f;
-            for (int i = 0; i < n_dq_ctas; ++i) t += dtau_part[i];
-            *dtau = t * inv_sqrt_d;
+        // dtau: strided partial sums, then a fixed tree (the same order on every run)
+        float t = 0.0f;
+        for (int i = threadIdx.x; i < n_dq_ctas; i += blockDim.x) t += dtau_part[i];
+        red[threadIdx.x] = t;
+        __syncthreads();
+        for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+            if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+            __syncthreads();
         }
+        if (dtau && threadIdx.x == 0) *dtau = red[0] * inv_sqrt_d;
     }
 }
 
@@ -852,7 +885,7 @@ tg_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtens
         if (!set_max_dynamic_smem(kern, bwd::CfgQ<D>::kSmem, smem_set)) return TG_ERR_CUDA;
         const int64_t grid = static_cast<int64_t>(aq.num_q_tiles) * aq.Hq;
         if (grid > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
-        kern<<<static_cast<unsigned>(grid), bwd::CfgQ<D>::kThreads, bwd::CfgQ<D>::kSmem, st>>>(mq, mdo, mk, mv, aq);
+        kern<<<static_cast<unsigned>(grid), bwd::kThreads, bwd::CfgQ<D>::kSmem, st>>>(mq, mdo, mk, mv, aq);
         if (launch_status() != TG_OK) return TG_ERR_CUDA;
     }
     {
@@ -861,7 +894,7 @@ tg_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtens
         if (!set_max_dynamic_smem(kern, bwd::CfgKV<D>::kSmem, smem_set)) return TG_ERR_CUDA;
         const int64_t grid = static_cast<int64_t>(akv.num_k_tiles) * akv.Hkv;
         if (grid > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
-        kern<<<static_cast<unsigned>(grid), bwd::CfgKV<D>::kThreads, bwd::CfgKV<D>::kSmem, st>>>(mq, mdo, mk, mv, akv);
+        kern<<<static_cast<unsigned>(grid), bwd::kThreads, bwd::CfgKV<D>::kSmem, st>>>(mq, mdo, mk, mv, akv);
         if (launch_status() != TG_OK) return TG_ERR_CUDA;
     }
     return TG_OK;
@@ -901,11 +934,16 @@ extern "C" tg_status tg_gated_attention_backward(const tg_bf16* q, int64_t ld_q,
     float* dg_part = reinterpret_cast<float*>(ws + L.dg_part);
     float* dtau_part = reinterpret_cast<float*>(ws + L.dtau_part);
     {
-        const int64_t warps = L.Kp * Hq;
-        const int64_t blocks = std::min<int64_t>((warps + 7) / 8, static_cast<int64_t>(num_sms()) * 16);
-        bwd::bwd_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-            reinterpret_cast<const __nv_bfloat16*>(out), reinterpret_cast<const __nv_bfloat16*>(dout), lse, K, L.Kp,
-            Hq, d_h, lse2, dvec);
+        const int64_t items = L.Kp * Hq;
+        const int64_t blocks = std::min<int64_t>((items + 255) / 256, static_cast<int64_t>(num_sms()) * 64);
+        const auto* o16 = reinterpret_cast<const __nv_bfloat16*>(out);
+        const auto* g16 = reinterpret_cast<const __nv_bfloat16*>(dout);
+        if (d_h == 128)
+            bwd::bwd_prep_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(o16, g16, lse, K, L.Kp, Hq, lse2,
+                                                                                     dvec);
+        else
+            bwd::bwd_prep_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(o16, g16, lse, K, L.Kp, Hq, lse2,
+                                                                                    dvec);
         if (launch_status() != TG_OK) return TG_ERR_CUDA;
     }
     CUtensorMap mq, mdo, mk, mv;
