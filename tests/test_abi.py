@@ -122,3 +122,31 @@ def test_decode_and_random_select_argument_errors(lib):
     assert rs(1000, 0, 900, 10, 7, vp(16), vp(256), 16, None) == INV       # workspace too small
     assert rs(1000, 0, 900, 10, 7, vp(16), None, 1 << 20, None) == INV     # no workspace
     assert rs(0, 0, 0, 5, 7, None, None, 0, None) == tg.TG_OK              # nothing to keep
+
+
+def test_backward_workspace_and_argument_errors(lib):
+    vp = ctypes.c_void_p
+    INV, UNS = tg.TG_ERR_INVALID_ARG, tg.TG_ERR_UNSUPPORTED
+    # workspace: lse2 and D per head and padded row, ds per KV head and padded row, dg and dtau partials
+    ws = tg.tg_workspace_bytes(tg.TG_OP_ATTENTION_BACKWARD, 4608, 16, 8)
+    assert ws >= 256 + 4 * (2 * 16 * 4608 + 8 * 4608 + 2 * 16 * 36) and ws % 256 == 0
+    assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION_BACKWARD, 4608, 16, 3) == 0   # Hq % Hkv
+    assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION_BACKWARD, -1, 16, 8) == 0
+    big = tg.tg_workspace_bytes(tg.TG_OP_ATTENTION_BACKWARD, 300, 16, 8)
+
+    def bwd(q=16, K=300, Hq=16, Hkv=8, d_h=128, tau=1.0, lse=16, dq=16, ws_bytes=big, ldq=None):
+        ldq = Hq * d_h if ldq is None else ldq
+        return lib.tg_gated_attention_backward(vp(q), ldq, vp(4096), Hkv * d_h, vp(8192), Hkv * d_h, K, Hq, Hkv,
+                                               d_h, None, None, tau, vp(16), vp(32), vp(lse) if lse else None,
+                                               vp(dq) if dq else None, vp(48), vp(64), None, None, None, vp(256),
+                                               ws_bytes, None)
+
+    assert bwd(tau=0.0) == INV and bwd(tau=float("nan")) == INV
+    assert bwd(Hq=12, Hkv=8) == INV
+    assert bwd(d_h=96) == UNS
+    assert bwd(Hq=16, Hkv=1) == UNS                 # 16 query heads per KV head
+    assert bwd(lse=0) == INV                        # the forward's log-sum-exp is required
+    assert bwd(dq=0) == INV
+    assert bwd(q=24) == INV                         # misaligned
+    assert bwd(ldq=16 * 128 + 4) == INV             # stride not a multiple of 8
+    assert bwd(ws_bytes=big - 256) == INV
