@@ -245,6 +245,70 @@ def oracle_sample(w, gi, ap, budget_s, seed=0):
     return total, sample, parts
 
 
+def oracle_backward_sample(K, Hq, Hkv, d_h, budget_s=10.0, seed=0):
+    """Time the single-threaded oracle backward on a bounded sample and extrapolate one full backward.
+
+    Sample: one KV head and its G = Hq / Hkv query heads (an independent problem) over the first K' of
+    the K tokens, K' chosen so the sample takes about budget_s; the causal work grows as K'(K'+1)/2,
+    so the time is scaled by K(K+1) / (K'(K'+1)) and by the Hkv KV heads."""
+    import numpy as np
+
+    import oracle
+
+    G = Hq // Hkv
+    # about 5 multiply-adds of d_h per visible (query, key, head) pair at ~1.2e9 per second
+    per_pair = 5.0 * d_h / 1.2e9 * G
+    Ks = int(min(K, max(64, (2.0 * budget_s / per_pair) ** 0.5)))
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((Ks, G, d_h)).astype(np.float32)
+    k = rng.standard_normal((Ks, 1, d_h)).astype(np.float32)
+    v = rng.standard_normal((Ks, 1, d_h)).astype(np.float32)
+    do = rng.standard_normal((Ks, G, d_h)).astype(np.float32)
+    s = rng.standard_normal(Ks).astype(np.float32)
+    g = rng.random(G).astype(np.float32)
+    t0 = time.perf_counter()
+    oracle.gated_attention_backward(q, k, v, do, s=s, g=g, tau=1.1)
+    t = time.perf_counter() - t0
+    total = t * (K * (K + 1.0)) / (Ks * (Ks + 1.0)) * Hkv
+    sample = (f"oracle backward, 1 thread: 1 of {Hkv} KV heads ({G} query heads) over the first {Ks} of {K} "
+              f"tokens, extrapolated by the causal pair count and the KV heads")
+    return total, sample
+
+
+def oracle_decode_sample(keys_per_layer, Hq, Hkv, d_h, budget_s=5.0, seed=0):
+    """Time the single-threaded oracle on one decoding query over a T_s-key cache (the oracle's gated
+    attention for the last row) and extrapolate by the keys of every layer (work is linear in keys)."""
+    import numpy as np
+
+    import oracle
+
+    per_key = 2.0 * d_h * Hq / 1.2e9
+    Ts = int(min(max(keys_per_layer), max(256, budget_s / per_key)))
+    rng = np.random.default_rng(seed)
+    q = np.zeros((Ts, Hq, d_h), dtype=np.float32)
+    q[-1] = rng.standard_normal((Hq, d_h))
+    k = rng.standard_normal((Ts, Hkv, d_h)).astype(np.float32)
+    v = rng.standard_normal((Ts, Hkv, d_h)).astype(np.float32)
+    s = rng.standard_normal(Ts).astype(np.float32)
+    g = rng.random(Hq).astype(np.float32)
+    t0 = time.perf_counter()
+    oracle.gated_attention(q, k, v, s=s, g=g, tau=1.1, rows=[Ts - 1])
+    t = time.perf_counter() - t0
+    total = t / Ts * float(sum(keys_per_layer))
+    sample = (f"oracle, 1 thread: one decoding query over a {Ts}-key cache ({Hq} heads), extrapolated by the "
+              f"{sum(keys_per_layer)} cached keys of the {len(keys_per_layer)} layer(s)")
+    return total, sample
+
+
+def decode_cpu_baseline(args, keys_per_layer, Hq, Hkv, d_h, unit_scale, unit):
+    if args.no_cpu_baseline:
+        return {}
+    cores = pin_one_core()
+    t, sample = oracle_decode_sample(keys_per_layer, Hq, Hkv, d_h, budget_s=min(args.cpu_budget, 5.0))
+    return {"cpu_baseline": {"value": t * unit_scale, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": sample}}
+
+
 def pin_one_core():
     try:
         os.sched_setaffinity(0, {sorted(os.sched_getaffinity(0))[0]})
@@ -618,7 +682,9 @@ def run_decode(args, rank, world, local_rank):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "gated_decode_kernel",
                          "dense_frac": b_dense / (ms_dense * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-            "gpu_launches": cfg.n_layers * reps, "clocks": clk.summary(), "device_status": status}
+            "gpu_launches": cfg.n_layers * reps, "clocks": clk.summary(), "device_status": status,
+            **decode_cpu_baseline(args, [T_all if li <= L else T_kept for li in range(cfg.n_layers)], Hq, Hkv,
+                                  d_h, 1e3, "ms")}
 
 
 def run_decode_layer(args, rank, world, local_rank):
@@ -664,7 +730,8 @@ def run_decode_layer(args, rank, world, local_rank):
             "impl": "tokengate",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "gated_decode_kernel"},
-            "gpu_launches": reps, "device_status": tg.tg_device_status(ws)}
+            "gpu_launches": reps, "device_status": tg.tg_device_status(ws),
+            **decode_cpu_baseline(args, [T], cfg.Hq, cfg.Hkv, cfg.d_h, 1e6, "us")}
 
 
 def run_backward(args, rank, world, local_rank):
@@ -724,7 +791,17 @@ def run_backward(args, rank, world, local_rank):
                          "frac": tf / peaks["bf16_tflops"], "traffic": None,
                          "kernel": "whole backward (prep, dq, dkdv, finish)",
                          "algorithmic_flop": flop},
-            "clocks": clk.summary(), "gpu_launches": 4 * reps, "device_status": tg.tg_device_status(ws)}
+            "clocks": clk.summary(), "gpu_launches": 4 * reps, "device_status": tg.tg_device_status(ws),
+            **backward_cpu_baseline(args, K, Hq, Hkv, d_h)}
+
+
+def backward_cpu_baseline(args, K, Hq, Hkv, d_h):
+    """The oracle backward beside the GPU one (rank 0 only; skipped with --no-cpu-baseline)."""
+    if args.no_cpu_baseline:
+        return {}
+    cores = pin_one_core()
+    t, sample = oracle_backward_sample(K, Hq, Hkv, d_h, budget_s=min(args.cpu_budget, 15.0))
+    return {"cpu_baseline": {"value": t * 1e6, "unit": "us", "cores": cores, "kind": "oracle", "sample": sample}}
 
 
 def main():
