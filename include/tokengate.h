@@ -71,7 +71,8 @@ typedef enum {
     TG_OP_ATTENTION = 2,
     TG_OP_ALL = 3, /* one buffer usable by every call above */
     TG_OP_DECODE = 4,
-    TG_OP_ATTENTION_BACKWARD = 5
+    TG_OP_ATTENTION_BACKWARD = 5,
+    TG_OP_PROJECT = 6
 } tg_op;
 
 /* Bits of the device status word (first 4 bytes of the workspace). */
@@ -80,6 +81,7 @@ typedef enum {
 #define TG_STATUS_ATTENTION_TIMEOUT 0x4u
 #define TG_STATUS_DECODE_TIMEOUT 0x8u
 #define TG_STATUS_BACKWARD_TIMEOUT 0x10u
+#define TG_STATUS_PROJECT_TIMEOUT 0x20u
 
 /* Static description of a status code.  Never NULL. */
 const char* tg_status_string(tg_status status);
@@ -102,6 +104,7 @@ int64_t tg_kept_count(int64_t N, int64_t doc_begin, int64_t doc_end, int64_t k_d
  *   TG_OP_DECODE     tg_gated_decode with d = Hq query heads (N, d_g unused)
  *   TG_OP_ATTENTION_BACKWARD  tg_gated_attention_backward with N = K kept
  *                    tokens, d = Hq query heads, d_g = Hkv KV heads
+ *   TG_OP_PROJECT    tg_project_rope with N = K kept tokens, d = d_h
  * Returns 0 for bad arguments. */
 size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g);
 
@@ -277,6 +280,28 @@ tg_status tg_gated_attention_backward(const tg_bf16* q, int64_t ld_q, const tg_b
                                       const tg_bf16* out, const tg_bf16* dout, const float* lse,
                                       tg_bf16* dq, tg_bf16* dk, tg_bf16* dv, float* ds, float* dg,
                                       float* dtau, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The Q/K/V projection of the kept rows with the rotary embedding fused into
+ * the GEMM epilogue (layers above the gate see only the kept tokens, rotated
+ * at their original positions; aiproducthub.cn article, paragraph 事件详情):
+ *   qkv[r, :] = x[r, :] W^T, then for every query and key head the
+ *   rotate-half pairs (t, t + d_h/2) turned by pos[r] * base^(-2t/d_h)
+ *   (angles in fp64, as tg_rope_apply), from the fp32 accumulators;
+ *   value heads are stored as they are, and also in fp16 into v16.
+ * x: [K, d] bf16, row stride ld_x (multiple of 8).  W: [(Hq + 2 Hkv) d_h, d]
+ * bf16 (query heads, then key heads, then value heads, as an nn.Linear
+ * weight).  pos: [K] int32.  qkv: [K, (Hq + 2 Hkv) d_h] bf16, row stride
+ * ld_qkv (multiple of 8).  v16: [K, Hkv d_h] fp16 (uint16 bit patterns)
+ * dense, or NULL.  workspace: tg_workspace_bytes(TG_OP_PROJECT, K, d_h, 0)
+ * bytes (the cos / sin table of the K rows).
+ * Supported: d a multiple of 64; (Hq + 2 Hkv) d_h a multiple of 256; d_h in
+ * {64, 128}; x, W, qkv, v16 16-byte aligned.  Two launches: the cos / sin
+ * table, then a persistent tcgen05 GEMM (128 x 256 tiles, TMA-staged
+ * operands, TMEM accumulators double-buffered against the epilogue).
+ * Waits are bounded (TG_STATUS_PROJECT_TIMEOUT). */
+tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int64_t ld_x, const tg_bf16* W, int32_t Hq,
+                          int32_t Hkv, int32_t d_h, const int32_t* pos, double base, tg_bf16* qkv, int64_t ld_qkv,
+                          uint16_t* v16, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Test hook (fault injection without a fault): sets the time limit of the
  * grid barrier inside tg_topk_select, tg_topk_select_noalloc and

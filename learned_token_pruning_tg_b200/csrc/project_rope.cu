@@ -1,0 +1,364 @@
+// project_rope.cu -- the Q/K/V projection of the kept rows with the rotary
+// embedding and V's fp16 copy fused into the GEMM's epilogue.
+//
+// Layers above the gate see only the kept tokens (aiproducthub.cn article,
+// paragraph 事件详情; chathome.org article, section TokenGate の学習可能な
+// トークンプルーニングの仕組み); their queries and keys are rotated at the kept
+// tokens' original positions (the specification's reading: positions travel
+// with the rows).  Unfused, the kept rows' projection is a library GEMM whose
+// bf16 output RoPE then reads and rewrites, and the attention converts V to
+// fp16 in one more pass; here one kernel does all three:
+//   qkv[r, :] = x[r, :] W^T                     (bf16 x bf16 -> fp32 in TMEM)
+//   q/k heads: rotate-half pairs (t, t + d_h/2) at pos[r], from the fp32
+//              accumulator (one bf16 rounding instead of two)
+//   v heads:   bf16 into qkv and, when asked, fp16 into v16
+// Angles are formed in fp64 exactly as tg_rope_apply forms them (a small
+// kernel writes the cos / sin table of every kept row into the workspace).
+//
+// Kernel (persistent, one CTA per SM, 8 warps): tiles of 128 rows x 256
+// output columns, row-tile-major so the CTAs working at one time share the
+// rows of x in L2.
+//   warp 0      TMA producer: 128 x 64 tiles of x and 256 x 64 tiles of W into
+//               a 4-deep ring (128-byte swizzle)
+//   warp 1      TMEM allocation (2 x 256 columns) and the single thread that
+//               issues tcgen05.mma (M = 128, N = 256, K = 16)
+//   warps 4-7   epilogue, one row per thread, double-buffered with the next
+//               tile's main loop
+// Every wait is bounded (TG_STATUS_PROJECT_TIMEOUT).
+#include <cuda_fp16.h>
+
+#include <cmath>
+
+#include "tg_host.cuh"
+
+namespace tg {
+namespace proj {
+
+constexpr int kBM = 128;       // rows per tile
+constexpr int kBN = 256;       // output columns per tile
+constexpr int kBK = 64;        // K elements per stage (one 128-byte swizzle row)
+constexpr int kStages = 4;
+constexpr int kThreads = 256;  // 8 warps
+constexpr int kStageA = kBM * kBK * 2;
+constexpr int kStageB = kBN * kBK * 2;
+constexpr int kStage = kStageA + kStageB;
+constexpr int kOffBar = kStages * kStage;
+constexpr int kNumBars = 2 * kStages + 5;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmem = kOffMisc + 16 + 1024;
+
+struct Args {
+    int64_t K;
+    int d;
+    int Hq, Hkv, D;
+    int num_col_tiles;
+    int64_t num_tiles;
+    const float* cos_t;   // [K, D/2]
+    const float* sin_t;   // [K, D/2]
+    __nv_bfloat16* qkv;
+    int64_t ld_qkv;
+    __half* v16;          // [K, Hkv D] or null
+    unsigned int* status;
+};
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// cos / sin of pos[r] * base^(-2t / d_h), t < d_h / 2, in fp64, rounded to fp32.
+__global__ void __launch_bounds__(64) rope_table_kernel(const int32_t* __restrict__ pos, int64_t K, int D,
+                                                        double base, float* __restrict__ cos_t,
+                                                        float* __restrict__ sin_t) {
+    const int half = D >> 1;
+    for (int64_t r = blockIdx.x; r < K; r += gridDim.x) {
+        const double p = static_cast<double>(__ldg(pos + r));
+        for (int t = threadIdx.x; t < half; t += blockDim.x) {
+            const double inv_freq = pow(base, -2.0 * static_cast<double>(t) / static_cast<double>(D));
+            double s, c;
+            sincos(p * inv_freq, &s, &c);
+            cos_t[r * half + t] = static_cast<float>(c);
+            sin_t[r * half + t] = static_cast<float>(s);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+project_rope_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                    const Args a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* full = bars;                   // [kStages] TMA -> MMA
+    uint64_t* empty = bars + kStages;        // [kStages] MMA commit -> TMA
+    uint64_t* acc_full = bars + 2 * kStages; // [2] MMA commit -> epilogue
+    uint64_t* acc_empty = acc_full + 2;      // [2] 128 epilogue threads -> MMA
+    uint64_t* drain = acc_full + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kb_per_tile = a.d / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmap_x);
+        tma_prefetch_desc(&tmap_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 2 * kBN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int last_ph[kStages];
+            for (int i = 0; i < kStages; ++i) last_ph[i] = -1;
+            for (int64_t t = blockIdx.x; t < a.num_tiles && !*abort_flag; t += gridDim.x) {
+                const int rt = static_cast<int>(t / a.num_col_tiles);
+                const int ct = static_cast<int>(t % a.num_col_tiles);
+                for (int kb = 0; kb < kb_per_tile; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT)) break;
+                    uint8_t* sa = smem + s * kStage;
+                    mbar_arrive_expect_tx(&full[s], kStage);
+                    tma_load_2d(sa, &tmap_x, &full[s], kb * kBK, rt * kBM, kEvictLast);
+                    tma_load_2d(sa + kStageA, &tmap_w, &full[s], kb * kBK, ct * kBN, kEvictLast);
+                    last_ph[s] = static_cast<int>(ph);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+            }
+            // every issued copy lands before shared memory is released (matters on abort only)
+            volatile int no_abort = 0;
+            for (int i = 0; i < kStages; ++i)
+                if (last_ph[i] >= 0)
+                    mbar_wait(&full[i], static_cast<uint32_t>(last_ph[i]), &no_abort, a.status,
+                              TG_STATUS_PROJECT_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, false);
+            int s = 0;
+            uint32_t ph = 0;
+            int64_t it = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < a.num_tiles && ok; t += gridDim.x, ++it) {
+                const int buf = static_cast<int>(it & 1);
+                const uint32_t use = static_cast<uint32_t>(it >> 1);
+                if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
+                for (int kb = 0; kb < kb_per_tile; ++kb) {
+                    if (!mbar_wait(&full[s], ph, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * kStage);
+                    const uint64_t da = smem_desc_sw128(sa, 16, 1024);
+                    const uint64_t db = smem_desc_sw128(sa + kStageA, 16, 1024);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)  // +32 bytes per K = 16 step inside the swizzle row
+                        mma_ss(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    mma_commit(&empty[s]);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (ok) mma_commit(&acc_full[buf]);
+            }
+            if (!ok) {
+                mma_commit(drain);
+                volatile int no_abort = 0;
+                mbar_wait(drain, 0, &no_abort, a.status, TG_STATUS_PROJECT_TIMEOUT);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue
+        const int qd = warp & 3;             // TMEM lane quarter of this warp
+        const int row = qd * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
+        const int D = a.D, half = a.D >> 1;
+        int64_t it = 0;
+        for (int64_t t = blockIdx.x; t < a.num_tiles; t += gridDim.x, ++it) {
+            const int rt = static_cast<int>(t / a.num_col_tiles);
+            const int ct = static_cast<int>(t % a.num_col_tiles);
+            const int buf = static_cast<int>(it & 1);
+            const uint32_t par = static_cast<uint32_t>(it >> 1) & 1;
+            // warp-uniform outcome: tcgen05.ld below is warp-collective
+            const bool ok = mbar_wait(&acc_full[buf], par, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int64_t grow = static_cast<int64_t>(rt) * kBM + row;
+            const bool live = grow < a.K;
+            const uint32_t taddr = tmem_base + lane_off + static_cast<uint32_t>(buf * kBN);
+            __nv_bfloat16* orow = a.qkv + grow * a.ld_qkv + static_cast<int64_t>(ct) * kBN;
+            for (int c_head = 0; c_head < kBN; c_head += D) {
+                const int head = (ct * kBN + c_head) / D;
+                if (head < a.Hq + a.Hkv) {
+                    // rotate-half pairs (t, t + D/2) of a query or key head, 32 pairs at a time
+                    for (int t0 = 0; t0 < half; t0 += 32) {
+                        uint32_t x1[32], x2[32];
+                        tmem_ld32(taddr + c_head + t0, x1);
+                        tmem_ld32(taddr + c_head + half + t0, x2);
+                        tmem_ld_wait();
+                        if (live) {
+                            const float4* cp = reinterpret_cast<const float4*>(a.cos_t + grow * half + t0);
+                            const float4* sp = reinterpret_cast<const float4*>(a.sin_t + grow * half + t0);
+                            uint32_t o1[16], o2[16];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float4 c4 = cp[i], s4 = sp[i];
+                                const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+                                float r1[4], r2[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float u = __uint_as_float(x1[4 * i + e]);
+                                    const float w = __uint_as_float(x2[4 * i + e]);
+                                    r1[e] = u * cc[e] - w * ss[e];
+                                    r2[e] = w * cc[e] + u * ss[e];
+                                }
+                                o1[2 * i] = pack_bf16x2(r1[0], r1[1]);
+                                o1[2 * i + 1] = pack_bf16x2(r1[2], r1[3]);
+                                o2[2 * i] = pack_bf16x2(r2[0], r2[1]);
+                                o2[2 * i + 1] = pack_bf16x2(r2[2], r2[3]);
+                            }
+                            uint4* d1 = reinterpret_cast<uint4*>(orow + c_head + t0);
+                            uint4* d2 = reinterpret_cast<uint4*>(orow + c_head + half + t0);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                d1[i] = make_uint4(o1[4 * i], o1[4 * i + 1], o1[4 * i + 2], o1[4 * i + 3]);
+                                d2[i] = make_uint4(o2[4 * i], o2[4 * i + 1], o2[4 * i + 2], o2[4 * i + 3]);
+                            }
+                        }
+                    }
+                } else {
+                    // a value head: bf16 into qkv and fp16 into v16
+                    const int vh = head - a.Hq - a.Hkv;
+                    for (int t0 = 0; t0 < D; t0 += 32) {
+                        uint32_t x[32];
+                        tmem_ld32(taddr + c_head + t0, x);
+                        tmem_ld_wait();
+                        if (live) {
+                            uint32_t ob[16], oh[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float lo = __uint_as_float(x[2 * i]), hi = __uint_as_float(x[2 * i + 1]);
+                                ob[i] = pack_bf16x2(lo, hi);
+                                oh[i] = pack_f16x2(lo, hi);
+                            }
+                            uint4* db = reinterpret_cast<uint4*>(orow + c_head + t0);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) db[i] = make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+                            if (a.v16) {
+                                uint4* dh = reinterpret_cast<uint4*>(a.v16 + grow * (static_cast<int64_t>(a.Hkv) * D) +
+                                                                     static_cast<int64_t>(vh) * D + t0);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    dh[i] = make_uint4(oh[4 * i], oh[4 * i + 1], oh[4 * i + 2], oh[4 * i + 3]);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 2 * kBN);
+    }
+}
+
+}  // namespace proj
+
+size_t ws_project_bytes(int64_t K, int32_t d_h) {
+    if (K < 0 || (d_h != 64 && d_h != 128)) return 0;
+    return kWsHeader + ((static_cast<size_t>(K) * d_h * 4 + 255) / 256) * 256;  // cos and sin, K x d_h/2 each
+}
+
+}  // namespace tg
+
+using namespace tg;
+
+extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int64_t ld_x, const tg_bf16* W,
+                                     int32_t Hq, int32_t Hkv, int32_t d_h, const int32_t* pos, double base,
+                                     tg_bf16* qkv, int64_t ld_qkv, uint16_t* v16, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    if (K < 0 || d <= 0 || Hq <= 0 || Hkv <= 0 || ld_x < d || !(base > 0.0)) return TG_ERR_INVALID_ARG;
+    if (d_h != 64 && d_h != 128) return TG_ERR_UNSUPPORTED;
+    const int64_t cols = static_cast<int64_t>(Hq + 2 * Hkv) * d_h;
+    if ((d % 64) != 0 || (cols % proj::kBN) != 0 || cols > (1 << 20)) return TG_ERR_UNSUPPORTED;
+    if (K > 0x7fffffffLL - proj::kBM) return TG_ERR_UNSUPPORTED;
+    if (K == 0) return TG_OK;
+    if (!x || !W || !pos || !qkv || !workspace) return TG_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(qkv) || (v16 && !aligned16(v16)) || !aligned16(workspace) ||
+        (ld_x % 8) != 0 || (ld_qkv % 8) != 0 || ld_qkv < cols)
+        return TG_ERR_INVALID_ARG;
+    if (workspace_bytes < ws_project_bytes(K, d_h)) return TG_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    float* cos_t = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeader);
+    float* sin_t = cos_t + K * (d_h / 2);
+    {
+        const int64_t blocks = std::min<int64_t>(K, static_cast<int64_t>(num_sms()) * 16);
+        proj::rope_table_kernel<<<static_cast<unsigned>(blocks), 64, 0, st>>>(pos, K, d_h, base, cos_t, sin_t);
+        if (launch_status() != TG_OK) return TG_ERR_CUDA;
+    }
+    CUtensorMap mx, mw;
+    const uint64_t xd[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(K)};
+    const uint64_t xs[1] = {static_cast<uint64_t>(ld_x) * 2};
+    const uint32_t xb[2] = {proj::kBK, proj::kBM};
+    const uint64_t wd[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(cols)};
+    const uint64_t wsd[1] = {static_cast<uint64_t>(d) * 2};
+    const uint32_t wb[2] = {proj::kBK, proj::kBN};
+    if (!make_tmap_bf16(&mx, x, 2, xd, xs, xb) || !make_tmap_bf16(&mw, W, 2, wd, wsd, wb)) return TG_ERR_CUDA;
+
+    proj::Args a;
+    a.K = K;
+    a.d = d;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.D = d_h;
+    a.num_col_tiles = static_cast<int>(cols / proj::kBN);
+    a.num_tiles = ((K + proj::kBM - 1) / proj::kBM) * a.num_col_tiles;
+    a.cos_t = cos_t;
+    a.sin_t = sin_t;
+    a.qkv = reinterpret_cast<__nv_bfloat16*>(qkv);
+    a.ld_qkv = ld_qkv;
+    a.v16 = reinterpret_cast<__half*>(v16);
+    a.status = status_word(workspace);
+    auto kern = proj::project_rope_kernel;
+    static std::atomic<int> smem_set[64];
+    if (!set_max_dynamic_smem(kern, proj::kSmem, smem_set)) return TG_ERR_CUDA;
+    const int grid = static_cast<int>(std::min<int64_t>(a.num_tiles, num_sms()));
+    kern<<<grid, proj::kThreads, proj::kSmem, st>>>(mx, mw, a);
+    return launch_status();
+}

@@ -17,6 +17,7 @@ namespace tg {
 size_t ws_gate_offset() { return kWsHeader + ((sizeof(SelectScratch) + 255) / 256) * 256; }
 size_t ws_decode_bytes(int32_t Hq);  // gated_decode.cu
 size_t ws_attn_bwd_bytes(int64_t K, int32_t Hq, int32_t Hkv);  // gated_attention_bwd.cu
+size_t ws_project_bytes(int64_t K, int32_t d_h);                 // project_rope.cu
 }  // namespace tg
 
 using namespace tg;
@@ -51,6 +52,7 @@ extern "C" size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g
         case TG_OP_ALL: return ws_gate_offset() + (gate > attn ? gate : attn);
         case TG_OP_DECODE: return (d > 0 && d <= 512) ? ws_decode_bytes(d) : 0;
         case TG_OP_ATTENTION_BACKWARD: return ws_attn_bwd_bytes(N, d, d_g);
+        case TG_OP_PROJECT: return ws_project_bytes(N, d);
     }
     return 0;
 }

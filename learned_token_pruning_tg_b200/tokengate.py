@@ -18,9 +18,9 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtokengate.so")
 
 TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_CUDA, TG_ERR_TIMEOUT = range(5)
-TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL, TG_OP_DECODE, TG_OP_ATTENTION_BACKWARD = range(6)
+TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL, TG_OP_DECODE, TG_OP_ATTENTION_BACKWARD, TG_OP_PROJECT = range(7)
 TG_STATUS_SELECT_TIMEOUT, TG_STATUS_GATE_TIMEOUT, TG_STATUS_ATTENTION_TIMEOUT, TG_STATUS_DECODE_TIMEOUT = 1, 2, 4, 8
-TG_STATUS_BACKWARD_TIMEOUT = 16
+TG_STATUS_BACKWARD_TIMEOUT, TG_STATUS_PROJECT_TIMEOUT = 16, 32
 
 _lib = None
 
@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
         L.tg_gated_attention.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp,
                                          vp, sz, vp]
         L.tg_gated_decode.argtypes = [vp, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp, vp, sz, vp]
+        L.tg_project_rope.argtypes = [vp, i64, i32, i64, vp, i32, i32, i32, vp, f64, vp, i64, vp, vp, sz, vp]
         L.tg_gated_attention_backward.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp,
                                                   vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.tg_debug_set_select_wait_limit.argtypes = [ctypes.c_uint64]
@@ -269,6 +270,29 @@ def tg_gated_attention_backward(q, k, v, out, dout, lse, dq, dk, dv, workspace, 
         d_h, _ptr(s_kept), _ptr(gain), tau, _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
         _ptr(ds), _ptr(dg), _ptr(dtau), _ptr(workspace), workspace.numel(), _stream(stream)))
     return dq, dk, dv
+
+
+def tg_project_rope(x, W, pos, qkv, workspace, Hq: int, Hkv: int, d_h: int, base: float = 1e6, v16=None,
+                    stream=None):
+    """qkv [K, (Hq + 2 Hkv) d_h] = x [K, d] W^T with RoPE at pos on the query and key heads; the value
+    heads also into v16 [K, Hkv d_h] fp16 when given."""
+    _req(x, "x", torch.bfloat16, 2)
+    _req(W, "W", torch.bfloat16, 2)
+    _req(pos, "pos", torch.int32, 1)
+    _req(qkv, "qkv", torch.bfloat16, 2)
+    _req(v16, "v16", torch.float16, 2)
+    K, d = x.shape
+    cols = (Hq + 2 * Hkv) * d_h
+    if tuple(W.shape) != (cols, d) or not W.is_contiguous():
+        raise ValueError("W must be a contiguous [(Hq + 2 Hkv) d_h, d] tensor")
+    if qkv.shape[0] != K or qkv.shape[1] != cols or qkv.stride(1) != 1 or pos.shape[0] < K:
+        raise ValueError("shape mismatch")
+    if v16 is not None and (tuple(v16.shape) != (K, Hkv * d_h) or not v16.is_contiguous()):
+        raise ValueError("v16 must be a contiguous [K, Hkv d_h] tensor")
+    _check("tg_project_rope", lib().tg_project_rope(
+        _ptr(x), K, d, x.stride(0), _ptr(W), Hq, Hkv, d_h, _ptr(pos), float(base), _ptr(qkv), qkv.stride(0),
+        _ptr(v16), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return qkv
 
 
 def tg_gated_decode(q, k_cache, v_cache, out, workspace, s_cache=None, gain=None, tau: float = 1.0, lse=None,

@@ -150,3 +150,26 @@ def test_backward_workspace_and_argument_errors(lib):
     assert bwd(q=24) == INV                         # misaligned
     assert bwd(ldq=16 * 128 + 4) == INV             # stride not a multiple of 8
     assert bwd(ws_bytes=big - 256) == INV
+
+
+def test_project_rope_workspace_and_argument_errors(lib):
+    vp = ctypes.c_void_p
+    INV, UNS = tg.TG_ERR_INVALID_ARG, tg.TG_ERR_UNSUPPORTED
+    ws = tg.tg_workspace_bytes(tg.TG_OP_PROJECT, 4608, 128)
+    assert ws >= 256 + 4608 * 128 * 4 and ws % 256 == 0       # cos and sin of K rows x d_h / 2
+    assert tg.tg_workspace_bytes(tg.TG_OP_PROJECT, 4608, 96) == 0
+
+    def proj(x=16, K=300, d=2048, ldx=2048, Hq=16, Hkv=8, d_h=128, base=1e6, ldo=4096, v16=None, ws_bytes=ws):
+        return lib.tg_project_rope(vp(x), K, d, ldx, vp(4096), Hq, Hkv, d_h, vp(64), base, vp(8192), ldo,
+                                   vp(v16) if v16 else None, vp(256), ws_bytes, None)
+
+    assert proj(base=0.0) == INV
+    assert proj(d=2000, ldx=2000) == UNS            # d not a multiple of 64
+    assert proj(Hq=15, Hkv=8) == UNS                # (Hq + 2 Hkv) d_h not a multiple of 256
+    assert proj(d_h=96) == UNS
+    assert proj(x=24) == INV                        # misaligned
+    assert proj(ldo=4092) == INV                    # output stride not a multiple of 8
+    assert proj(ldo=2048) == INV                    # output stride shorter than a row
+    assert proj(v16=40) == INV                      # misaligned fp16 copy
+    assert proj(ws_bytes=1024) == INV
+    assert proj(K=0) == tg.TG_OK
