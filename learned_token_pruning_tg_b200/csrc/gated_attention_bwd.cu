@@ -177,6 +177,15 @@ struct CfgQ {
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
 };
 
+// 128-byte-swizzled TMA destinations start on 1024-byte boundaries; everything fits in 227 KB.
+template <int D>
+constexpr bool layout_ok_q() {
+    using C = CfgQ<D>;
+    return C::kOffDO % 1024 == 0 && C::kOffK % 1024 == 0 && C::kOffV % 1024 == 0 && C::kTile % 1024 == 0 &&
+           C::kOffAugA % 16 == 0 && C::kOffAugB % 16 == 0 && C::kOffBar % 8 == 0 && C::kSmem <= 232448;
+}
+static_assert(layout_ok_q<64>() && layout_ok_q<128>(), "dq kernel shared-memory layout");
+
 struct ArgsQ {
     int64_t K, Kp;
     int Hq, G, num_q_tiles;
@@ -481,6 +490,15 @@ struct CfgKV {
     static constexpr int kSmem = kOffMisc + 16 + 1024;
     static constexpr uint32_t kColDV = 256, kColDK = 256 + D;
 };
+
+template <int D>
+constexpr bool layout_ok_kv() {
+    using C = CfgKV<D>;
+    return C::kOffV % 1024 == 0 && C::kOffQ % 1024 == 0 && C::kOffDO % 1024 == 0 && C::kTile % 1024 == 0 &&
+           C::kOffVec % 16 == 0 && C::kOffAugA % 16 == 0 && C::kOffAugB % 16 == 0 && C::kOffBar % 8 == 0 &&
+           C::kSmem <= 232448;
+}
+static_assert(layout_ok_kv<64>() && layout_ok_kv<128>(), "dk/dv kernel shared-memory layout");
 
 struct ArgsKV {
     int64_t K, Kp;

@@ -46,6 +46,9 @@ constexpr int kOffBar = kStages * kStage;
 constexpr int kNumBars = 2 * kStages + 5;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffMisc + 16 + 1024;
+// 128-byte-swizzled TMA destinations start on 1024-byte boundaries; everything fits in 227 KB.
+static_assert(kStageA % 1024 == 0 && kStage % 1024 == 0 && kOffBar % 8 == 0 && kSmem <= 232448,
+              "projection shared-memory layout");
 
 struct Args {
     int64_t K;
