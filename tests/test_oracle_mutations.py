@@ -55,6 +55,7 @@ def test_pins_catch_mutation(name, tmp_path):
     env = dict(os.environ, TG_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         "tests/test_oracle_gate.py", "tests/test_oracle_select.py",
-                        "tests/test_oracle_attention.py", "tests/test_oracle_attention_backward.py"],
+                        "tests/test_oracle_attention.py", "tests/test_oracle_attention_backward.py",
+                        "tests/test_oracle_properties.py"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"no pin caught mutation {name}:\n{r.stdout[-2000:]}"

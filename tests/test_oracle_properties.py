@@ -33,3 +33,44 @@ def test_select_matches_the_specified_order(data):
     scores = np.array(vals, dtype=np.float32)
     got = oracle.topk_select(scores, db, de, k) if N else np.empty(0, np.int32)
     assert list(got) == brute(scores, db, de, k)
+
+
+def _torch_gated_attention(q, k, v, s, g, tau, pos):
+    """The gated attention written with torch ops in fp64 (masked logits, softmax, weighted sum)."""
+    import torch
+    K, Hq, d_h = q.shape
+    G = Hq // k.shape[1]
+    kk, vv = k.repeat_interleave(G, dim=1), v.repeat_interleave(G, dim=1)
+    logits = torch.einsum("rhd,chd->hrc", q, kk) * tau / d_h ** 0.5 + g[:, None, None] * s[None, None, :]
+    logits = logits.masked_fill(~(pos[None, :] <= pos[:, None])[None], float("-inf"))
+    return torch.einsum("hrc,chd->rhd", torch.softmax(logits, dim=-1), vv)
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.data())
+def test_attention_forward_and_backward_match_torch(data):
+    """Random tiny shapes, gains, temperatures and position patterns: the oracle's forward against a
+    torch fp64 forward, and its backward against torch autograd of that forward."""
+    import torch
+    Hkv = data.draw(st.integers(1, 3))
+    G = data.draw(st.sampled_from([1, 2, 4]))
+    Hq, d_h, K = Hkv * G, data.draw(st.sampled_from([2, 4, 8])), data.draw(st.integers(1, 12))
+    tau = data.draw(st.floats(0.25, 3.0))
+    seed = data.draw(st.integers(0, 2 ** 31 - 1))
+    gaps = data.draw(st.booleans())
+    rng = np.random.default_rng(seed)
+    x = {n: rng.standard_normal(shape).astype(np.float32) for n, shape in
+         (("q", (K, Hq, d_h)), ("k", (K, Hkv, d_h)), ("v", (K, Hkv, d_h)), ("dout", (K, Hq, d_h)), ("s", (K,)))}
+    x["g"] = (2.0 * rng.random(Hq)).astype(np.float32)
+    pos = np.sort(rng.choice(5 * K, K, replace=False)).astype(np.int32) if gaps else None
+    want_out = oracle.gated_attention(x["q"], x["k"], x["v"], s=x["s"], g=x["g"], tau=tau, pos=pos)
+    grads = oracle.gated_attention_backward(x["q"], x["k"], x["v"], x["dout"], s=x["s"], g=x["g"], tau=tau, pos=pos)
+    t = {n: torch.tensor(a, dtype=torch.float64, requires_grad=n != "dout") for n, a in x.items()}
+    tt = torch.tensor(tau, dtype=torch.float64, requires_grad=True)
+    tp = torch.arange(K) if pos is None else torch.tensor(pos.astype(np.int64))
+    out = _torch_gated_attention(t["q"], t["k"], t["v"], t["s"], t["g"], tt, tp)
+    np.testing.assert_allclose(want_out, out.detach().numpy(), rtol=1e-10, atol=1e-12)
+    (out * t["dout"]).sum().backward()
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("s", "ds"), ("g", "dg")):
+        np.testing.assert_allclose(grads[key], t[name].grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=key)
+    assert abs(grads["dtau"] - tt.grad.item()) <= 1e-9 * max(1.0, abs(tt.grad.item()))
