@@ -74,3 +74,30 @@ def test_attention_forward_and_backward_match_torch(data):
     for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("s", "ds"), ("g", "dg")):
         np.testing.assert_allclose(grads[key], t[name].grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=key)
     assert abs(grads["dtau"] - tt.grad.item()) <= 1e-9 * max(1.0, abs(tt.grad.item()))
+
+
+@settings(max_examples=80, deadline=None)
+@given(st.data())
+def test_gate_matches_torch_library_ops(data):
+    """Random tiny gate shapes, eps, biases and RMSNorm weights against torch's rms_norm, linear and
+    silu in fp64 (the RMSNorm weight applied exactly: fold_gamma_bf16=False)."""
+    import torch
+    import torch.nn.functional as F
+    N, d, d_g = data.draw(st.integers(1, 9)), data.draw(st.integers(1, 24)), data.draw(st.integers(1, 8))
+    eps = data.draw(st.sampled_from([0.0, 1e-6, 1e-2]))
+    b2 = data.draw(st.floats(-2.0, 2.0))
+    use_b1, use_gamma = data.draw(st.booleans()), data.draw(st.booleans())
+    rng = np.random.default_rng(data.draw(st.integers(0, 2 ** 31 - 1)))
+    h = rng.standard_normal((N, d)).astype(np.float32)
+    if eps == 0.0:
+        h[np.all(h == 0, axis=1)] = 1.0     # no all-zero row when nothing keeps the norm finite
+    W1 = rng.standard_normal((d_g, d)).astype(np.float32)
+    w2 = rng.standard_normal(d_g).astype(np.float32)
+    b1 = rng.standard_normal(d_g).astype(np.float32) if use_b1 else None
+    gamma = (1 + 0.5 * rng.standard_normal(d)).astype(np.float32) if use_gamma else None
+    s = oracle.gate_score(h, W1, w2, b1=b1, b2=b2, gamma=gamma, eps=eps, fold_gamma_bf16=False)
+    x = F.rms_norm(torch.from_numpy(h).double(), (d,), weight=None if gamma is None else
+                   torch.from_numpy(gamma).double(), eps=eps)
+    a = F.silu(F.linear(x, torch.from_numpy(W1).double(), None if b1 is None else torch.from_numpy(b1).double()))
+    ref = (a @ torch.from_numpy(w2).double()) + b2
+    np.testing.assert_allclose(s, ref.numpy(), rtol=1e-9, atol=1e-10)
