@@ -101,3 +101,39 @@ def test_gate_matches_torch_library_ops(data):
     a = F.silu(F.linear(x, torch.from_numpy(W1).double(), None if b1 is None else torch.from_numpy(b1).double()))
     ref = (a @ torch.from_numpy(w2).double()) + b2
     np.testing.assert_allclose(s, ref.numpy(), rtol=1e-9, atol=1e-10)
+
+
+@settings(max_examples=80, deadline=None)
+@given(st.data())
+def test_rope_matches_complex_rotation(data):
+    """Random shapes, positions and bases against numpy's complex multiplication: the rotate-half
+    pair (t, t + d_h/2) is the complex number x_t + i x_{t+d_h/2} turned by pos * base^(-2t/d_h)."""
+    K, H = data.draw(st.integers(1, 6)), data.draw(st.integers(1, 4))
+    d_h = 2 * data.draw(st.integers(1, 16))
+    base = data.draw(st.sampled_from([10.0, 1e4, 1e6]))
+    rng = np.random.default_rng(data.draw(st.integers(0, 2 ** 31 - 1)))
+    x = rng.standard_normal((K, H, d_h)).astype(np.float32)
+    pos = rng.integers(0, 200000, K).astype(np.int32)
+    got = oracle.rope(x, pos, base)
+    half = d_h // 2
+    z = x[..., :half].astype(np.float64) + 1j * x[..., half:].astype(np.float64)
+    ang = pos.astype(np.float64)[:, None, None] * base ** (-2.0 * np.arange(half) / d_h)[None, None, :]
+    w = z * np.exp(1j * ang)
+    np.testing.assert_allclose(got, np.concatenate([w.real, w.imag], axis=-1), rtol=1e-9, atol=1e-9)
+
+
+@settings(max_examples=80, deadline=None)
+@given(st.data())
+def test_gather_matches_fancy_indexing(data):
+    """Random kept sets (ascending, as the select produces them) against numpy fancy indexing of the
+    rows, the positions and the scores."""
+    N, d = data.draw(st.integers(1, 40)), data.draw(st.integers(1, 12))
+    rng = np.random.default_rng(data.draw(st.integers(0, 2 ** 31 - 1)))
+    idx = np.sort(rng.choice(N, data.draw(st.integers(0, N)), replace=False)).astype(np.int32)
+    bits = rng.integers(0, 2 ** 16, (N, d)).astype(np.uint16)
+    pos_in = np.sort(rng.choice(10 * N, N, replace=False)).astype(np.int32)
+    scores = rng.standard_normal(N).astype(np.float32)
+    h_out, pos_out, s_out = oracle.gather_compact(bits, idx, pos_in=pos_in, scores=scores)
+    assert np.array_equal(h_out, bits[idx])
+    assert np.array_equal(pos_out, pos_in[idx])
+    assert np.array_equal(s_out, scores[idx])
