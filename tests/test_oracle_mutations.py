@@ -36,6 +36,8 @@ MUTATIONS = {
     "bwd_ds_no_gain": ("ds[c] += dl * gain;", "ds[c] += dl;"),
     "bwd_kv_head": ("int kv_head = h / group;", "int kv_head = h % Hkv;"),
     "bwd_unnormalised_p": ("prob[c] /= denom;", "(void)denom;"),
+    "rope_frequency_exponent": ("double inv_freq = pow(base, -2.0 * (double)t / (double)d_h);",
+                                "double inv_freq = pow(base, -(double)t / (double)d_h);"),
     "gather_pos_index": ("pos_out[r] = pos_in ? pos_in[i] : (int32_t)i;",
                          "pos_out[r] = pos_in ? pos_in[r] : (int32_t)i;"),
 }
