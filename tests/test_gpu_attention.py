@@ -8,7 +8,6 @@ the kernel's arithmetic (P and V in fp16 for the P V product, the key bias as
 a sum of bf16 part products on the tensor core, fp32 online softmax with
 ex2.approx).  The log-sum-exp agrees to 1e-3.
 """
-import math
 
 import numpy as np
 import pytest
