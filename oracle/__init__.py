@@ -33,6 +33,8 @@ def lib():
         L.tgo_topk_threshold.restype = dbl
         L.tgo_gather_compact.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, vp, vp]
         L.tgo_gather_compact.restype = i32
+        L.tgo_project.argtypes = [vp, i64, i32, i64, vp, i32, vp]
+        L.tgo_project.restype = i32
         L.tgo_rope.argtypes = [vp, i64, i32, i32, vp, dbl, vp]
         L.tgo_rope.restype = i32
         L.tgo_gated_attention.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, dbl, vp, i64, vp, vp]
@@ -142,6 +144,20 @@ def gather_compact(h_bits, idx, pos_in=None, scores=None):
     return h_out, pos_out, s_out
 
 
+def project(x, W):
+    """x [K, d] fp32 values, W [n_out, d] (one row per output feature); returns fp64 [K, n_out]
+    = x W^T."""
+    x = _f32(x)
+    W = _f32(W)
+    K, d = x.shape
+    n_out = W.shape[0]
+    assert W.shape == (n_out, d)
+    out = np.empty((max(K, 1), n_out), dtype=np.float64)
+    if lib().tgo_project(_p(x), K, d, d, _p(W), n_out, _p(out)) != 0:
+        raise ValueError("tgo_project: bad arguments")
+    return out[:K]
+
+
 def rope(x, pos, base=1e6):
     """x: [K, H, d_h] fp32 values; returns fp64 rotated copy."""
     x = _f32(x)
@@ -200,4 +216,4 @@ def gated_attention_backward(q, k, v, dout, s=None, g=None, tau=1.0, pos=None):
 
 
 __all__ = ["lib", "kept_count", "round_bf16", "gate_score", "topk_select", "topk_threshold",
-           "gather_compact", "rope", "gated_attention", "gated_attention_backward"]
+           "gather_compact", "project", "rope", "gated_attention", "gated_attention_backward"]

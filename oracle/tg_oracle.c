@@ -310,6 +310,34 @@ int tgo_rope(const float* x, int64_t K, int H, int d_h, const int32_t* pos,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Q/K/V projection of the kept rows.  Above the gate only the kept tokens
+ * are processed and only they produce keys and values (aiproducthub.cn
+ * article, paragraph 事件详情; chathome.org article, section TokenGate の
+ * 学習可能なトークンプルーニングの仕組み), so the next layer's projections
+ * run on the compacted rows.  A linear map with no bias (Qwen3's attention
+ * projections), weight in the nn.Linear layout, one row per output feature:
+ *   out[r, j] = sum_c x[r, c] * W[j, c].
+ * Stacking Wq, Wk, Wv as the rows of W gives Q, K and V as consecutive
+ * column blocks of out. */
+int tgo_project(const float* x, int64_t K, int d, int64_t ld_x,
+                const float* W, int n_out, double* out)
+{
+    if (!x || !W || !out || K < 0 || d <= 0 || n_out <= 0 || ld_x < d)
+        return -1;
+    for (int64_t r = 0; r < K; ++r) {
+        const float* xr = x + r * ld_x;
+        for (int j = 0; j < n_out; ++j) {
+            const float* wj = W + (size_t)j * (size_t)d;
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += (double)xr[c] * (double)wj[c];
+            out[r * n_out + j] = acc;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Token-gated attention: the kept token's score becomes a bias on the
  * attention logits, plus a learned per-head gain and a learned temperature
  * (aiproducthub.cn article, paragraph 事件详情; aisight.pl article, section

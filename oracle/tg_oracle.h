@@ -100,6 +100,13 @@ int tgo_gather_compact(const uint16_t* h, int64_t N, int d, int64_t ld_h,
 int tgo_rope(const float* x, int64_t K, int H, int d_h, const int32_t* pos,
              double base, double* out);
 
+/* Projection of the kept rows, fp64: out[r, j] = sum_c x[r, c] * W[j, c].
+ * x: [K, ld_x] row-major (first d columns used); W: [n_out, d] (one row per
+ * output feature, so stacked Wq, Wk, Wv give Q, K, V as column blocks);
+ * out: [K, n_out].  Returns 0, or -1 on bad arguments. */
+int tgo_project(const float* x, int64_t K, int d, int64_t ld_x,
+                const float* W, int n_out, double* out);
+
 /* Token-gated causal GQA attention, fp64, for a subset of query rows.
  * q: [K, Hq, d_h], k and v: [K, Hkv, d_h]; query head h reads kv head
  * h / (Hq/Hkv).  s: [K] kept-token scores or NULL (= 0); g: [Hq] or NULL (= 0).

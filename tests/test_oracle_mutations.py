@@ -38,6 +38,10 @@ MUTATIONS = {
     "bwd_unnormalised_p": ("prob[c] /= denom;", "(void)denom;"),
     "rope_frequency_exponent": ("double inv_freq = pow(base, -2.0 * (double)t / (double)d_h);",
                                 "double inv_freq = pow(base, -(double)t / (double)d_h);"),
+    "project_transposed_w": ("acc += (double)xr[c] * (double)wj[c];",
+                             "acc += (double)xr[c] * (double)W[(size_t)c * (size_t)n_out + j];"),
+    "project_drop_last_term": ("for (int c = 0; c < d; ++c)\n                acc += (double)xr[c]",
+                               "for (int c = 0; c < d - 1; ++c)\n                acc += (double)xr[c]"),
     "gather_pos_index": ("pos_out[r] = pos_in ? pos_in[i] : (int32_t)i;",
                          "pos_out[r] = pos_in ? pos_in[r] : (int32_t)i;"),
 }
@@ -58,6 +62,6 @@ def test_pins_catch_mutation(name, tmp_path):
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         "tests/test_oracle_gate.py", "tests/test_oracle_select.py",
                         "tests/test_oracle_attention.py", "tests/test_oracle_attention_backward.py",
-                        "tests/test_oracle_properties.py"],
+                        "tests/test_oracle_properties.py", "tests/test_oracle_project.py"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"no pin caught mutation {name}:\n{r.stdout[-2000:]}"
