@@ -2,8 +2,7 @@
 gradients are the direct backward call's, bit for bit (same kernels, same inputs), and therefore
 match the oracle's backward within the backward's tolerance.
 
-Skipped until its first run on a GPU (the wrapper's plumbing is checked on the CPU with fake
-kernels in tests/test_autograd_host.py; both kernels it calls are covered by their own GPU tests).
+The wrapper's plumbing is also checked on the CPU with fake kernels (tests/test_autograd_host.py).
 """
 import numpy as np
 import pytest
@@ -13,7 +12,7 @@ from learned_token_pruning_tg_b200 import autograd as ag
 from learned_token_pruning_tg_b200 import synth
 from tests.test_gpu_attention_backward import compare, run_gpu, want_grads
 
-pytestmark = [pytest.mark.gpu, pytest.mark.skip(reason="the autograd op has not yet run on a GPU")]
+pytestmark = pytest.mark.gpu
 
 
 def test_autograd_equals_direct_backward_and_oracle():

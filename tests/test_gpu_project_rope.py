@@ -5,9 +5,6 @@ Tolerance: the kernel rotates the fp32 accumulators and rounds once to bf16, so 
 within half a bf16 ulp of the exact value plus fp32 accumulation over d products and fp32 cos / sin
 (2^-20 of the sum of absolute terms bounds both here); the fp16 copy of V is the same accumulator
 rounded to fp16 (half an fp16 ulp, 2^-11 relative, plus the same accumulation bound).
-
-Skipped until the kernel's first run on a GPU: it has been compiled and its host-side checks pass,
-but it has not yet executed on a B200.
 """
 import numpy as np
 import pytest
@@ -17,7 +14,7 @@ import oracle
 from learned_token_pruning_tg_b200 import tokengate as tg
 from tests.guards import guarded
 
-pytestmark = [pytest.mark.gpu, pytest.mark.skip(reason="tg_project_rope has not yet run on a GPU")]
+pytestmark = pytest.mark.gpu
 
 
 def half_ulp_bf16(x):
