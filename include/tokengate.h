@@ -62,7 +62,8 @@ typedef enum {
     TG_ERR_INVALID_ARG = 1,
     TG_ERR_UNSUPPORTED = 2,
     TG_ERR_CUDA = 3,
-    TG_ERR_TIMEOUT = 4
+    TG_ERR_TIMEOUT = 4,
+    TG_ERR_RANGE = 5
 } tg_status;
 
 typedef enum {
@@ -82,6 +83,11 @@ typedef enum {
 #define TG_STATUS_DECODE_TIMEOUT 0x8u
 #define TG_STATUS_BACKWARD_TIMEOUT 0x10u
 #define TG_STATUS_PROJECT_TIMEOUT 0x20u
+/* Not a timeout: a value of V beyond fp16's range (|v| > 65504) was written
+ * into an fp16 copy of V (tg_gated_attention, tg_project_rope); the outputs
+ * that read it are not the specified values. */
+#define TG_STATUS_V_RANGE 0x40u
+#define TG_STATUS_TIMEOUT_BITS 0x3fu
 
 /* Static description of a status code.  Never NULL. */
 const char* tg_status_string(tg_status status);
@@ -120,7 +126,9 @@ size_t tg_workspace_bytes(tg_op op, int64_t N, int32_t d, int32_t d_g);
  * Supported: d a multiple of 64 (64..16384), d_g in {64, 128, 256},
  * N in [0, 2^31).  h, W1 16-byte aligned.
  * Tensor cores (tcgen05, bf16 in, fp32 accumulate in TMEM); the RMS factor,
- * bias, SiLU and the d_g -> 1 projection are applied in the epilogue. */
+ * bias, SiLU and the d_g -> 1 projection are applied in the epilogue.  With
+ * d_g = 256 two CTAs of a cluster share each 256-row tile (one M = 256 MMA per
+ * step, each CTA holding half of W1), where the device offers clusters of 2. */
 tg_status tg_gate_score(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
                         const tg_bf16* rms_weight, float eps,
                         const tg_bf16* W1, const float* b1, const float* w2, float b2,
@@ -136,7 +144,12 @@ tg_status tg_gate_score(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
  * The result is unique, so it is bit-exact with any correct implementation.
  * Supported: N < 2^31 and doc_end - doc_begin <= 2424832 (148 * 1024 * 16).
  * Multi-pass radix select (11/11/10-bit digits of the order-preserving key
- * of each fp32 score) in one cooperative launch. */
+ * of each fp32 score) in one launch: spans of up to 16 * 1024 * 16 = 262144
+ * tokens (131072 on a device that offers clusters of 8 only) in one
+ * thread-block cluster that merges its histograms through distributed shared
+ * memory, longer spans in one cooperative grid that merges them in the
+ * workspace.  The cluster shape writes nothing but kept_idx and waits only at
+ * hardware cluster barriers; the workspace is still required. */
 tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_begin,
                          int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
                          void* workspace, size_t workspace_bytes, void* stream);
@@ -184,8 +197,13 @@ tg_status tg_random_select(int64_t N, int64_t doc_begin, int64_t doc_end, int64_
  *   pos_out[r]  = pos_in ? pos_in[kept_idx[r]] : kept_idx[r]
  *   s_out[r]    = scores[kept_idx[r]]          (if both are non-NULL)
  * h: [N, d] bf16 with row stride ld_h; h_out: [K, d] contiguous.
- * kept_idx entries must lie in [0, N) (not checked on the device).
- * Supported: d a multiple of 8; h, h_out 16-byte aligned, ld_h multiple of 8. */
+ * kept_idx entries are checked on the device: an entry outside [0, N) is not
+ * read; its h_out row is zero-filled, pos_out gets -1 and s_out (if given)
+ * NaN, so any negative pos_out marks a bad index (-2: a row copy that did not
+ * complete within the library's wait limit).
+ * Supported: d a multiple of 8; h, h_out 16-byte aligned, ld_h multiple of 8.
+ * One launch: rows up to 20 KB (d <= 10240) move by the bulk-copy engine, one
+ * row per lane and 32 rows per SM in flight; wider rows by 16-byte loads. */
 tg_status tg_gather_compact(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
                             const int32_t* kept_idx, int64_t K, const int32_t* pos_in,
                             const float* scores, tg_bf16* h_out, int32_t* pos_out,
@@ -216,12 +234,28 @@ tg_status tg_rope_apply(tg_bf16* q, int64_t ld_q, tg_bf16* k, int64_t ld_k,
  * Two launches: V to fp16 into the workspace, then the attention kernel:
  * tensor cores for Q K^T (the key bias added by one extra MMA step) and P V
  * (tcgen05, accumulators in TMEM), K/V tiles staged by TMA, online softmax in
- * fp32, P and V in fp16 for the P V product. */
+ * fp32, P and V in fp16 for the P V product.
+ * Range: V goes through fp16, so |v| must stay within 65504 (fp16's largest
+ * finite value; bf16 reaches 3.4e38).  A larger finite v has no fp16 value:
+ * the conversion sets TG_STATUS_V_RANGE in the workspace's status word
+ * (tg_device_status then returns TG_ERR_RANGE), and the outputs of the rows
+ * that attend to that key are not the specified values. */
 tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
                              const tg_bf16* v, int64_t ld_v, int64_t K, int32_t Hq,
                              int32_t Hkv, int32_t d_h, const float* s_kept,
                              const float* gain, float tau, tg_bf16* out, float* lse,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* tg_gated_attention over a V that is already an fp16 copy, as
+ * tg_project_rope writes it: one launch, no conversion pass.
+ * v16: [K, Hkv, d_h] fp16 (uint16_t bit patterns), dense, 16-byte aligned.
+ * workspace: at least tg_workspace_bytes(TG_OP_ATTENTION, 0, Hkv * d_h, 0)
+ * bytes (the status word; no per-call region).  Every other argument, the
+ * formula and the limits are those of tg_gated_attention. */
+tg_status tg_gated_attention_f16v(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
+                                  const uint16_t* v16, int64_t K, int32_t Hq, int32_t Hkv, int32_t d_h,
+                                  const float* s_kept, const float* gain, float tau, tg_bf16* out,
+                                  float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /* One decoding step of token-gated attention over a KV cache (the layers
  * above the gate layer keep only the kept tokens' keys, each with its gate
@@ -298,7 +332,8 @@ tg_status tg_gated_attention_backward(const tg_bf16* q, int64_t ld_q, const tg_b
  * {64, 128}; x, W, qkv, v16 16-byte aligned.  Two launches: the cos / sin
  * table, then a persistent tcgen05 GEMM (128 x 256 tiles, TMA-staged
  * operands, TMEM accumulators double-buffered against the epilogue).
- * Waits are bounded (TG_STATUS_PROJECT_TIMEOUT). */
+ * Waits are bounded (TG_STATUS_PROJECT_TIMEOUT).  A value head element above
+ * fp16's range (|v| > 65504) written into v16 sets TG_STATUS_V_RANGE. */
 tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int64_t ld_x, const tg_bf16* W, int32_t Hq,
                           int32_t Hkv, int32_t d_h, const int32_t* pos, double base, tg_bf16* qkv, int64_t ld_qkv,
                           uint16_t* v16, void* workspace, size_t workspace_bytes, void* stream);
@@ -316,7 +351,8 @@ tg_status tg_debug_set_select_wait_limit(uint64_t ns);
 
 /* Reads the workspace's status word after synchronizing `stream`.
  * *status_word receives the raw TG_STATUS_* bits (may be NULL).
- * Returns TG_ERR_TIMEOUT if any bit is set, TG_OK otherwise. */
+ * Returns TG_ERR_TIMEOUT if a timeout bit is set, else TG_ERR_RANGE if
+ * TG_STATUS_V_RANGE is set, TG_OK otherwise. */
 tg_status tg_device_status(const void* workspace, uint32_t* status_word, void* stream);
 
 #ifdef __cplusplus

@@ -24,6 +24,8 @@
 //               tiles (one thread per row), handed to the epilogue
 // The accumulators are double-buffered, so the epilogue of tile t overlaps the
 // main loop of tile t+1.  Every wait is bounded (TG_STATUS_GATE_TIMEOUT).
+// For d_g = 256 the same roles run on CTA pairs (gate_score_pair_kernel below),
+// which halves the W bytes each SM moves per stage.
 #include "tg_host.cuh"
 
 namespace tg {
@@ -277,12 +279,319 @@ gate_score_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_const
     }
 }
 
+// ---------------------------------------------------------------- CTA-pair kernel (d_g = 256)
+// The same gate on 256-row tiles shared by the two CTAs of a cluster: one
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16) per 16 columns of h, with
+// each CTA holding its own 128 rows of h and HALF of W (128 of its 256 rows) in
+// its own shared memory.  Per 64-column stage a CTA then moves 16 KB of W
+// instead of 32 KB, and its shared memory supplies (and receives) half as many
+// W bytes -- the single-CTA kernel is bound by shared-memory traffic, W's share
+// of which this halves.  No multicast: every TMA copy lands in the CTA that
+// issues it; only completion is counted on the even CTA's barrier.
+//   both CTAs   warp 0 TMA (own rows of h, own half of W), warps 4-7 epilogue
+//               of own rows, warps 8-11 own rows' sums of squares, warp 1 the
+//               pair's TMEM allocation
+//   even CTA    warp 1 lane 0 issues the pair's MMAs; their completion is
+//               committed to both CTAs' barriers
+constexpr int kPairBN = 128;  // rows of W per CTA
+struct PairCfg {
+    static constexpr int kDG = 256;
+    static constexpr int kStageA = kBM * kBK * 2;       // 16 KB
+    static constexpr int kStageB = kPairBN * kBK * 2;   // 16 KB
+    static constexpr int kStage = kStageA + kStageB;
+    static constexpr int kStages = 6;
+    static constexpr int kTmemCols = 2 * kDG;           // two 256-column accumulators
+    static constexpr int kOffSS = kStages * kStage;
+    static constexpr int kOffW2 = kOffSS + 2 * kBM * 4;
+    static constexpr int kOffB1 = kOffW2 + kDG * 4;
+    static constexpr int kOffBar = kOffB1 + kDG * 4;
+    // full, empty, a_full per stage; acc_full, acc_empty, ss_full, ss_empty per buffer; drain
+    static constexpr int kNumBars = 3 * kStages + 9;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmem = kOffMisc + 16 + 1024;
+};
+static_assert(PairCfg::kStageA % 1024 == 0 && PairCfg::kStage % 1024 == 0 && PairCfg::kOffBar % 8 == 0 &&
+                  PairCfg::kSmem <= 232448,
+              "gate pair kernel shared-memory layout");
+
+__global__ void __launch_bounds__(kThreads, 1)
+gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w,
+                       const Args a) {
+    using C = PairCfg;
+    constexpr int DG = C::kDG;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* ss_s = reinterpret_cast<float*>(smem + C::kOffSS);
+    float* w2_s = reinterpret_cast<float*>(smem + C::kOffW2);
+    float* b1_s = reinterpret_cast<float*>(smem + C::kOffB1);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* full = bars;                      // [S] even CTA: both CTAs' copies of the stage landed
+    uint64_t* empty = bars + C::kStages;        // [S] pair MMA commit + 128 sum-of-squares threads
+    uint64_t* a_full = bars + 2 * C::kStages;   // [S] odd CTA: the even CTA saw `full` (own rows landed)
+    uint64_t* acc_full = bars + 3 * C::kStages; // [2] pair MMA commit -> epilogue (both CTAs)
+    uint64_t* acc_empty = acc_full + 2;         // [2] even CTA: 256 epilogue threads of the pair -> MMA
+    uint64_t* ss_full = acc_full + 4;           // [2] 128 sum-of-squares threads -> epilogue
+    uint64_t* ss_empty = acc_full + 6;          // [2] 128 epilogue threads -> sum-of-squares
+    uint64_t* drain = acc_full + 8;             // [1] MMA completion on the abort path
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank_in();   // 0: issues the MMAs
+    const bool leader = rank == 0;
+    const int64_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+    const int64_t num_tiles = (a.N + 2 * kBM - 1) / (2 * kBM);  // 256-row tiles of the pair
+    const int kb_per_tile = a.d / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + 128);
+            mbar_init(&a_full[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 2 * 128);
+            mbar_init(&ss_full[b], 128);
+            mbar_init(&ss_empty[b], 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmap_h);
+        tma_prefetch_desc(&tmap_w);
+    }
+    for (int j = threadIdx.x; j < DG; j += kThreads) {
+        w2_s[j] = a.w2[j];
+        b1_s[j] = a.b1 ? a.b1[j] : 0.0f;
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers are initialised before either touches the other's
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int last_ph[C::kStages];
+            for (int i = 0; i < C::kStages; ++i) last_ph[i] = -1;
+            for (int64_t t = pair; t < num_tiles && !*abort_flag; t += num_pairs) {
+                const int row0 = static_cast<int>(t * 2 * kBM + rank * kBM);
+                for (int kb = 0; kb < kb_per_tile; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT)) break;
+                    uint8_t* sa = smem + s * C::kStage;
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::kStage);
+                    const uint32_t fb = cluster_addr(&full[s], 0);
+                    tma_load_2d_pair(sa, &tmap_h, fb, kb * kBK, row0, kEvictFirst);
+                    tma_load_2d_pair(sa + C::kStageA, &tmap_w, fb, kb * kBK, static_cast<int>(rank) * kPairBN,
+                                     kEvictLast);
+                    last_ph[s] = static_cast<int>(ph);
+                    if (++s == C::kStages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+            }
+            if (*abort_flag && leader) {
+                // Let every issued copy land before the CTA's shared memory is released.
+                volatile int no_abort = 0;
+                for (int i = 0; i < C::kStages; ++i)
+                    if (last_ph[i] >= 0)
+                        mbar_wait_cluster(&full[i], static_cast<uint32_t>(last_ph[i]), &no_abort, a.status,
+                                          TG_STATUS_GATE_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (leader && lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, DG, false);
+            int s = 0;
+            uint32_t ph = 0;
+            int64_t it = 0;
+            bool ok = true;
+            for (int64_t t = pair; t < num_tiles && ok; t += num_pairs, ++it) {
+                const int buf = static_cast<int>(it & 1);
+                const uint32_t use = static_cast<uint32_t>(it >> 1);
+                if (!mbar_wait_cluster(&acc_empty[buf], (use & 1) ^ 1, abort_flag, a.status,
+                                       TG_STATUS_GATE_TIMEOUT)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * DG);
+                for (int kb = 0; kb < kb_per_tile; ++kb) {
+                    if (!mbar_wait_cluster(&full[s], ph, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_cluster(cluster_addr(&a_full[s], 1));  // the odd CTA's rows have landed too
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * C::kStage);
+                    const uint64_t da = smem_desc_sw128(sa, 16, 1024);
+                    const uint64_t db = smem_desc_sw128(sa + C::kStageA, 16, 1024);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        mma_ss_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    mma_commit_pair_mc(&empty[s], 0x3);
+                    if (++s == C::kStages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (ok) mma_commit_pair_mc(&acc_full[buf], 0x3);
+            }
+            if (!ok) {
+                mma_commit_pair(drain);
+                volatile int no_abort = 0;
+                mbar_wait(drain, 0, &no_abort, a.status, TG_STATUS_GATE_TIMEOUT);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ epilogue (own rows)
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        const float inv_d = 1.0f / static_cast<float>(a.d);
+        const uint32_t acc_empty_leader[2] = {cluster_addr(&acc_empty[0], 0), cluster_addr(&acc_empty[1], 0)};
+        int64_t it = 0;
+        for (int64_t t = pair; t < num_tiles; t += num_pairs, ++it) {
+            const int buf = static_cast<int>(it & 1);
+            const uint32_t par = static_cast<uint32_t>(it >> 1) & 1;
+            bool ok = mbar_wait_cluster(&acc_full[buf], par, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT) &&
+                      mbar_wait(&ss_full[buf], par, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const float r = rsqrtf(ss_s[buf * kBM + row] * inv_d + a.eps);
+            mbar_arrive(&ss_empty[buf]);
+            float acc = 0.0f;
+            const uint32_t taddr = tmem_base + lane_off + static_cast<uint32_t>(buf * DG);
+#pragma unroll 1
+            for (int c0 = 0; c0 < DG; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(taddr + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float u = fmaf(r, __uint_as_float(v[j]), b1_s[c0 + j]);
+                    const float e = __expf(fminf(-u, 80.0f));
+                    acc = fmaf(__fdividef(u, 1.0f + e), w2_s[c0 + j], acc);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(acc_empty_leader[buf]);
+            const int64_t grow = t * 2 * kBM + static_cast<int64_t>(rank) * kBM + row;
+            if (grow < a.N) a.scores[grow] = acc + a.b2;
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ row sums of squares (own rows)
+        const int row = (warp - 8) * 32 + lane;
+        const int sw = row & 7;
+        uint64_t* landed = leader ? full : a_full;
+        int s = 0;
+        uint32_t ph = 0;
+        int64_t it = 0;
+        bool ok = true;
+        for (int64_t t = pair; t < num_tiles && ok; t += num_pairs, ++it) {
+            float ss0 = 0.0f, ss1 = 0.0f;
+            for (int kb = 0; kb < kb_per_tile; ++kb) {
+                if (!mbar_wait_cluster(&landed[s], ph, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* rp = smem + s * C::kStage + row * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(rp + ((c ^ sw) << 4));
+                    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float lo = __uint_as_float(w[e] << 16);
+                        const float hi = __uint_as_float(w[e] & 0xffff0000u);
+                        ss0 = fmaf(lo, lo, ss0);
+                        ss1 = fmaf(hi, hi, ss1);
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&empty[s]);
+                if (++s == C::kStages) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+            if (!ok) break;
+            const int buf = static_cast<int>(it & 1);
+            const uint32_t use = static_cast<uint32_t>(it >> 1);
+            if (!mbar_wait(&ss_empty[buf], (use & 1) ^ 1, abort_flag, a.status, TG_STATUS_GATE_TIMEOUT)) break;
+            ss_s[buf * kBM + row] = ss0 + ss1;
+            mbar_arrive(&ss_full[buf]);
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync_all();  // neither CTA leaves while the other may still read its barriers or shared memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    }
+}
+
 // W'_jc = bf16(gamma_c * W1_jc): the RMSNorm weight folded into the first layer.
 __global__ void fold_gamma_kernel(const __nv_bfloat16* __restrict__ W1, const __nv_bfloat16* __restrict__ gamma,
                                   __nv_bfloat16* __restrict__ out, int d, int64_t total) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride)
         out[i] = __float2bfloat16_rn(__bfloat162float(W1[i]) * __bfloat162float(gamma[i % d]));
+}
+
+// Whether this device runs the pair kernel (clusters of 2 with its shared memory), queried once per device.
+static bool pair_kernel_available() {
+    static std::atomic<int> cache[64];
+    const int dev = current_device();
+    if (dev >= 0 && cache[dev].load() != 0) return cache[dev].load() == 2;
+    static std::atomic<int> smem_set[64];
+    bool ok = set_max_dynamic_smem(gate_score_pair_kernel, PairCfg::kSmem, smem_set);
+    if (ok) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = PairCfg::kSmem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        ok = cudaOccupancyMaxActiveClusters(&n, gate_score_pair_kernel, &cfg) == cudaSuccess && n >= 1;
+        cudaGetLastError();
+    }
+    if (dev >= 0) cache[dev].store(ok ? 2 : 1);
+    return ok;
+}
+
+static tg_status launch_pair(const CUtensorMap& mh, const CUtensorMap& mw, const Args& a, cudaStream_t st) {
+    const int64_t pair_tiles = (a.N + 2 * kBM - 1) / (2 * kBM);
+    const int pairs = static_cast<int>(std::min<int64_t>(pair_tiles, num_sms() / 2));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = PairCfg::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gate_score_pair_kernel, mh, mw, a) == cudaSuccess ? TG_OK : TG_ERR_CUDA;
 }
 
 template <int DG>
@@ -347,6 +656,13 @@ extern "C" tg_status tg_gate_score(const tg_bf16* h, int64_t N, int32_t d, int64
     a.scores = scores;
     a.status = status_word(workspace);
     const int64_t num_tiles = (N + gate::kBM - 1) / gate::kBM;
+    if (d_g == 256 && gate::pair_kernel_available()) {
+        // W's half tile: 128 rows per CTA
+        CUtensorMap mw2;
+        const uint32_t wb2[2] = {gate::kBK, static_cast<uint32_t>(gate::kPairBN)};
+        if (!make_tmap_bf16(&mw2, wsrc, 2, wd, wsd, wb2)) return TG_ERR_CUDA;
+        return gate::launch_pair(mh, mw2, a, st);
+    }
     switch (d_g) {
         case 64: return gate::launch<64>(mh, mw, a, num_tiles, st);
         case 128: return gate::launch<128>(mh, mw, a, num_tiles, st);

@@ -30,9 +30,9 @@
 //               warp w owns TMEM lanes 32 (w mod 4) ..): the row's 128 S values
 //               are read from TMEM into registers, row max, then
 //               P = 2^(S c - m) with c = tau / sqrt(d_h) log2(e), as fp16 into
-//               the S columns.
+//               the S columns (packed fp16 ex2: two values per MUFU operation).
 //               Lazy rescaling: O is rescaled (in TMEM) only when a row max
-//               grows by more than 2^8, so P <= 256.  Causal masking only on
+//               grows by more than 2^2, so P <= 4.  Causal masking only on
 //               the diagonal tile.  At the end O / l to bf16 and the
 //               log-sum-exp.
 // The key bias rides in the tensor core: S is computed as
@@ -53,6 +53,8 @@
 // wait is bounded (TG_STATUS_ATTENTION_TIMEOUT).
 #include <cmath>
 
+#include <cfloat>
+
 #include "tg_host.cuh"
 
 namespace tg {
@@ -61,7 +63,10 @@ namespace attn {
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kBN = 128;        // keys per tile
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+// log2 units: O is rescaled when a row's max grows by more than 2, so every exponent
+// y = S c - m stays <= 2 and P <= 4 (the exponent goes through fp16, whose
+// absolute error grows with |y|; see the softmax below)
+constexpr float kRescaleThreshold = 2.0f;
 
 template <int D, int NQ>
 struct Cfg {
@@ -104,6 +109,26 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for both halves of a packed fp16 pair (one MUFU operation for two values).
+__device__ __forceinline__ uint32_t ex2_h2(uint32_t x) {
+    uint32_t y;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+// fp16 pair sum and its widening to fp32.
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ float2 h2_to_f2(uint32_t h) {
+    float lo, hi;
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.f32.f16 %0, l;\n cvt.f32.f16 %1, h;\n}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h));
+    return make_float2(lo, hi);
 }
 
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
@@ -455,9 +480,15 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                     tmem_st16(o_addr + c0, v);
                 }
             }
-            // P = 2^(S c - m) as fp16 over the first kBN / 2 S columns (already read)
+            // P = 2^(S c - m) as fp16 over the first kBN / 2 S columns (already read).  The exponent
+            // y = S c - m is formed in fp32, rounded to an fp16 pair, and raised by one packed ex2
+            // (two values per MUFU operation, already the fp16 pair the P V product reads).  The
+            // rounding of y to fp16 changes P by at most 2^-11 |y| ln 2 of itself: 0.07% for the
+            // largest weights (|y| <= 2, the rescale threshold), 0.5% at y = -16 where P < 2^-16.
+            // The row sum l adds the same fp16 values, four per fp16 lane (at most 16) and then
+            // in fp32.
             const float2 neg_m = make_float2(-m_run, -m_run);
-            float2 ls[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+            float2 ls = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int c0 = 0; c0 < kBN; c0 += 32) {
                 uint32_t p16[16];
@@ -465,18 +496,16 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 for (int i = 0; i < 32; i += 4) {
                     const float2 y0 = ffma2(make_float2(x[c0 + i], x[c0 + i + 1]), sc2, neg_m);
                     const float2 y1 = ffma2(make_float2(x[c0 + i + 2], x[c0 + i + 3]), sc2, neg_m);
-                    const float2 p0 = make_float2(ex2(y0.x), ex2(y0.y));
-                    const float2 p1 = make_float2(ex2(y1.x), ex2(y1.y));
-                    ls[0] = fadd2(ls[0], p0);
-                    ls[1] = fadd2(ls[1], p1);
-                    p16[i / 2] = f16x2(p0.x, p0.y);
-                    p16[i / 2 + 1] = f16x2(p1.x, p1.y);
+                    p16[i / 2] = ex2_h2(f16x2(y0.x, y0.y));
+                    p16[i / 2 + 1] = ex2_h2(f16x2(y1.x, y1.y));
                 }
+#pragma unroll
+                for (int g = 0; g < 16; g += 4)
+                    ls = fadd2(ls, h2_to_f2(hadd2(hadd2(p16[g], p16[g + 1]), hadd2(p16[g + 2], p16[g + 3]))));
                 tmem_st16(s_addr + (c0 >> 1), p16);
             }
-            const float2 lsum = fadd2(ls[0], ls[1]);
             tmem_st_wait();
-            l_run += lsum.x + lsum.y;
+            l_run += ls.x + ls.y;
             tc_fence_before();
             mbar_arrive(&p_full[h]);
         }
@@ -516,18 +545,26 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
 }
 
 // V [K, Hkv d_h] bf16 (token stride ld_v) -> dense fp16 [K, Hkv d_h], eight
-// elements per 16-byte load and store.
+// elements per 16-byte load and store.  A finite value above fp16's range
+// (|v| > 65504) becomes +-inf in the copy; the kernel then sets
+// TG_STATUS_V_RANGE in the status word so the caller learns of it.
 __global__ void __launch_bounds__(128) v_to_f16_kernel(const uint4* __restrict__ v, int64_t ld_v8, int64_t K,
-                                                       int w8, uint4* __restrict__ v16) {
+                                                       int w8, uint4* __restrict__ v16, unsigned int* status) {
+    bool out_of_range = false;
     for (int64_t r = blockIdx.x; r < K; r += gridDim.x) {
         for (int c = threadIdx.x; c < w8; c += blockDim.x) {
             const uint4 x = v[r * ld_v8 + c];
             uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) w[e] = f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+                out_of_range |= (fabsf(lo) > 65504.0f && fabsf(lo) <= FLT_MAX) || (fabsf(hi) > 65504.0f && fabsf(hi) <= FLT_MAX);
+                w[e] = f16x2(lo, hi);
+            }
             v16[r * w8 + c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     }
+    if (out_of_range) atomicOr(status, TG_STATUS_V_RANGE);
 }
 
 template <int D, int NQ>
@@ -550,33 +587,12 @@ static tg_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
 
 using namespace tg;
 
-extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
-                                        const tg_bf16* v, int64_t ld_v, int64_t K, int32_t Hq, int32_t Hkv,
-                                        int32_t d_h, const float* s_kept, const float* gain, float tau,
-                                        tg_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
-                                        void* stream) {
-    if (K < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || !std::isfinite(tau) || !(tau > 0.0f))
-        return TG_ERR_INVALID_ARG;
-    if (d_h != 64 && d_h != 128) return TG_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TG_ERR_INVALID_ARG;
-    if (K == 0) return TG_OK;
-    if (K > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
-    if (!q || !k || !v || !out || !workspace || !aligned16(workspace)) return TG_ERR_INVALID_ARG;
-    if (workspace_bytes < tg_workspace_bytes(TG_OP_ATTENTION, K, Hkv * d_h, 0)) return TG_ERR_INVALID_ARG;
-    if (ld_q < static_cast<int64_t>(Hq) * d_h || ld_k < static_cast<int64_t>(Hkv) * d_h ||
-        ld_v < static_cast<int64_t>(Hkv) * d_h || (ld_q % 8) || (ld_k % 8) || (ld_v % 8))
-        return TG_ERR_INVALID_ARG;
-
-    // fp16 copy of V in the workspace, dense [K, Hkv, d_h]
-    void* v16 = static_cast<char*>(workspace) + ws_gate_offset();
-    cudaStream_t st = as_stream(stream);
-    {
-        const int w8 = Hkv * d_h / 8;
-        const int64_t grid = K < static_cast<int64_t>(num_sms()) * 16 ? K : static_cast<int64_t>(num_sms()) * 16;
-        attn::v_to_f16_kernel<<<static_cast<unsigned>(grid), 128, 0, st>>>(
-            reinterpret_cast<const uint4*>(v), ld_v / 8, K, w8, reinterpret_cast<uint4*>(v16));
-        if (launch_status() != TG_OK) return TG_ERR_CUDA;
-    }
+// Shared by both entry points: checks, tensor maps and the launch over a dense
+// fp16 V ([K, Hkv, d_h]) that is already in device memory.
+static tg_status attention_over_v16(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k, const void* v16,
+                                    int64_t K, int32_t Hq, int32_t Hkv, int32_t d_h, const float* s_kept,
+                                    const float* gain, float tau, tg_bf16* out, float* lse, void* workspace,
+                                    cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const uint32_t qbox[3] = {64, 1, 128};
     const uint32_t kvbox[3] = {64, 1, static_cast<uint32_t>(attn::kBN)};
@@ -608,4 +624,56 @@ extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg
     const bool pairs = ((Hq / Hkv) % 2) == 0;
     if (d_h == 128) return pairs ? attn::launch<128, 2>(mq, mk, mv, a, st) : attn::launch<128, 1>(mq, mk, mv, a, st);
     return pairs ? attn::launch<64, 2>(mq, mk, mv, a, st) : attn::launch<64, 1>(mq, mk, mv, a, st);
+}
+
+static tg_status check_attention_args(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k, int64_t K,
+                                      int32_t Hq, int32_t Hkv, int32_t d_h, float tau, const tg_bf16* out) {
+    if (K < 0 || Hq <= 0 || Hkv <= 0 || (Hq % Hkv) != 0 || !std::isfinite(tau) || !(tau > 0.0f))
+        return TG_ERR_INVALID_ARG;
+    if (d_h != 64 && d_h != 128) return TG_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(out)) return TG_ERR_INVALID_ARG;
+    if (K > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
+    if (ld_q < static_cast<int64_t>(Hq) * d_h || ld_k < static_cast<int64_t>(Hkv) * d_h || (ld_q % 8) || (ld_k % 8))
+        return TG_ERR_INVALID_ARG;
+    return TG_OK;
+}
+
+extern "C" tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
+                                        const tg_bf16* v, int64_t ld_v, int64_t K, int32_t Hq, int32_t Hkv,
+                                        int32_t d_h, const float* s_kept, const float* gain, float tau,
+                                        tg_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+    const tg_status chk = check_attention_args(q, ld_q, k, ld_k, K, Hq, Hkv, d_h, tau, out);
+    if (chk != TG_OK) return chk;
+    if (!aligned16(v)) return TG_ERR_INVALID_ARG;
+    if (K == 0) return TG_OK;
+    if (!q || !k || !v || !out || !workspace || !aligned16(workspace)) return TG_ERR_INVALID_ARG;
+    if (workspace_bytes < tg_workspace_bytes(TG_OP_ATTENTION, K, Hkv * d_h, 0)) return TG_ERR_INVALID_ARG;
+    if (ld_v < static_cast<int64_t>(Hkv) * d_h || (ld_v % 8)) return TG_ERR_INVALID_ARG;
+
+    // fp16 copy of V in the workspace, dense [K, Hkv, d_h]
+    void* v16 = static_cast<char*>(workspace) + ws_gate_offset();
+    cudaStream_t st = as_stream(stream);
+    {
+        const int w8 = Hkv * d_h / 8;
+        const int64_t grid = K < static_cast<int64_t>(num_sms()) * 16 ? K : static_cast<int64_t>(num_sms()) * 16;
+        attn::v_to_f16_kernel<<<static_cast<unsigned>(grid), 128, 0, st>>>(
+            reinterpret_cast<const uint4*>(v), ld_v / 8, K, w8, reinterpret_cast<uint4*>(v16), status_word(workspace));
+        if (launch_status() != TG_OK) return TG_ERR_CUDA;
+    }
+    return attention_over_v16(q, ld_q, k, ld_k, v16, K, Hq, Hkv, d_h, s_kept, gain, tau, out, lse, workspace, st);
+}
+
+extern "C" tg_status tg_gated_attention_f16v(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
+                                             const uint16_t* v16, int64_t K, int32_t Hq, int32_t Hkv, int32_t d_h,
+                                             const float* s_kept, const float* gain, float tau, tg_bf16* out,
+                                             float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    const tg_status chk = check_attention_args(q, ld_q, k, ld_k, K, Hq, Hkv, d_h, tau, out);
+    if (chk != TG_OK) return chk;
+    if (!aligned16(v16)) return TG_ERR_INVALID_ARG;
+    if (K == 0) return TG_OK;
+    if (!q || !k || !v16 || !out || !workspace || !aligned16(workspace)) return TG_ERR_INVALID_ARG;
+    if (workspace_bytes < tg_workspace_bytes(TG_OP_ATTENTION, 0, Hkv * d_h, 0)) return TG_ERR_INVALID_ARG;
+    return attention_over_v16(q, ld_q, k, ld_k, v16, K, Hq, Hkv, d_h, s_kept, gain, tau, out, lse, workspace,
+                              as_stream(stream));
 }

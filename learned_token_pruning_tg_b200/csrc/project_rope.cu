@@ -25,6 +25,9 @@
 //   warps 4-7   epilogue, one row per thread, double-buffered with the next
 //               tile's main loop
 // Every wait is bounded (TG_STATUS_PROJECT_TIMEOUT).
+// Where the device offers clusters of 2, the same roles run on CTA pairs with
+// 256 x 256 tiles (project_rope_pair_kernel below), which halves the W bytes
+// each SM moves per stage.
 #include <cuda_fp16.h>
 
 #include <cmath>
@@ -82,6 +85,85 @@ __global__ void __launch_bounds__(64) rope_table_kernel(const int32_t* __restric
             sincos(p * inv_freq, &s, &c);
             cos_t[r * half + t] = static_cast<float>(c);
             sin_t[r * half + t] = static_cast<float>(s);
+        }
+    }
+}
+
+// One output tile's epilogue for the thread that owns TMEM lane `row` (row
+// `grow` of qkv): the 128 x 256 fp32 accumulator at `taddr` (this thread's
+// lane), column tile `ct`.  Query and key heads are rotated and stored in
+// bf16; value heads are stored in bf16 and, when asked, fp16.
+__device__ __forceinline__ void epilogue_tile(const Args& a, uint32_t taddr, int64_t grow, int ct, bool& v_range) {
+    const bool live = grow < a.K;
+    const int D = a.D, half = a.D >> 1;
+    __nv_bfloat16* orow = a.qkv + grow * a.ld_qkv + static_cast<int64_t>(ct) * kBN;
+    for (int c_head = 0; c_head < kBN; c_head += D) {
+        const int head = (ct * kBN + c_head) / D;
+        if (head < a.Hq + a.Hkv) {
+            // rotate-half pairs (t, t + D/2) of a query or key head, 32 pairs at a time
+            for (int t0 = 0; t0 < half; t0 += 32) {
+                uint32_t x1[32], x2[32];
+                tmem_ld32(taddr + c_head + t0, x1);
+                tmem_ld32(taddr + c_head + half + t0, x2);
+                tmem_ld_wait();
+                if (live) {
+                    const float4* cp = reinterpret_cast<const float4*>(a.cos_t + grow * half + t0);
+                    const float4* sp = reinterpret_cast<const float4*>(a.sin_t + grow * half + t0);
+                    uint32_t o1[16], o2[16];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 c4 = cp[i], s4 = sp[i];
+                        const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+                        float r1[4], r2[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float u = __uint_as_float(x1[4 * i + e]);
+                            const float w = __uint_as_float(x2[4 * i + e]);
+                            r1[e] = u * cc[e] - w * ss[e];
+                            r2[e] = w * cc[e] + u * ss[e];
+                        }
+                        o1[2 * i] = pack_bf16x2(r1[0], r1[1]);
+                        o1[2 * i + 1] = pack_bf16x2(r1[2], r1[3]);
+                        o2[2 * i] = pack_bf16x2(r2[0], r2[1]);
+                        o2[2 * i + 1] = pack_bf16x2(r2[2], r2[3]);
+                    }
+                    uint4* d1 = reinterpret_cast<uint4*>(orow + c_head + t0);
+                    uint4* d2 = reinterpret_cast<uint4*>(orow + c_head + half + t0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        d1[i] = make_uint4(o1[4 * i], o1[4 * i + 1], o1[4 * i + 2], o1[4 * i + 3]);
+                        d2[i] = make_uint4(o2[4 * i], o2[4 * i + 1], o2[4 * i + 2], o2[4 * i + 3]);
+                    }
+                }
+            }
+        } else {
+            // a value head: bf16 into qkv and fp16 into v16
+            const int vh = head - a.Hq - a.Hkv;
+            for (int t0 = 0; t0 < D; t0 += 32) {
+                uint32_t x[32];
+                tmem_ld32(taddr + c_head + t0, x);
+                tmem_ld_wait();
+                if (live) {
+                    uint32_t ob[16], oh[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float lo = __uint_as_float(x[2 * i]), hi = __uint_as_float(x[2 * i + 1]);
+                        ob[i] = pack_bf16x2(lo, hi);
+                        oh[i] = pack_f16x2(lo, hi);
+                        v_range |= fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f;
+                    }
+                    uint4* db = reinterpret_cast<uint4*>(orow + c_head + t0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) db[i] = make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+                    if (a.v16) {
+                        uint4* dh = reinterpret_cast<uint4*>(a.v16 + grow * (static_cast<int64_t>(a.Hkv) * D) +
+                                                             static_cast<int64_t>(vh) * D + t0);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dh[i] = make_uint4(oh[4 * i], oh[4 * i + 1], oh[4 * i + 2], oh[4 * i + 3]);
+                    }
+                }
+            }
         }
     }
 }
@@ -205,7 +287,7 @@ project_rope_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         const int qd = warp & 3;             // TMEM lane quarter of this warp
         const int row = qd * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
-        const int D = a.D, half = a.D >> 1;
+        bool v_range = false;  // a value beyond fp16's range went into the fp16 copy of V
         int64_t it = 0;
         for (int64_t t = blockIdx.x; t < a.num_tiles; t += gridDim.x, ++it) {
             const int rt = static_cast<int>(t / a.num_col_tiles);
@@ -217,80 +299,11 @@ project_rope_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const int64_t grow = static_cast<int64_t>(rt) * kBM + row;
-            const bool live = grow < a.K;
-            const uint32_t taddr = tmem_base + lane_off + static_cast<uint32_t>(buf * kBN);
-            __nv_bfloat16* orow = a.qkv + grow * a.ld_qkv + static_cast<int64_t>(ct) * kBN;
-            for (int c_head = 0; c_head < kBN; c_head += D) {
-                const int head = (ct * kBN + c_head) / D;
-                if (head < a.Hq + a.Hkv) {
-                    // rotate-half pairs (t, t + D/2) of a query or key head, 32 pairs at a time
-                    for (int t0 = 0; t0 < half; t0 += 32) {
-                        uint32_t x1[32], x2[32];
-                        tmem_ld32(taddr + c_head + t0, x1);
-                        tmem_ld32(taddr + c_head + half + t0, x2);
-                        tmem_ld_wait();
-                        if (live) {
-                            const float4* cp = reinterpret_cast<const float4*>(a.cos_t + grow * half + t0);
-                            const float4* sp = reinterpret_cast<const float4*>(a.sin_t + grow * half + t0);
-                            uint32_t o1[16], o2[16];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const float4 c4 = cp[i], s4 = sp[i];
-                                const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
-                                float r1[4], r2[4];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const float u = __uint_as_float(x1[4 * i + e]);
-                                    const float w = __uint_as_float(x2[4 * i + e]);
-                                    r1[e] = u * cc[e] - w * ss[e];
-                                    r2[e] = w * cc[e] + u * ss[e];
-                                }
-                                o1[2 * i] = pack_bf16x2(r1[0], r1[1]);
-                                o1[2 * i + 1] = pack_bf16x2(r1[2], r1[3]);
-                                o2[2 * i] = pack_bf16x2(r2[0], r2[1]);
-                                o2[2 * i + 1] = pack_bf16x2(r2[2], r2[3]);
-                            }
-                            uint4* d1 = reinterpret_cast<uint4*>(orow + c_head + t0);
-                            uint4* d2 = reinterpret_cast<uint4*>(orow + c_head + half + t0);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                d1[i] = make_uint4(o1[4 * i], o1[4 * i + 1], o1[4 * i + 2], o1[4 * i + 3]);
-                                d2[i] = make_uint4(o2[4 * i], o2[4 * i + 1], o2[4 * i + 2], o2[4 * i + 3]);
-                            }
-                        }
-                    }
-                } else {
-                    // a value head: bf16 into qkv and fp16 into v16
-                    const int vh = head - a.Hq - a.Hkv;
-                    for (int t0 = 0; t0 < D; t0 += 32) {
-                        uint32_t x[32];
-                        tmem_ld32(taddr + c_head + t0, x);
-                        tmem_ld_wait();
-                        if (live) {
-                            uint32_t ob[16], oh[16];
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const float lo = __uint_as_float(x[2 * i]), hi = __uint_as_float(x[2 * i + 1]);
-                                ob[i] = pack_bf16x2(lo, hi);
-                                oh[i] = pack_f16x2(lo, hi);
-                            }
-                            uint4* db = reinterpret_cast<uint4*>(orow + c_head + t0);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) db[i] = make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
-                            if (a.v16) {
-                                uint4* dh = reinterpret_cast<uint4*>(a.v16 + grow * (static_cast<int64_t>(a.Hkv) * D) +
-                                                                     static_cast<int64_t>(vh) * D + t0);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    dh[i] = make_uint4(oh[4 * i], oh[4 * i + 1], oh[4 * i + 2], oh[4 * i + 3]);
-                            }
-                        }
-                    }
-                }
-            }
+            epilogue_tile(a, tmem_base + lane_off + static_cast<uint32_t>(buf * kBN), grow, ct, v_range);
             tc_fence_before();
             mbar_arrive(&acc_empty[buf]);
         }
+        if (v_range && a.v16) atomicOr(a.status, TG_STATUS_V_RANGE);
     }
 
     tc_fence_before();
@@ -299,6 +312,206 @@ project_rope_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         tc_fence_after();
         tmem_dealloc(tmem_base, 2 * kBN);
     }
+}
+
+// The same projection on CTA pairs: the two CTAs of a cluster share 256 x 256
+// output tiles through one tcgen05.mma.cta_group::2 (M = 256) per 16 columns of
+// x; each CTA holds its own 128 rows of x and 128 of the tile's 256 rows of W
+// in its own shared memory and receives its 128 rows of the accumulator in its
+// own TMEM.  Per 64-column stage a CTA moves 32 KB instead of 48 KB (half of
+// W), which is what bounds the single-CTA kernel.  No multicast: every TMA copy
+// lands in the CTA that issues it; only its completion is counted on the even
+// CTA's barrier, whose thread issues the pair's MMAs.
+constexpr int kPairStageA = kBM * kBK * 2;          // 16 KB: 128 rows of x
+constexpr int kPairStageB = (kBN / 2) * kBK * 2;    // 16 KB: 128 rows of W
+constexpr int kPairStage = kPairStageA + kPairStageB;
+constexpr int kPairStages = 6;
+constexpr int kPairOffBar = kPairStages * kPairStage;
+constexpr int kPairNumBars = 2 * kPairStages + 5;
+constexpr int kPairOffMisc = kPairOffBar + kPairNumBars * 8;
+constexpr int kPairSmem = kPairOffMisc + 16 + 1024;
+static_assert(kPairStageA % 1024 == 0 && kPairStage % 1024 == 0 && kPairOffBar % 8 == 0 && kPairSmem <= 232448,
+              "projection pair kernel shared-memory layout");
+
+__global__ void __launch_bounds__(kThreads, 1)
+project_rope_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                         const Args a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPairOffBar);
+    uint64_t* full = bars;                        // [S] even CTA: both CTAs' copies of the stage landed
+    uint64_t* empty = bars + kPairStages;         // [S] pair MMA commit -> each CTA's producer
+    uint64_t* acc_full = bars + 2 * kPairStages;  // [2] pair MMA commit -> epilogue (both CTAs)
+    uint64_t* acc_empty = acc_full + 2;           // [2] even CTA: 256 epilogue threads of the pair -> MMA
+    uint64_t* drain = acc_full + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kPairOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kPairOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank_in();
+    const bool leader = rank == 0;
+    const int64_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+    const int kb_per_tile = a.d / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 2 * 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmap_x);
+        tma_prefetch_desc(&tmap_w);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, 2 * kBN);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers are initialised before either touches the other's
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int last_ph[kPairStages];
+            for (int i = 0; i < kPairStages; ++i) last_ph[i] = -1;
+            for (int64_t t = pair; t < a.num_tiles && !*abort_flag; t += num_pairs) {
+                const int rt = static_cast<int>(t / a.num_col_tiles);
+                const int ct = static_cast<int>(t % a.num_col_tiles);
+                for (int kb = 0; kb < kb_per_tile; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT)) break;
+                    uint8_t* sa = smem + s * kPairStage;
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStage);
+                    const uint32_t fb = cluster_addr(&full[s], 0);
+                    tma_load_2d_pair(sa, &tmap_x, fb, kb * kBK, rt * 2 * kBM + static_cast<int>(rank) * kBM,
+                                     kEvictLast);
+                    tma_load_2d_pair(sa + kPairStageA, &tmap_w, fb, kb * kBK,
+                                     ct * kBN + static_cast<int>(rank) * (kBN / 2), kEvictLast);
+                    last_ph[s] = static_cast<int>(ph);
+                    if (++s == kPairStages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+            }
+            if (*abort_flag && leader) {
+                volatile int no_abort = 0;
+                for (int i = 0; i < kPairStages; ++i)
+                    if (last_ph[i] >= 0)
+                        mbar_wait_cluster(&full[i], static_cast<uint32_t>(last_ph[i]), &no_abort, a.status,
+                                          TG_STATUS_PROJECT_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (leader && lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, false);
+            int s = 0;
+            uint32_t ph = 0;
+            int64_t it = 0;
+            bool ok = true;
+            for (int64_t t = pair; t < a.num_tiles && ok; t += num_pairs, ++it) {
+                const int buf = static_cast<int>(it & 1);
+                const uint32_t use = static_cast<uint32_t>(it >> 1);
+                if (!mbar_wait_cluster(&acc_empty[buf], (use & 1) ^ 1, abort_flag, a.status,
+                                       TG_STATUS_PROJECT_TIMEOUT)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
+                for (int kb = 0; kb < kb_per_tile; ++kb) {
+                    if (!mbar_wait_cluster(&full[s], ph, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * kPairStage);
+                    const uint64_t da = smem_desc_sw128(sa, 16, 1024);
+                    const uint64_t db = smem_desc_sw128(sa + kPairStageA, 16, 1024);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        mma_ss_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    mma_commit_pair_mc(&empty[s], 0x3);
+                    if (++s == kPairStages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (ok) mma_commit_pair_mc(&acc_full[buf], 0x3);
+            }
+            if (!ok) {
+                mma_commit_pair(drain);
+                volatile int no_abort = 0;
+                mbar_wait(drain, 0, &no_abort, a.status, TG_STATUS_PROJECT_TIMEOUT);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue (own 128 rows)
+        const int qd = warp & 3;
+        const int row = qd * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
+        const uint32_t acc_empty_leader[2] = {cluster_addr(&acc_empty[0], 0), cluster_addr(&acc_empty[1], 0)};
+        bool v_range = false;
+        int64_t it = 0;
+        for (int64_t t = pair; t < a.num_tiles; t += num_pairs, ++it) {
+            const int rt = static_cast<int>(t / a.num_col_tiles);
+            const int ct = static_cast<int>(t % a.num_col_tiles);
+            const int buf = static_cast<int>(it & 1);
+            const uint32_t par = static_cast<uint32_t>(it >> 1) & 1;
+            const bool ok = mbar_wait_cluster(&acc_full[buf], par, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int64_t grow = static_cast<int64_t>(rt) * 2 * kBM + static_cast<int64_t>(rank) * kBM + row;
+            epilogue_tile(a, tmem_base + lane_off + static_cast<uint32_t>(buf * kBN), grow, ct, v_range);
+            tc_fence_before();
+            mbar_arrive_cluster(acc_empty_leader[buf]);
+        }
+        if (v_range && a.v16) atomicOr(a.status, TG_STATUS_V_RANGE);
+    }
+
+    tc_fence_before();
+    cluster_sync_all();  // neither CTA leaves while the other may still read its barriers or shared memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, 2 * kBN);
+    }
+}
+
+// Whether this device runs the pair kernel (clusters of 2 with its shared memory), once per device.
+static bool pair_kernel_available() {
+    static std::atomic<int> cache[64];
+    const int dev = current_device();
+    if (dev >= 0 && cache[dev].load() != 0) return cache[dev].load() == 2;
+    static std::atomic<int> smem_set[64];
+    bool ok = set_max_dynamic_smem(project_rope_pair_kernel, kPairSmem, smem_set);
+    if (ok) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kPairSmem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        ok = cudaOccupancyMaxActiveClusters(&n, project_rope_pair_kernel, &cfg) == cudaSuccess && n >= 1;
+        cudaGetLastError();
+    }
+    if (dev >= 0) cache[dev].store(ok ? 2 : 1);
+    return ok;
 }
 
 }  // namespace proj
@@ -358,6 +571,28 @@ extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int
     a.ld_qkv = ld_qkv;
     a.v16 = reinterpret_cast<__half*>(v16);
     a.status = status_word(workspace);
+    if (proj::pair_kernel_available()) {
+        // 256 x 256 tiles over CTA pairs; W's box is half a tile (128 rows)
+        CUtensorMap mw2;
+        const uint32_t wb2[2] = {proj::kBK, proj::kBN / 2};
+        if (!make_tmap_bf16(&mw2, W, 2, wd, wsd, wb2)) return TG_ERR_CUDA;
+        a.num_tiles = ((K + 2 * proj::kBM - 1) / (2 * proj::kBM)) * a.num_col_tiles;
+        const int pairs = static_cast<int>(std::min<int64_t>(a.num_tiles, num_sms() / 2));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * pairs);
+        cfg.blockDim = dim3(proj::kThreads);
+        cfg.dynamicSmemBytes = proj::kPairSmem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, proj::project_rope_pair_kernel, mx, mw2, a) == cudaSuccess ? TG_OK
+                                                                                                  : TG_ERR_CUDA;
+    }
     auto kern = proj::project_rope_kernel;
     static std::atomic<int> smem_set[64];
     if (!set_max_dynamic_smem(kern, proj::kSmem, smem_set)) return TG_ERR_CUDA;

@@ -29,6 +29,7 @@ extern "C" const char* tg_status_string(tg_status s) {
         case TG_ERR_UNSUPPORTED: return "unsupported shape";
         case TG_ERR_CUDA: return "CUDA launch or runtime error";
         case TG_ERR_TIMEOUT: return "device wait timed out";
+        case TG_ERR_RANGE: return "a value of V beyond fp16's range (|v| > 65504)";
     }
     return "unknown status";
 }
@@ -64,5 +65,6 @@ extern "C" tg_status tg_device_status(const void* workspace, uint32_t* status_wo
     if (cudaMemcpyAsync(&w, workspace, sizeof(w), cudaMemcpyDeviceToHost, st) != cudaSuccess) return TG_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return TG_ERR_CUDA;
     if (status_word_out) *status_word_out = w;
-    return w ? TG_ERR_TIMEOUT : TG_OK;
+    if (w & TG_STATUS_TIMEOUT_BITS) return TG_ERR_TIMEOUT;
+    return (w & TG_STATUS_V_RANGE) ? TG_ERR_RANGE : TG_OK;
 }

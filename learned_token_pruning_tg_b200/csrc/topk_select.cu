@@ -6,7 +6,16 @@
 // output order are the specification's; NaN ranks below every number and
 // -0 equals +0.
 //
-// Design (one cooperative launch, G <= #SM blocks of 1024 threads):
+// Two launch shapes, one algorithm.  Spans of up to 16 x 1024 x 16 keys (the
+// 16k-128k workloads) run in ONE thread-block cluster of 16 CTAs (8 where the
+// device does not offer 16), one per SM: the CTAs' histograms are merged
+// through distributed shared memory (each CTA sums one slice of the bins over
+// the cluster, then every CTA reads the slice totals and the one slice that
+// holds the target), and the hardware cluster barrier replaces the global
+// memory barrier; nothing is written to global memory but the result, so this
+// shape needs no scratch and has no software wait.  Each thread holds a run of
+// consecutive keys, so the ordered compaction takes one block scan.
+// Longer spans use one cooperative launch, G <= #SM blocks of 1024 threads:
 //   * every score is mapped to an order-preserving 32-bit key and kept in
 //     registers for the whole kernel (block b owns a contiguous chunk of the
 //     span, thread t the elements t, t+1024, ... of it);
@@ -259,6 +268,217 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const Se
         for (int b = tid; b < 3 * 2048; b += kSelectThreads) (&a.sc->hist[0][0])[b] = 0u;
 }
 
+// ---------------------------------------------------------------- one-cluster shape
+// Cluster rank and size, barrier and distributed-shared-memory access.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+// All threads of every CTA of the cluster; shared-memory writes before it are
+// visible cluster-wide after it (release / acquire at cluster scope).
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared-memory address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_map(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+constexpr int kSelectClusterMax = 16;
+
+// Keys per thread: a run of `a.ept` consecutive span elements (tb, tb + 1, ...).
+// Per radix pass: each CTA's histogram of the keys that match the prefix found
+// so far; CTA c then sums bins [c sl, (c + 1) sl) over the cluster (sl = bins /
+// cluster size) and their total; warp 0 of every CTA walks the slice totals
+// from the top digit down to the slice that holds the target, then that
+// slice's bins to the target bin.  Every CTA computes the same result.
+template <int EPT>
+__global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(const SelectArgs a) {
+    __shared__ unsigned int s_hist[2048];
+    __shared__ unsigned int s_slice[2048 / 8];   // this CTA's merged slice (at most 2048 / 8 bins)
+    __shared__ unsigned int s_tot;               // its total
+    __shared__ unsigned int s_cnt[2];            // this CTA's keys above / equal to the threshold
+    __shared__ unsigned int s_warp[32];
+    __shared__ unsigned int s_pick[2];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t rank = cluster_ctarank(), ncta = cluster_nctarank();
+    const int64_t chunk = static_cast<int64_t>(a.ept) * kSelectThreads;
+    const int64_t base = a.D0 + static_cast<int64_t>(rank) * chunk;
+    const int64_t end = min(base + chunk, a.D1);
+    const int64_t tb = base + static_cast<int64_t>(tid) * a.ept;
+
+    uint32_t key[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        const int64_t i = tb + j;
+        key[j] = (j < a.ept && i < end) ? (a.scores ? radix_key(__ldg(a.scores + i)) : random_key(a.seed, i)) : 0u;
+    }
+
+    uint32_t prefix = 0, pmask = 0;
+    unsigned int krem = a.kd;  // 1-based rank of the target among keys matching `prefix`
+#pragma unroll 1
+    for (int p = 0; p < 3; ++p) {
+        const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
+        const int nb = p == 2 ? 1024 : 2048;
+        const uint32_t dmask = static_cast<uint32_t>(nb - 1);
+        for (int b = tid; b < nb; b += kSelectThreads) s_hist[b] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            if (j < a.ept) {
+                const bool match = tb + j < end && (key[j] & pmask) == prefix;
+                const unsigned active = __ballot_sync(0xffffffffu, match);
+                if (match) {
+                    const uint32_t digit = (key[j] >> shift) & dmask;
+                    const unsigned peers = __match_any_sync(active, digit);
+                    if (lane == __ffs(peers) - 1) atomicAdd(&s_hist[digit], static_cast<unsigned>(__popc(peers)));
+                }
+            }
+        }
+        cluster_barrier();  // every CTA's histogram of this pass is complete
+
+        // this CTA's slice of the bins, summed over the cluster
+        const int sl = nb / static_cast<int>(ncta);
+        unsigned part = 0;
+        if (tid < sl) {
+            const int b = static_cast<int>(rank) * sl + tid;
+            for (uint32_t r = 0; r < ncta; ++r) part += dsmem_ld(dsmem_map(&s_hist[b], r));
+            s_slice[tid] = part;
+        }
+        if (warp < 8) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if (lane == 0) s_warp[warp] = part;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            unsigned t = 0;
+            for (int w = 0; w < 8; ++w) t += s_warp[w];
+            s_tot = t;
+        }
+        cluster_barrier();  // every slice and slice total is ready
+
+        if (warp == 0) {
+            // slices from the top digit down: lane l takes slice ncta - 1 - l
+            const uint32_t sli = ncta - 1 - static_cast<uint32_t>(lane);
+            const unsigned t = static_cast<uint32_t>(lane) < ncta ? dsmem_ld(dsmem_map(&s_tot, sli)) : 0u;
+            unsigned incl = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const unsigned hit = __ballot_sync(0xffffffffu, incl - t < krem && krem <= incl);
+            const int L = hit ? __ffs(hit) - 1 : 0;  // a lane always hits: krem <= the keys matching `prefix`
+            const uint32_t slice = ncta - 1 - static_cast<uint32_t>(L);
+            const unsigned before = __shfl_sync(0xffffffffu, incl - t, L);
+            // that slice's bins from the top down: lane l takes bins top - l per .. top - l per - per + 1
+            const int per = sl / 32;
+            const int top = sl - 1 - lane * per;  // index inside the slice
+            unsigned c[8];
+            unsigned lsum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                c[i] = i < per ? dsmem_ld(dsmem_map(&s_slice[top - i], slice)) : 0u;
+                lsum += c[i];
+            }
+            unsigned lincl = lsum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned y = __shfl_up_sync(0xffffffffu, lincl, o);
+                if (lane >= o) lincl += y;
+            }
+            const unsigned lex = before + lincl - lsum;
+            if (lane == 0) {
+                s_pick[0] = slice * static_cast<uint32_t>(sl);  // overwritten below by the lane that holds the target
+                s_pick[1] = before;
+            }
+            __syncwarp();
+            if (lex < krem && krem <= lex + lsum) {
+                unsigned acc = lex;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (i < per && acc < krem && krem <= acc + c[i]) {
+                        s_pick[0] = slice * static_cast<uint32_t>(sl) + static_cast<uint32_t>(top - i);
+                        s_pick[1] = acc;
+                    }
+                    acc += c[i];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= s_pick[0] << shift;
+        pmask |= dmask << shift;
+        krem -= s_pick[1];
+        __syncthreads();
+    }
+    const uint32_t T = prefix;
+
+    // counts of keys above T and equal to T: per thread, per CTA (< 2^16 each), per cluster prefix
+    unsigned cnt = 0;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j)
+        if (j < a.ept && tb + j < end) cnt += (key[j] > T ? 1u : 0u) + (key[j] == T ? 0x10000u : 0u);
+    unsigned btot;
+    const unsigned ex = block_excl_scan(cnt, s_warp, &btot);
+    if (tid == 0) {
+        s_cnt[0] = btot & 0xffffu;
+        s_cnt[1] = btot >> 16;
+    }
+    cluster_barrier();
+    if (warp == 0) {
+        unsigned g = 0, q = 0;
+        if (static_cast<uint32_t>(lane) < rank) {
+            g = dsmem_ld(dsmem_map(&s_cnt[0], lane));
+            q = dsmem_ld(dsmem_map(&s_cnt[1], lane));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            q += __shfl_xor_sync(0xffffffffu, q, o);
+        }
+        if (lane == 0) {
+            s_pick[0] = g;
+            s_pick[1] = q;
+        }
+    }
+    __syncthreads();
+    unsigned g_before = s_pick[0] + (ex & 0xffffu), e_before = s_pick[1] + (ex >> 16);
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        if (j < a.ept && tb + j < end) {
+            const int32_t i = static_cast<int32_t>(tb + j);
+            if (key[j] > T) {
+                a.out[a.D0 + g_before + min(e_before, krem)] = i;
+                ++g_before;
+            } else if (key[j] == T) {
+                if (e_before < krem) a.out[a.D0 + g_before + e_before] = i;
+                ++e_before;
+            }
+        }
+    }
+    // Tokens outside the span are always kept: [0, D0) first, [D1, N) after the kept document tokens.
+    const int64_t gstride = static_cast<int64_t>(ncta) * kSelectThreads;
+    for (int64_t i = static_cast<int64_t>(rank) * kSelectThreads + tid; i < a.D0; i += gstride)
+        a.out[i] = static_cast<int32_t>(i);
+    for (int64_t i = a.D1 + static_cast<int64_t>(rank) * kSelectThreads + tid; i < a.N; i += gstride)
+        a.out[a.D0 + a.kd + (i - a.D1)] = static_cast<int32_t>(i);
+    cluster_barrier();  // this CTA's shared memory stays alive until every CTA has read it
+}
+
 // K_doc == 0 (only tokens outside the span) or K_doc >= N_doc (every token).
 __global__ void select_trivial_kernel(int64_t N, int64_t D0, int64_t D1, int keep_doc, int32_t* out) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -277,6 +497,83 @@ static cudaError_t launch_select(const SelectArgs& a, int grid, cudaStream_t st)
     void* args[] = {const_cast<SelectArgs*>(&a)};
     return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(topk_select_kernel<EPT>), dim3(grid),
                                        dim3(kSelectThreads), args, 0, st);
+}
+
+// Largest cluster (16, else 8, else 0 = none) this device runs the cluster
+// kernel with, queried once per device.
+static int select_cluster_size() {
+    static std::atomic<int> cache[64];
+    const int dev = current_device();
+    if (dev >= 0 && cache[dev].load() != 0) return cache[dev].load() - 1;
+    int best = 0;
+    auto kern = topk_select_cluster_kernel<16>;
+    const bool nonportable =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    for (int cl : {16, 8}) {
+        if (cl > 8 && !nonportable) continue;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cl);
+        cfg.blockDim = dim3(kSelectThreads);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cl;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1) {
+            best = cl;
+            break;
+        }
+        cudaGetLastError();
+    }
+    if (dev >= 0) cache[dev].store(best + 1);
+    return best;
+}
+
+template <int EPT>
+static cudaError_t launch_select_cluster(const SelectArgs& a, int cl, cudaStream_t st) {
+    auto kern = topk_select_cluster_kernel<EPT>;
+    if (cl > 8) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cl);
+    cfg.blockDim = dim3(kSelectThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// The one-cluster shape when the span fits it (keys per thread <= 16);
+// returns false when the span is too long or the device offers no cluster.
+static bool try_select_cluster(SelectArgs a, int64_t n_doc, cudaStream_t st, cudaError_t* err) {
+    const int cl = select_cluster_size();
+    if (cl == 0) return false;
+    const int64_t per_cta = static_cast<int64_t>(cl) * kSelectThreads;
+    const int64_t ept = (n_doc + per_cta - 1) / per_cta;
+    if (ept > kSelectMaxEpt) return false;
+    a.ept = static_cast<int>(ept < 1 ? 1 : ept);
+    if (a.ept <= 1)
+        *err = launch_select_cluster<1>(a, cl, st);
+    else if (a.ept <= 2)
+        *err = launch_select_cluster<2>(a, cl, st);
+    else if (a.ept <= 4)
+        *err = launch_select_cluster<4>(a, cl, st);
+    else if (a.ept <= 8)
+        *err = launch_select_cluster<8>(a, cl, st);
+    else
+        *err = launch_select_cluster<16>(a, cl, st);
+    return true;
 }
 
 }  // namespace tg
@@ -303,14 +600,6 @@ static tg_status select_impl(const float* scores, uint64_t seed, int64_t N, int6
     }
     if (!workspace || workspace_bytes < tg_workspace_bytes(TG_OP_SELECT, N, 0, 0)) return TG_ERR_INVALID_ARG;
     if (!aligned16(workspace)) return TG_ERR_INVALID_ARG;
-    const int sms = num_sms();
-    const int64_t per_block_min = kSelectThreads;
-    int64_t ept = (n_doc + static_cast<int64_t>(sms) * per_block_min - 1) / (static_cast<int64_t>(sms) * per_block_min);
-    if (ept < 1) ept = 1;
-    if (ept > kSelectMaxEpt) return TG_ERR_UNSUPPORTED;
-    const int64_t chunk = ept * kSelectThreads;
-    const int grid = static_cast<int>((n_doc + chunk - 1) / chunk);
-    if (grid > kSelectMaxBlocks) return TG_ERR_UNSUPPORTED;
 
     SelectArgs a;
     a.scores = scores;
@@ -322,8 +611,18 @@ static tg_status select_impl(const float* scores, uint64_t seed, int64_t N, int6
     a.out = kept_idx;
     a.sc = reinterpret_cast<SelectScratch*>(static_cast<char*>(workspace) + kWsHeader);
     a.status = status_word(workspace);
-    a.ept = static_cast<int>(ept);
     cudaError_t e;
+    if (try_select_cluster(a, n_doc, st, &e)) return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;
+
+    const int sms = num_sms();
+    const int64_t per_block_min = kSelectThreads;
+    int64_t ept = (n_doc + static_cast<int64_t>(sms) * per_block_min - 1) / (static_cast<int64_t>(sms) * per_block_min);
+    if (ept < 1) ept = 1;
+    if (ept > kSelectMaxEpt) return TG_ERR_UNSUPPORTED;
+    const int64_t chunk = ept * kSelectThreads;
+    const int grid = static_cast<int>((n_doc + chunk - 1) / chunk);
+    if (grid > kSelectMaxBlocks) return TG_ERR_UNSUPPORTED;
+    a.ept = static_cast<int>(ept);
     if (ept <= 1)
         e = launch_select<1>(a, grid, st);
     else if (ept <= 2)

@@ -8,12 +8,15 @@ article, paragraph 事件详情; chathome.org article, sections TokenGate の学
 トークンプルーニングの仕組み and トークンゲート付きアテンションとは).
 
 Steps, in order, all on the caller's current CUDA stream:
-  gate     tg_gate_score        libtokengate (tcgen05 GEMM + fused epilogue)
-  select   tg_topk_select       libtokengate (radix select)
-  gather   tg_gather_compact    libtokengate (row copy)
-  qkv      h' Wqkv^T            torch.matmul (cuBLAS): projection glue
-  rope     tg_rope_apply        libtokengate
-  attn     tg_gated_attention   libtokengate (tcgen05 flash attention)
+  gate     tg_gate_score            libtokengate (tcgen05 GEMM + fused epilogue)
+  select   tg_topk_select           libtokengate (radix select)
+  gather   tg_gather_compact        libtokengate (row copy)
+  proj     tg_project_rope          libtokengate (tcgen05 GEMM of the kept rows with
+                                    RoPE and V's fp16 copy in its epilogue)
+  attn     tg_gated_attention_f16v  libtokengate (tcgen05 flash attention)
+With fused_projection=False the projection is instead a library GEMM
+(torch.matmul, cuBLAS) followed by tg_rope_apply, and the attention converts V
+itself (tg_gated_attention); stages "qkv", "rope", "attn".
 torch allocates every buffer once (plumbing); the kept count K is known on the
 host, so nothing synchronizes inside a step.
 """
@@ -25,7 +28,9 @@ import torch
 
 from . import tokengate as tg
 
-STAGES = ("gate", "select", "gather", "qkv", "rope", "attn")
+STAGES_FUSED = ("gate", "select", "gather", "proj", "attn")
+STAGES_UNFUSED = ("gate", "select", "gather", "qkv", "rope", "attn")
+STAGES = STAGES_FUSED
 
 
 def nvtx_marks() -> Callable[[str], None]:
@@ -47,7 +52,7 @@ class GatedPrefillLayer:
     def __init__(self, N: int, doc_begin: int, doc_end: int, k_doc: int, W1: torch.Tensor, w2: torch.Tensor,
                  Wqkv: torch.Tensor, Hq: int, Hkv: int, d_h: int, gain: torch.Tensor, tau: float,
                  b1: Optional[torch.Tensor] = None, b2: float = 0.0, rms_weight: Optional[torch.Tensor] = None,
-                 eps: float = 1e-6, rope_base: float = 1e6, device="cuda"):
+                 eps: float = 1e-6, rope_base: float = 1e6, device="cuda", fused_projection: bool = True):
         self.N, self.doc_begin, self.doc_end, self.k_doc = N, doc_begin, doc_end, k_doc
         self.K = tg.tg_kept_count(N, doc_begin, doc_end, k_doc)
         if self.K < 0:
@@ -61,11 +66,21 @@ class GatedPrefillLayer:
         self.b2 = float(b2)
         self.rms_weight = None if rms_weight is None else rms_weight.to(dev, torch.bfloat16).contiguous()
         self.eps, self.rope_base, self.tau = eps, rope_base, float(tau)
-        self.WqkvT = Wqkv.to(dev, torch.bfloat16).t().contiguous()      # [d, (Hq + 2 Hkv) d_h]
+        self.fused = fused_projection
+        self.stages = STAGES_FUSED if fused_projection else STAGES_UNFUSED
+        self.Wqkv = Wqkv.to(dev, torch.bfloat16).contiguous()             # [(Hq + 2 Hkv) d_h, d]
+        self.WqkvT = None if fused_projection else self.Wqkv.t().contiguous()
         self.gain = gain.to(dev, torch.float32).contiguous()
         K, d = self.K, self.d
         self.ws = tg.new_workspace(N, d, self.d_g, op=tg.TG_OP_GATE, device=dev)  # gate and select
-        self.ws_attn = tg.new_workspace(K, Hkv * d_h, op=tg.TG_OP_ATTENTION, device=dev)
+        if fused_projection:
+            self.ws_proj = tg.new_workspace(K, d_h, op=tg.TG_OP_PROJECT, device=dev)
+            self.ws_attn = tg.new_workspace(0, Hkv * d_h, op=tg.TG_OP_ATTENTION, device=dev)
+            self.v16 = torch.empty(K, Hkv * d_h, dtype=torch.float16, device=dev)
+        else:
+            self.ws_proj = None
+            self.ws_attn = tg.new_workspace(K, Hkv * d_h, op=tg.TG_OP_ATTENTION, device=dev)
+            self.v16 = None
         self.scores = torch.empty(N, dtype=torch.float32, device=dev)
         self.kept = torch.empty(max(K, 1), dtype=torch.int32, device=dev)
         self.h_kept = torch.empty(K, d, dtype=torch.bfloat16, device=dev)
@@ -78,8 +93,8 @@ class GatedPrefillLayer:
         self.out = torch.empty(K, Hq, d_h, dtype=torch.bfloat16, device=dev)
 
     def run(self, h: torch.Tensor, mark: Optional[Callable[[str], None]] = None):
-        """Runs the six steps on device-resident h [N, d]; returns (out [K, Hq, d_h], kept [K]).
-        `mark(name)` is called before each step and with "end" after the last (event hooks)."""
+        """Runs the steps on device-resident h [N, d]; returns (out [K, Hq, d_h], kept [K]).
+        `mark(name)` is called before each step (self.stages) and with "end" after the last."""
         m = mark or (lambda _n: None)
         K = self.K
         m("gate")
@@ -90,13 +105,21 @@ class GatedPrefillLayer:
         m("gather")
         tg.tg_gather_compact(h, self.kept[:K], self.h_kept, self.pos[:K], scores=self.scores,
                              s_out=self.s_kept[:K])
-        m("qkv")
-        torch.matmul(self.h_kept, self.WqkvT, out=self.qkv)
-        m("rope")
-        tg.tg_rope_apply(self.q, self.k, self.pos[:K], self.rope_base)
-        m("attn")
-        tg.tg_gated_attention(self.q, self.k, self.v, self.out, self.ws_attn, s_kept=self.s_kept[:K],
-                              gain=self.gain, tau=self.tau)
+        if self.fused:
+            m("proj")
+            tg.tg_project_rope(self.h_kept, self.Wqkv, self.pos[:K], self.qkv, self.ws_proj, self.Hq, self.Hkv,
+                               self.d_h, base=self.rope_base, v16=self.v16)
+            m("attn")
+            tg.tg_gated_attention_f16v(self.q, self.k, self.v16, self.out, self.ws_attn, s_kept=self.s_kept[:K],
+                                       gain=self.gain, tau=self.tau)
+        else:
+            m("qkv")
+            torch.matmul(self.h_kept, self.WqkvT, out=self.qkv)
+            m("rope")
+            tg.tg_rope_apply(self.q, self.k, self.pos[:K], self.rope_base)
+            m("attn")
+            tg.tg_gated_attention(self.q, self.k, self.v, self.out, self.ws_attn, s_kept=self.s_kept[:K],
+                                  gain=self.gain, tau=self.tau)
         m("end")
         return self.out, self.kept[:K]
 
@@ -111,10 +134,13 @@ class GatedPrefillLayer:
         return out_host, kept_host
 
     def launches_per_step(self) -> int:
-        """libtokengate kernels per run(): gate (+ the RMSNorm-weight fold), select, gather, rope, and the
-        attention's two (V to fp16, attention)."""
+        """libtokengate kernels per run(): gate (+ the RMSNorm-weight fold), select, gather, then either the
+        projection's two (cos / sin table, GEMM) and the attention, or RoPE and the attention's two (V to
+        fp16, attention) after the library GEMM."""
         return 6 + (1 if self.rms_weight is not None else 0)
 
     def device_status(self) -> int:
-        """OR of the status words of the layer's workspaces (synchronizes the stream); 0 = no timeout."""
-        return tg.tg_device_status(self.ws) | tg.tg_device_status(self.ws_attn)
+        """OR of the status words of the layer's workspaces (synchronizes the stream); 0 = no timeout
+        and no value out of range."""
+        st = tg.tg_device_status(self.ws) | tg.tg_device_status(self.ws_attn)
+        return st | (tg.tg_device_status(self.ws_proj) if self.ws_proj is not None else 0)

@@ -16,8 +16,10 @@ rotate-half RoPE at the original positions, SwiGLU MLP, residual adds.
                   per token, so this equals running it on N and gathering)
   layers L+1..    over the K kept rows, token-gated attention
 Attention (dense layers: K = N, no bias, tau = 1, i.e. plain causal attention),
-the gate, the select, the gather and RoPE run in libtokengate; RMSNorm, the
-projections, SwiGLU and the residual adds are torch (cuBLAS) glue.  The same
+the Q/K/V projection with RoPE (tg_project_rope, which also writes V's fp16
+copy for the attention), the gate, the select and the gather run in
+libtokengate; RMSNorm, the output and MLP projections, SwiGLU and the residual
+adds are torch (cuBLAS) glue.  The same
 object runs the unpruned stack (every layer dense over N) for comparison.
 Weights are random (seeded, drawn on the device): there are no trained weights.
 """
@@ -127,7 +129,9 @@ class PrunedPrefillStack:
         self.cfg, self.wts = cfg, weights
         self.dev = torch.device(device)
         self.ws_gate = tg.new_workspace(cfg.N, cfg.d, cfg.d_g, op=tg.TG_OP_GATE, device=self.dev)
-        self.ws_attn = tg.new_workspace(cfg.N, cfg.Hkv * cfg.d_h, op=tg.TG_OP_ATTENTION, device=self.dev)
+        self.ws_attn = tg.new_workspace(0, cfg.Hkv * cfg.d_h, op=tg.TG_OP_ATTENTION, device=self.dev)
+        self.ws_proj = tg.new_workspace(cfg.N, cfg.d_h, op=tg.TG_OP_PROJECT, device=self.dev)
+        self.v16 = torch.empty(cfg.N, cfg.Hkv * cfg.d_h, dtype=torch.float16, device=self.dev)
         self.captured: Dict[str, torch.Tensor] = {}
         self.kept: Optional[torch.Tensor] = None
         self.scores: Optional[torch.Tensor] = None
@@ -139,18 +143,20 @@ class PrunedPrefillStack:
                    keep_kv: bool):
         c, lw = self.cfg, self.wts.layers[li]
         n = x.shape[0]
-        qkv = torch.matmul(rms_norm(x, lw.ln1, c.eps), lw.Wqkv.t())
+        qkv = torch.empty(n, (c.Hq + 2 * c.Hkv) * c.d_h, dtype=torch.bfloat16, device=self.dev)
+        v16 = self.v16[:n]
+        tg.tg_project_rope(rms_norm(x, lw.ln1, c.eps), lw.Wqkv, pos, qkv, self.ws_proj, c.Hq, c.Hkv, c.d_h,
+                           base=c.rope_base, v16=v16)
         q = qkv[:, : c.Hq * c.d_h].view(n, c.Hq, c.d_h)
         k = qkv[:, c.Hq * c.d_h: (c.Hq + c.Hkv) * c.d_h].view(n, c.Hkv, c.d_h)
         v = qkv[:, (c.Hq + c.Hkv) * c.d_h:].view(n, c.Hkv, c.d_h)
-        tg.tg_rope_apply(q, k, pos, c.rope_base)
         if keep_kv:
             self.kv.append((k.clone(), v.clone(), s_kept if gated else None))
         out = torch.empty(n, c.Hq, c.d_h, dtype=torch.bfloat16, device=self.dev)
         if gated:
-            tg.tg_gated_attention(q, k, v, out, self.ws_attn, s_kept=s_kept, gain=lw.gain, tau=lw.tau)
+            tg.tg_gated_attention_f16v(q, k, v16, out, self.ws_attn, s_kept=s_kept, gain=lw.gain, tau=lw.tau)
         else:
-            tg.tg_gated_attention(q, k, v, out, self.ws_attn, tau=1.0)
+            tg.tg_gated_attention_f16v(q, k, v16, out, self.ws_attn, tau=1.0)
         if capture:
             self.captured = {"q": q.clone(), "k": k.clone(), "v": v.clone(), "out": out.clone(),
                              "s": None if s_kept is None else s_kept.clone(), "gain": lw.gain.clone(),
@@ -194,4 +200,5 @@ class PrunedPrefillStack:
                    (0 if sc is None else sc.numel() * 4) for k, v, sc in self.kv)
 
     def device_status(self) -> int:
-        return tg.tg_device_status(self.ws_gate) | tg.tg_device_status(self.ws_attn)
+        return (tg.tg_device_status(self.ws_gate) | tg.tg_device_status(self.ws_attn) |
+                tg.tg_device_status(self.ws_proj))

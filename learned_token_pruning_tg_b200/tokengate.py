@@ -17,10 +17,10 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtokengate.so")
 
-TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_CUDA, TG_ERR_TIMEOUT = range(5)
+TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_CUDA, TG_ERR_TIMEOUT, TG_ERR_RANGE = range(6)
 TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL, TG_OP_DECODE, TG_OP_ATTENTION_BACKWARD, TG_OP_PROJECT = range(7)
 TG_STATUS_SELECT_TIMEOUT, TG_STATUS_GATE_TIMEOUT, TG_STATUS_ATTENTION_TIMEOUT, TG_STATUS_DECODE_TIMEOUT = 1, 2, 4, 8
-TG_STATUS_BACKWARD_TIMEOUT, TG_STATUS_PROJECT_TIMEOUT = 16, 32
+TG_STATUS_BACKWARD_TIMEOUT, TG_STATUS_PROJECT_TIMEOUT, TG_STATUS_V_RANGE = 16, 32, 64
 
 _lib = None
 
@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.tg_rope_apply.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, f64, vp]
         L.tg_gated_attention.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp,
                                          vp, sz, vp]
+        L.tg_gated_attention_f16v.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, vp, vp, f32, vp, vp, vp, sz,
+                                              vp]
         L.tg_gated_decode.argtypes = [vp, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp, vp, sz, vp]
         L.tg_project_rope.argtypes = [vp, i64, i32, i64, vp, i32, i32, i32, vp, f64, vp, i64, vp, vp, sz, vp]
         L.tg_gated_attention_backward.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp,
@@ -63,7 +65,8 @@ def lib() -> ctypes.CDLL:
         L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
         for fn in ("tg_gate_score", "tg_topk_select", "tg_topk_select_noalloc", "tg_random_select", "tg_gather_compact",
                    "tg_rope_apply",
-                   "tg_gated_attention", "tg_gated_decode", "tg_debug_set_select_wait_limit", "tg_device_status"):
+                   "tg_gated_attention", "tg_gated_attention_f16v", "tg_project_rope",
+                   "tg_gated_attention_backward", "tg_gated_decode", "tg_debug_set_select_wait_limit", "tg_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -246,6 +249,29 @@ def tg_gated_attention(q, k, v, out, workspace, s_kept=None, gain=None, tau: flo
     return out
 
 
+def tg_gated_attention_f16v(q, k, v16, out, workspace, s_kept=None, gain=None, tau: float = 1.0, lse=None,
+                            stream=None):
+    """tg_gated_attention over an fp16 copy of V (v16 [K, Hkv, d_h] or [K, Hkv d_h] fp16, dense), as
+    tg_project_rope writes it."""
+    _req(q, "q", torch.bfloat16, 3)
+    _req(k, "k", torch.bfloat16, 3)
+    _req(v16, "v16", torch.float16)
+    _req(out, "out", torch.bfloat16, 3)
+    _req(s_kept, "s_kept", torch.float32, 1)
+    _req(gain, "gain", torch.float32, 1)
+    _req(lse, "lse", torch.float32, 2)
+    K, Hq, d_h = q.shape
+    Hkv = k.shape[1]
+    if not out.is_contiguous() or out.shape != (K, Hq, d_h):
+        raise ValueError("out must be a contiguous [K, Hq, d_h] tensor")
+    if not v16.is_contiguous() or v16.numel() != K * Hkv * d_h or v16.shape[0] != K:
+        raise ValueError("v16 must be a contiguous [K, Hkv, d_h] fp16 tensor")
+    _check("tg_gated_attention_f16v", lib().tg_gated_attention_f16v(
+        _ptr(q), _row_stride(q, "q"), _ptr(k), _row_stride(k, "k"), _ptr(v16), K, Hq, Hkv, d_h, _ptr(s_kept),
+        _ptr(gain), tau, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
 def tg_gated_attention_backward(q, k, v, out, dout, lse, dq, dk, dv, workspace, s_kept=None, gain=None,
                                 tau: float = 1.0, ds=None, dg=None, dtau=None, stream=None):
     """Gradients of tg_gated_attention: out, dout [K, Hq, d_h] and lse [Hq, K] from the forward call;
@@ -325,9 +351,9 @@ def tg_debug_set_select_wait_limit(ns: int) -> None:
 
 
 def tg_device_status(workspace, stream=None) -> int:
-    """Raw status bits of the workspace (synchronizes the stream); raises on timeout bits."""
+    """Raw TG_STATUS_* bits of the workspace (synchronizes the stream); raises only if the read fails."""
     w = ctypes.c_uint32(0)
     st = lib().tg_device_status(_ptr(workspace), ctypes.byref(w), _stream(stream))
-    if st not in (TG_OK, TG_ERR_TIMEOUT):
+    if st not in (TG_OK, TG_ERR_TIMEOUT, TG_ERR_RANGE):
         raise TokenGateError("tg_device_status", st)
     return int(w.value)

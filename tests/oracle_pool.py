@@ -4,6 +4,7 @@ The pool uses the spawn start method, so it is safe to create after CUDA has
 been initialised in the parent.  Each worker runs the unmodified oracle on its
 chunk; results are concatenated in row order.
 """
+import atexit
 import concurrent.futures as cf
 import multiprocessing as mp
 import os
@@ -18,6 +19,7 @@ def pool():
     if _pool is None:
         n = max(1, min(16, (os.cpu_count() or 2) - 1))
         _pool = cf.ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn"))
+        atexit.register(_pool.shutdown, wait=True)
     return _pool
 
 
@@ -70,3 +72,16 @@ def gated_attention_backward(q, k, v, dout, s=None, g=None, tau=1.0):
             "ds": np.sum([p["ds"] for p in parts], axis=0),
             "dg": np.concatenate([p["dg"] for p in parts]),
             "dtau": float(np.sum([p["dtau"] for p in parts]))}
+
+
+def _project_chunk(x, W):
+    import oracle
+    return oracle.project(x, W)
+
+
+def project(x, W, chunk=None):
+    """Oracle projection x W^T (fp64) of every row of x, row chunks split across workers."""
+    n_workers = pool()._max_workers
+    chunk = chunk or max(64, -(-x.shape[0] // (2 * n_workers)))
+    futs = [pool().submit(_project_chunk, x[lo:lo + chunk], W) for lo in range(0, x.shape[0], chunk)]
+    return np.concatenate([f.result() for f in futs]) if futs else np.empty((0, W.shape[0]))

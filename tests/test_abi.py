@@ -63,6 +63,7 @@ def test_host_only_calls(lib):
     assert tg.tg_workspace_bytes(tg.TG_OP_ALL, 4608, 1024, 256) >= tg.tg_workspace_bytes(tg.TG_OP_GATE, 4608, 1024, 256)
     assert tg.status_string(tg.TG_OK) == "ok"
     assert "timed out" in tg.status_string(tg.TG_ERR_TIMEOUT)
+    assert "fp16" in tg.status_string(tg.TG_ERR_RANGE)
     assert tg.tg_version() >= 100
 
 
@@ -92,6 +93,23 @@ def test_argument_errors_before_launch(lib):
                                       vp(16), None, vp(256), 1 << 20, None) == tg.TG_ERR_INVALID_ARG
     assert lib.tg_gated_attention(vp(16), 128, vp(16), 128, vp(16), 128, 5, 2, 2, 64, None, None, 1.0,
                                   vp(16), None, vp(256), 256, None) == tg.TG_ERR_INVALID_ARG  # workspace too small
+    # the fp16-V variant: same checks, and a workspace of the status header only is enough
+    f16v = lib.tg_gated_attention_f16v
+    assert f16v(vp(16), 128, vp(16), 128, vp(16), 5, 3, 2, 64, None, None, 1.0, vp(16), None, vp(256), 1 << 20,
+                None) == tg.TG_ERR_INVALID_ARG    # Hq % Hkv
+    assert f16v(vp(16), 96, vp(16), 96, vp(16), 5, 1, 1, 96, None, None, 1.0, vp(16), None, vp(256), 1 << 20,
+                None) == tg.TG_ERR_UNSUPPORTED    # d_h = 96
+    assert f16v(vp(16), 128, vp(16), 128, vp(24), 5, 2, 2, 64, None, None, 1.0, vp(16), None, vp(256), 1 << 20,
+                None) == tg.TG_ERR_INVALID_ARG    # v16 misaligned
+    assert f16v(vp(16), 128, vp(16), 128, None, 5, 2, 2, 64, None, None, 1.0, vp(16), None, vp(256), 1 << 20,
+                None) == tg.TG_ERR_INVALID_ARG    # no v16
+    assert f16v(vp(16), 128, vp(16), 128, vp(16), 5, 2, 2, 64, None, None, -1.0, vp(16), None, vp(256), 1 << 20,
+                None) == tg.TG_ERR_INVALID_ARG    # tau <= 0
+    assert f16v(vp(16), 128, vp(16), 128, vp(16), 5, 2, 2, 64, None, None, 1.0, vp(16), None, vp(256), 16,
+                None) == tg.TG_ERR_INVALID_ARG    # workspace too small
+    assert f16v(vp(16), 128, vp(16), 128, vp(16), 0, 2, 2, 64, None, None, 1.0, vp(16), None, vp(256), 16,
+                None) == tg.TG_OK                 # K = 0: nothing to do
+    assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, 0, 1024) < tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, 4608, 1024)
 
 
 def test_decode_and_random_select_argument_errors(lib):

@@ -32,7 +32,7 @@ def install_fakes(monkeypatch, calls):
     monkeypatch.setattr(tg, "tg_gated_attention_backward", bwd)
 
 
-def inputs(K=5, Hq=4, Hkv=2, d_h=8):
+def inputs(K=5, Hq=4, Hkv=2, d_h=64):
     g = torch.Generator().manual_seed(0)
     q = torch.randn(K, Hq, d_h, generator=g).to(torch.bfloat16).requires_grad_()
     k = torch.randn(K, Hkv, d_h, generator=g).to(torch.bfloat16).requires_grad_()
@@ -72,3 +72,43 @@ def test_gradients_only_when_asked(monkeypatch):
     out.float().sum().backward()
     assert calls["fwd"]["s"] is None and calls["fwd"]["g"] is None
     assert torch.all(q2.grad == 1.0)
+
+
+def test_tau_gradient_takes_tau_shape_and_device(monkeypatch):
+    calls = {}
+    install_fakes(monkeypatch, calls)
+    q, k, v, s, gain = inputs()
+    tau = torch.tensor([1.1], requires_grad=True)            # one element, shape [1]
+    ag.gated_attention(q, k, v, s, gain, tau).float().sum().backward()
+    assert tau.grad.shape == (1,) and tau.grad.item() == 6.0
+
+
+def test_backward_limits_fail_in_the_forward(monkeypatch):
+    import pytest
+    calls = {}
+    install_fakes(monkeypatch, calls)
+    g = torch.Generator().manual_seed(1)
+    q = torch.randn(5, 16, 64, generator=g).to(torch.bfloat16).requires_grad_()
+    k = torch.randn(5, 1, 64, generator=g).to(torch.bfloat16).requires_grad_()   # Hq / Hkv = 16 > 8
+    with pytest.raises(ValueError, match="Hq / Hkv"):
+        ag.gated_attention(q, k, k.detach().clone())
+    q96 = torch.randn(5, 4, 96, generator=g).to(torch.bfloat16).requires_grad_()
+    k96 = torch.randn(5, 2, 96, generator=g).to(torch.bfloat16)
+    with pytest.raises(ValueError, match="d_h"):
+        ag.gated_attention(q96, k96, k96)
+    # without a graph to build, the forward alone has the forward's own limits
+    out = ag.gated_attention(q.detach(), k.detach(), k.detach())
+    assert "fwd" in calls and out.shape == q.shape
+
+
+def test_status_check_raises_on_a_set_bit(monkeypatch):
+    import pytest
+    calls = {}
+    install_fakes(monkeypatch, calls)
+    monkeypatch.setattr(tg, "tg_device_status", lambda ws, stream=None: tg.TG_STATUS_ATTENTION_TIMEOUT)
+    q, k, v, s, gain = inputs()
+    with pytest.raises(tg.TokenGateError):
+        ag.gated_attention(q, k, v, s, gain, 1.0, check_status=True)
+    monkeypatch.setattr(tg, "tg_device_status", lambda ws, stream=None: 0)
+    ag.gated_attention(q, k, v, s, gain, 1.0, check_status=True).float().sum().backward()
+    assert torch.all(q.grad == 1.0)

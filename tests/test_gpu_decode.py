@@ -60,9 +60,12 @@ def check(d, strided=False, use_bias=True):
     want, want_lse = oracle.gated_attention(q, k, v, s=s, g=g, tau=d.tau, rows=[T - 1], want_lse=True)
     want, want_lse = want[0], want_lse[0]
     assert np.all(np.isfinite(got))
-    excess = np.abs(got - want) - half_ulp_bf16(want)
+    # raw error where |out| < 2 (its bf16 rounding is at most 2^-8 there), else above its half ulp
+    err = np.abs(got - want)
+    excess = np.where(np.abs(want) < 2.0, err, err - half_ulp_bf16(want))
     assert np.max(excess) <= SPEC_TOL
-    assert np.max(excess) <= DERIVED_TOL, np.max(excess)
+    # the derived bar bounds the kernel's own arithmetic: the error beyond the output's rounding
+    assert np.max(err - half_ulp_bf16(want)) <= DERIVED_TOL, np.max(err - half_ulp_bf16(want))
     assert np.max(np.abs(lse - want_lse)) <= LSE_TOL
 
 

@@ -1,6 +1,8 @@
 """Failure detection without a GPU fault.
 
-The select's grid barrier is a bounded spin.  With its time limit shrunk to a
+The select's grid barrier (the cooperative launch shape, used for spans longer than one
+thread-block cluster holds; shorter spans use hardware cluster barriers, which need no limit) is a
+bounded spin.  With its time limit shrunk to a
 nanosecond (tg_debug_set_select_wait_limit, a test hook) the blocks of a call
 stop waiting for one another: the call must end by itself, report
 TG_STATUS_SELECT_TIMEOUT in the workspace's status word (tg_device_status), and
@@ -19,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 
 def test_select_barrier_timeout_is_reported_and_the_context_recovers():
-    N, db, de, k = 131072, 0, 130560, 4096
+    N, db, de, k = 600000, 0, 599000, 4096   # beyond the one-cluster shape: the cooperative one
     s = synth.score_vector(N, seed=11, kind="normal").cuda()
     K = tg.tg_kept_count(N, db, de, k)
     out = torch.full((K,), -1, dtype=torch.int32, device="cuda")

@@ -68,6 +68,12 @@ def test_gate_full_workloads(w):
     (4099, 2048, 256, False, True),   # many tiles, tail of 3 rows
     (20000, 1024, 64, True, False),   # more tiles than SMs, narrow gate
     (300, 8192, 128, False, False),   # long K loop
+    # d_g = 256 runs on CTA pairs (256-row tiles shared by two CTAs): a pair with one row, a pair
+    # whose second CTA has no rows, a tail of one row past a pair, a long K loop
+    (1, 64, 256, False, False),
+    (129, 128, 256, True, False),
+    (257, 256, 256, False, False),
+    (300, 8192, 256, True, True),
 ])
 def test_gate_shapes(N, d, d_g, bias, gamma):
     w = synth.scaled(synth.L16K, N=N, doc_end=N, d=d, d_g=d_g, n_scaled=min(8, N), seed=N + d)

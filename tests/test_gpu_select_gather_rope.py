@@ -42,6 +42,8 @@ SELECT_CASES = [
     (300000, 1000, 299000, 100000, "ties", 7),      # two keys per thread
     (2000000, 0, 1999000, 65536, "heavy", 8),       # many keys per thread
     (3, 0, 2, 1, "normal", 9),
+    (262656, 0, 262144, 30000, "heavy", 10),      # the one-cluster shape's longest span (16 keys per thread)
+    (262657, 0, 262145, 30000, "normal", 12),     # one key more: the cooperative shape
 ]
 
 
@@ -69,7 +71,11 @@ def test_select_empty_span_and_repeat_calls():
 
 
 @pytest.mark.parametrize("N,d,K,ld_pad", [(1024, 256, 256, 0), (16384, 2048, 1408, 0), (5000, 2048, 777, 64),
-                                          (300, 136, 299, 8), (4096, 4096, 100, 0)])
+                                          (300, 136, 299, 8), (4096, 4096, 100, 0),
+                                          (131072, 2048, 4608, 0),   # the 128k workload's kept set (bulk copies)
+                                          (100, 2048, 33, 0),        # one row past a 32-row block
+                                          (40, 16384, 9, 0),         # 32 KB rows: the 16-byte-vector copy
+                                          (10, 64, 1, 0)])
 def test_gather_bit_exact(N, d, K, ld_pad):
     g = torch.Generator().manual_seed(N + d)
     h_full = torch.randn(N, d + ld_pad, generator=g).to(torch.bfloat16)
@@ -92,6 +98,33 @@ def test_gather_bit_exact(N, d, K, ld_pad):
     tg.tg_gather_compact(hd, idx.cuda(), h_out, pos_out)
     torch.cuda.synchronize()
     assert np.array_equal(pos_out.cpu().numpy(), idx.numpy())
+
+
+@pytest.mark.parametrize("d", [2048, 16384])
+def test_gather_rejects_out_of_range_indices_without_reading(d):
+    # A kept index outside [0, N) is not read: its row comes out zero, its position -1 and its score
+    # NaN; every other row is copied exactly.  (The indices are only checked, never dereferenced, so
+    # nothing here reads outside h.)
+    N, K = 64, 12
+    g = torch.Generator().manual_seed(d)
+    h = torch.randn(N, d, generator=g).to(torch.bfloat16)
+    s = torch.randn(N, generator=g)
+    idx = torch.tensor([0, 3, N, 5, -1, 9, 2 ** 31 - 1, 20, 21, -(2 ** 31), 40, N - 1], dtype=torch.int32)
+    h_out, check_h = guarded((K, d), torch.bfloat16)
+    pos_out, check_p = guarded((K,), torch.int32)
+    s_out, check_s = guarded((K,), torch.float32)
+    h_out.fill_(7.0)
+    tg.tg_gather_compact(h.cuda(), idx.cuda(), h_out, pos_out, scores=s.cuda(), s_out=s_out)
+    torch.cuda.synchronize()
+    check_h(), check_p(), check_s()
+    bad = (idx < 0) | (idx >= N)
+    got_h, got_p, got_s = h_out.cpu(), pos_out.cpu(), s_out.cpu()
+    assert torch.equal(got_p[bad], torch.full((int(bad.sum()),), -1, dtype=torch.int32))
+    assert torch.all(torch.isnan(got_s[bad])) and torch.all(got_h[bad] == 0)
+    good = ~bad
+    assert torch.equal(got_p[good], idx[good])
+    assert torch.equal(got_h[good].view(torch.int16), h[idx[good].long()].view(torch.int16))
+    assert torch.equal(got_s[good], s[idx[good].long()])
 
 
 @pytest.mark.parametrize("K,Hq,Hkv,d_h,max_pos", [(256, 4, 2, 64, 1024), (1408, 16, 8, 128, 16384),
