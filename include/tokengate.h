@@ -173,11 +173,20 @@ tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_begin,
  * Limit: doc_end - doc_begin <= #SMs * 1024 * 16 (2,424,832 on a 148-SM B200,
  * the largest grid the select kernel uses); longer spans return
  * TG_ERR_UNSUPPORTED before anything is launched.
- * A device-side wait that times out leaves kept_idx undefined; this entry
- * point reports launch errors only. */
+ * A device-side wait that times out leaves kept_idx undefined and sets
+ * TG_STATUS_SELECT_TIMEOUT in the array's status word, which
+ * tg_topk_select_noalloc_status reads back; this entry point itself reports
+ * launch errors only. */
 tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int64_t doc_begin,
                                  int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
                                  void* stream);
+
+/* The status word the last tg_topk_select_noalloc call on the current device
+ * left in its static array (each call clears it first): synchronizes `stream`
+ * (the stream of that call), writes the raw TG_STATUS_* bits to *status_word
+ * (may be NULL) and returns TG_ERR_TIMEOUT if a timeout bit is set, TG_OK
+ * otherwise.  Allocates nothing. */
+tg_status tg_topk_select_noalloc_status(uint32_t* status_word, void* stream);
 
 /* Random-K selector (the pages' budget-matched random baseline): keeps
  * min(k_doc, doc_end - doc_begin) document tokens chosen at random, plus every

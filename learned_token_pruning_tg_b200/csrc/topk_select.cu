@@ -749,3 +749,14 @@ extern "C" tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int6
         e = launch_select<16>(a, grid, st);
     return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;
 }
+
+extern "C" tg_status tg_topk_select_noalloc_status(uint32_t* status_word_out, void* stream) {
+    unsigned char* scratch = nullptr;
+    if (noalloc::scratch_for_current_device(&scratch) != TG_OK) return TG_ERR_CUDA;
+    uint32_t w = 0;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemcpyAsync(&w, scratch, sizeof(w), cudaMemcpyDeviceToHost, st) != cudaSuccess) return TG_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return TG_ERR_CUDA;
+    if (status_word_out) *status_word_out = w;
+    return (w & TG_STATUS_TIMEOUT_BITS) ? TG_ERR_TIMEOUT : TG_OK;
+}

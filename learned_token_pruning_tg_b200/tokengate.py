@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         L.tg_gate_score.argtypes = [vp, i64, i32, i64, vp, f32, vp, vp, vp, f32, i32, vp, vp, sz, vp]
         L.tg_topk_select.argtypes = [vp, i64, i64, i64, i64, vp, vp, sz, vp]
         L.tg_topk_select_noalloc.argtypes = [vp, i64, i64, i64, i64, vp, vp]
+        L.tg_topk_select_noalloc_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
         L.tg_random_select.argtypes = [i64, i64, i64, i64, ctypes.c_uint64, vp, vp, sz, vp]
         L.tg_gather_compact.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, vp, vp, vp]
         L.tg_rope_apply.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, f64, vp]
@@ -180,6 +181,16 @@ def tg_topk_select_noalloc(scores, doc_begin: int, doc_end: int, k_doc: int, kep
     _check("tg_topk_select_noalloc", lib().tg_topk_select_noalloc(
         _ptr(scores), N, doc_begin, doc_end, k_doc, _ptr(kept_idx), _stream(stream)))
     return kept_idx
+
+
+def tg_topk_select_noalloc_status(stream=None) -> int:
+    """Raw TG_STATUS_* bits the last tg_topk_select_noalloc call on the current device left (synchronizes
+    the stream); raises only if the read fails."""
+    w = ctypes.c_uint32(0)
+    st = lib().tg_topk_select_noalloc_status(ctypes.byref(w), _stream(stream))
+    if st not in (TG_OK, TG_ERR_TIMEOUT):
+        raise TokenGateError("tg_topk_select_noalloc_status", st)
+    return int(w.value)
 
 
 def tg_random_select(N: int, doc_begin: int, doc_end: int, k_doc: int, seed: int, kept_idx, workspace, stream=None):

@@ -64,3 +64,22 @@ def test_noalloc_rejects_spans_beyond_its_limit():
     with pytest.raises(tg.TokenGateError) as e:
         tg.tg_topk_select_noalloc(big, 0, n_doc, 16, out)
     assert e.value.status == tg.TG_ERR_UNSUPPORTED
+
+
+def test_noalloc_timeout_is_reported_by_its_status_query():
+    # The static array's status word carries a select timeout to the caller.  The grid barrier's limit is
+    # shrunk to a nanosecond (the fault-injection hook: nothing traps or hangs), the call's blocks stop
+    # waiting and set TG_STATUS_SELECT_TIMEOUT, the status query reports it, and the next call -- which
+    # clears the array first -- is exact again and reports nothing.
+    s = synth.score_vector(131072, 34, "normal").cuda()
+    want = _reference(s, 0, 130560, 4096)
+    try:
+        tg.tg_debug_set_select_wait_limit(1)
+        _noalloc(s, 0, 130560, 4096)
+        bits = tg.tg_topk_select_noalloc_status()
+    finally:
+        tg.tg_debug_set_select_wait_limit(0)
+    assert bits & tg.TG_STATUS_SELECT_TIMEOUT
+    again = _noalloc(s, 0, 130560, 4096)
+    assert tg.tg_topk_select_noalloc_status() == 0
+    assert torch.equal(again, want)
