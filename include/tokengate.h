@@ -247,8 +247,9 @@ tg_status tg_rope_apply(tg_bf16* q, int64_t ld_q, tg_bf16* k, int64_t ld_k,
  * Range: V goes through fp16, so |v| must stay within 65504 (fp16's largest
  * finite value; bf16 reaches 3.4e38).  A larger finite v has no fp16 value:
  * the conversion sets TG_STATUS_V_RANGE in the workspace's status word
- * (tg_device_status then returns TG_ERR_RANGE), and the outputs of the rows
- * that attend to that key are not the specified values. */
+ * (tg_device_status then returns TG_ERR_RANGE), and the outputs of the query
+ * heads that read that KV head are undefined (any of their rows may hold
+ * non-finite values). */
 tg_status tg_gated_attention(const tg_bf16* q, int64_t ld_q, const tg_bf16* k, int64_t ld_k,
                              const tg_bf16* v, int64_t ld_v, int64_t K, int32_t Hq,
                              int32_t Hkv, int32_t d_h, const float* s_kept,

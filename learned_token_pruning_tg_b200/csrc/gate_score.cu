@@ -327,7 +327,7 @@ gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* full = bars;                      // [S] even CTA: both CTAs' copies of the stage landed
     uint64_t* empty = bars + C::kStages;        // [S] pair MMA commit + 128 sum-of-squares threads
-    uint64_t* a_full = bars + 2 * C::kStages;   // [S] odd CTA: the even CTA saw `full` (own rows landed)
+    uint64_t* a_full = bars + 2 * C::kStages;   // [S] pair MMA commit: the stage was consumed (odd CTA's row sums)
     uint64_t* acc_full = bars + 3 * C::kStages; // [2] pair MMA commit -> epilogue (both CTAs)
     uint64_t* acc_empty = acc_full + 2;         // [2] even CTA: 256 epilogue threads of the pair -> MMA
     uint64_t* ss_full = acc_full + 4;           // [2] 128 sum-of-squares threads -> epilogue
@@ -430,7 +430,6 @@ gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_
                         ok = false;
                         break;
                     }
-                    mbar_arrive_cluster(cluster_addr(&a_full[s], 1));  // the odd CTA's rows have landed too
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + s * C::kStage);
                     const uint64_t da = smem_desc_sw128(sa, 16, 1024);
@@ -438,6 +437,9 @@ gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
                         mma_ss_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    // the stage's MMAs done: the odd CTA's rows of h had landed, its row sums may read
+                    // them (they are released only after that); then the stage's MMA share of `empty`
+                    mma_commit_pair_mc(&a_full[s], 0x3);
                     mma_commit_pair_mc(&empty[s], 0x3);
                     if (++s == C::kStages) {
                         s = 0;

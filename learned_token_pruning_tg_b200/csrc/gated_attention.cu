@@ -30,9 +30,9 @@
 //               warp w owns TMEM lanes 32 (w mod 4) ..): the row's 128 S values
 //               are read from TMEM into registers, row max, then
 //               P = 2^(S c - m) with c = tau / sqrt(d_h) log2(e), as fp16 into
-//               the S columns (packed fp16 ex2: two values per MUFU operation).
+//               the S columns.
 //               Lazy rescaling: O is rescaled (in TMEM) only when a row max
-//               grows by more than 2^2, so P <= 4.  Causal masking only on
+//               grows by more than 2^8, so P <= 256.  Causal masking only on
 //               the diagonal tile.  At the end O / l to bf16 and the
 //               log-sum-exp.
 // The key bias rides in the tensor core: S is computed as
@@ -63,10 +63,7 @@ namespace attn {
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kBN = 128;        // keys per tile
 constexpr float kLog2e = 1.4426950408889634f;
-// log2 units: O is rescaled when a row's max grows by more than 2, so every exponent
-// y = S c - m stays <= 2 and P <= 4 (the exponent goes through fp16, whose
-// absolute error grows with |y|; see the softmax below)
-constexpr float kRescaleThreshold = 2.0f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 
 template <int D, int NQ>
 struct Cfg {
@@ -109,26 +106,6 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// 2^x for both halves of a packed fp16 pair (one MUFU operation for two values).
-__device__ __forceinline__ uint32_t ex2_h2(uint32_t x) {
-    uint32_t y;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
-// fp16 pair sum and its widening to fp32.
-__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ float2 h2_to_f2(uint32_t h) {
-    float lo, hi;
-    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.f32.f16 %0, l;\n cvt.f32.f16 %1, h;\n}"
-        : "=f"(lo), "=f"(hi)
-        : "r"(h));
-    return make_float2(lo, hi);
 }
 
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
@@ -480,15 +457,9 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                     tmem_st16(o_addr + c0, v);
                 }
             }
-            // P = 2^(S c - m) as fp16 over the first kBN / 2 S columns (already read).  The exponent
-            // y = S c - m is formed in fp32, rounded to an fp16 pair, and raised by one packed ex2
-            // (two values per MUFU operation, already the fp16 pair the P V product reads).  The
-            // rounding of y to fp16 changes P by at most 2^-11 |y| ln 2 of itself: 0.07% for the
-            // largest weights (|y| <= 2, the rescale threshold), 0.5% at y = -16 where P < 2^-16.
-            // The row sum l adds the same fp16 values, four per fp16 lane (at most 16) and then
-            // in fp32.
+            // P = 2^(S c - m) as fp16 over the first kBN / 2 S columns (already read)
             const float2 neg_m = make_float2(-m_run, -m_run);
-            float2 ls = make_float2(0.0f, 0.0f);
+            float2 ls[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
             for (int c0 = 0; c0 < kBN; c0 += 32) {
                 uint32_t p16[16];
@@ -496,16 +467,18 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 for (int i = 0; i < 32; i += 4) {
                     const float2 y0 = ffma2(make_float2(x[c0 + i], x[c0 + i + 1]), sc2, neg_m);
                     const float2 y1 = ffma2(make_float2(x[c0 + i + 2], x[c0 + i + 3]), sc2, neg_m);
-                    p16[i / 2] = ex2_h2(f16x2(y0.x, y0.y));
-                    p16[i / 2 + 1] = ex2_h2(f16x2(y1.x, y1.y));
+                    const float2 p0 = make_float2(ex2(y0.x), ex2(y0.y));
+                    const float2 p1 = make_float2(ex2(y1.x), ex2(y1.y));
+                    ls[0] = fadd2(ls[0], p0);
+                    ls[1] = fadd2(ls[1], p1);
+                    p16[i / 2] = f16x2(p0.x, p0.y);
+                    p16[i / 2 + 1] = f16x2(p1.x, p1.y);
                 }
-#pragma unroll
-                for (int g = 0; g < 16; g += 4)
-                    ls = fadd2(ls, h2_to_f2(hadd2(hadd2(p16[g], p16[g + 1]), hadd2(p16[g + 2], p16[g + 3]))));
                 tmem_st16(s_addr + (c0 >> 1), p16);
             }
+            const float2 lsum = fadd2(ls[0], ls[1]);
             tmem_st_wait();
-            l_run += ls.x + ls.y;
+            l_run += lsum.x + lsum.y;
             tc_fence_before();
             mbar_arrive(&p_full[h]);
         }

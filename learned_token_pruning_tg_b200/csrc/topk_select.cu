@@ -355,7 +355,13 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(
         unsigned part = 0;
         if (tid < sl) {
             const int b = static_cast<int>(rank) * sl + tid;
-            for (uint32_t r = 0; r < ncta; ++r) part += dsmem_ld(dsmem_map(&s_hist[b], r));
+            // every CTA's count of bin b, all loads in flight at once (up to 16 CTAs)
+            uint32_t c[kSelectClusterMax];
+#pragma unroll
+            for (int r = 0; r < kSelectClusterMax; ++r)
+                c[r] = static_cast<uint32_t>(r) < ncta ? dsmem_ld(dsmem_map(&s_hist[b], static_cast<uint32_t>(r))) : 0u;
+#pragma unroll
+            for (int r = 0; r < kSelectClusterMax; ++r) part += c[r];
             s_slice[tid] = part;
         }
         if (warp < 8) {
