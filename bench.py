@@ -468,30 +468,29 @@ def run_tokengate(args, rank, world, local_rank):
         return m
 
     gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    # (3) per-stage kernel times without host launch gaps: the K steps and their stage events captured
-    # in one graph (event-record nodes between the kernels), replayed once inside the timed region
-    sev = [[torch.cuda.Event(enable_timing=True) for _ in names] for _ in range(K)]
-
-    def smarker(i):
-        def m(name):
-            sev[i][names.index(name)].record()
-        return m
-
-    staged, staged_err = None, None
-    if not graph_failed:
-        try:
+    # (3) per-step kernel times in the step's own context and without host launch gaps: one CUDA graph
+    # per prefix of the step (gate; gate + select; ...), each replayed R times between its own events
+    # (after an L2 flush where the workload needs one); a step's time is the difference between the
+    # mean times of the prefix that ends with it and the prefix before it.
+    R = max(10, min(K, 40))
+    prefix_graphs, staged_err = [], None
+    try:
+        calls = list(layer.stage_calls(h).values())
+        for n in range(1, len(calls) + 1):
             gs = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gs):
-                for i in range(K):
-                    between_steps()
-                    layer.run(h, mark=smarker(i))
+                for call in calls[:n]:
+                    call()
             gs.replay()
-            torch.cuda.synchronize()
-            staged = gs
-        except Exception as e:  # report, fall back to the kernel-by-kernel stage times
-            staged_err = f"{type(e).__name__}: {e}"[:200]
-            torch.cuda.synchronize()
-    staged_failed = reduce_max(0.0 if staged is not None else 1.0, dev) > 0.0
+            prefix_graphs.append(gs)
+        torch.cuda.synchronize()
+    except Exception as e:  # report, fall back to the kernel-by-kernel stage times
+        staged_err = f"{type(e).__name__}: {e}"[:200]
+        prefix_graphs = []
+        torch.cuda.synchronize()
+    staged_failed = reduce_max(0.0 if prefix_graphs else 1.0, dev) > 0.0
+    pev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(R)]
+           for _ in prefix_graphs]
     with ClockSampler(dev.index) as clk:
         # (1) K steps launched one kernel at a time, with per-stage events
         if world > 1:
@@ -514,22 +513,26 @@ def run_tokengate(args, rank, world, local_rank):
             torch.cuda.synchronize()
             if world > 1:
                 torch.distributed.barrier()
-        # (3) the K steps with stage events inside one graph
+        # (3) the step's prefixes
         if not staged_failed:
-            staged.replay()
+            for gs, evs in zip(prefix_graphs, pev):
+                for e0, e1 in evs:
+                    between_steps()
+                    e0.record()
+                    gs.replay()
+                    e1.record()
             torch.cuda.synchronize()
             if world > 1:
                 torch.distributed.barrier()
     ms_launched = reduce_max(sum(e[0].elapsed_time(e[-1]) for e in ev) / K, dev)
     stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / K for j, s in enumerate(stages)}
-    stage_timing = "kernel-by-kernel launches (host launch gaps included)"
+    stage_timing = "kernel-by-kernel launches of the timed steps (host launch gaps included)"
     if not staged_failed:
-        try:
-            stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in sev) / K for j, s in enumerate(stages)}
-            stage_timing = "event nodes between the kernels of K steps captured in one CUDA graph"
-        except Exception as e:
-            staged_err = f"{type(e).__name__}: {e}"[:200]
-    del staged
+        prefix_ms = [reduce_max(sum(e0.elapsed_time(e1) for e0, e1 in evs) / R, dev) for evs in pev]
+        stage_ms = {s: prefix_ms[j] - (prefix_ms[j - 1] if j else 0.0) for j, s in enumerate(stages)}
+        stage_timing = (f"step prefixes (gate; gate + select; ...) each captured in a CUDA graph and replayed {R} "
+                        f"times between events; a step's time is the difference of consecutive prefix means")
+    del prefix_graphs
     status = layer.device_status()
     ungraphed = {"ms_per_step": ms_launched, "value": job_throughput(w.N, world, ms_launched), "unit": "tokens/s"}
     if not graph_failed:
@@ -641,7 +644,7 @@ def run_tokengate(args, rank, world, local_rank):
             "step_roofline_frac": step_bound / (ms_step * 1e-3),
             "timing": "value and ms_per_step: K replays of the step captured in one CUDA graph, each between its "
                       "own events; 'ungraphed': the same K steps launched kernel by kernel; path_ms, the kernels "
-                      "and the path fractions come from the stage events named in stage_timing",
+                      "and the path fractions come from the step times named in stage_timing",
             "graph": graph_line, "ungraphed": ungraphed,
             "stage_timing": stage_timing if staged_err is None else f"{stage_timing} ({staged_err})",
             "attention_bias_cost": {"with_bias_ms": t_bias, "without_bias_ms": t_plain, "ratio": t_bias / t_plain},

@@ -154,6 +154,28 @@ tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_begin,
                          int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* The gate and the select as a pair on one workspace, for the path where the
+ * select runs right after the gate: tg_gate_score_for_select is tg_gate_score
+ * (same arguments, same scores bit for bit) that also counts, in its
+ * epilogue, the scores of the rows in [doc_begin, doc_end) by the top 11 bits
+ * of their order-preserving key -- the select's first radix pass -- into the
+ * workspace's select scratch; tg_topk_select_after_gate is tg_topk_select
+ * (same arguments and result) that starts from that count instead of making
+ * the first pass itself, and leaves the count at zero again.  Call them in
+ * this order, on the same stream and workspace, with the same scores, N and
+ * span; a tg_topk_select_after_gate without its gate call, or two gate calls
+ * in a row, select from a wrong count.  The workspace is the gate's
+ * (tg_workspace_bytes(TG_OP_GATE, N, d, d_g), which holds the select
+ * scratch); after a timeout it must be zero-filled again, as for every call. */
+tg_status tg_gate_score_for_select(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
+                                   const tg_bf16* rms_weight, float eps,
+                                   const tg_bf16* W1, const float* b1, const float* w2, float b2,
+                                   int32_t d_g, float* scores, int64_t doc_begin, int64_t doc_end,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+tg_status tg_topk_select_after_gate(const float* scores, int64_t N, int64_t doc_begin,
+                                    int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Top-K selection that allocates nothing and takes no workspace.
  * There is no counterpart on the TokenGate pages: this is a calling-convention
  * variant of tg_topk_select for callers that cannot allocate device memory

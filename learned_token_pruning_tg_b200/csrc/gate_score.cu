@@ -34,6 +34,7 @@ namespace gate {
 constexpr int kBM = 128;       // rows per tile
 constexpr int kBK = 64;        // K elements per stage (one 128-byte swizzle row)
 constexpr int kThreads = 384;  // 12 warps
+constexpr int kHistBins = 2048;  // bins of the select's first radix pass (top 11 bits of the key)
 
 template <int DG>
 struct Cfg {
@@ -49,7 +50,9 @@ struct Cfg {
     static constexpr int kOffBar = kOffB1 + DG * 4;
     static constexpr int kNumBars = 2 * kStages + 7;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmem = kOffMisc + 16 + 1024;  // + alignment slack
+    static constexpr int kOffHist = kOffMisc + 16;
+    static constexpr int kSmem = kOffHist + kHistBins * 4 + 1024;  // + alignment slack
+    static_assert(kStage % 1024 == 0 && kOffBar % 8 == 0 && kSmem <= 232448, "gate shared-memory layout");
 };
 
 struct Args {
@@ -61,7 +64,33 @@ struct Args {
     float b2;
     float* scores;
     unsigned int* status;
+    // when non-null: histogram of the top 11 bits of the radix keys of the scores of rows in [D0, D1)
+    // (the select's first pass), added into these 2048 global counters
+    unsigned int* hist0;
+    int64_t D0, D1;
 };
+
+
+// The select's first-pass histogram of one warp's 32 scores: rows in the document span count; lanes
+// that share a digit are folded into one shared-memory increment.
+__device__ __forceinline__ void hist0_add(unsigned int* s_hist, const Args& a, int64_t grow, float score) {
+    const bool in = grow < a.N && grow >= a.D0 && grow < a.D1;
+    const unsigned active = __ballot_sync(0xffffffffu, in);
+    if (in) {
+        const uint32_t digit = radix_key(score) >> kSelectDigit0Shift;
+        const unsigned peers = __match_any_sync(active, digit);
+        if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(peers) - 1))
+            atomicAdd(&s_hist[digit], static_cast<unsigned>(__popc(peers)));
+    }
+}
+
+// Adds a CTA's histogram into the global one (nonzero bins only).
+__device__ __forceinline__ void hist0_flush(const unsigned int* s_hist, unsigned int* hist0) {
+    for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) {
+        const unsigned c = s_hist[b];
+        if (c) atomicAdd(&hist0[b], c);
+    }
+}
 
 template <int DG>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -82,9 +111,12 @@ gate_score_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_const
     uint64_t* drain = acc_full + 6;             // [1]        MMA completion on the abort path
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    unsigned int* s_hist = reinterpret_cast<unsigned int*>(smem + C::kOffHist);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t num_tiles = (a.N + kBM - 1) / kBM;
+    if (a.hist0)
+        for (int bb = threadIdx.x; bb < kHistBins; bb += kThreads) s_hist[bb] = 0u;
     const int kb_per_tile = a.d / kBK;
 
     if (threadIdx.x == 0) {
@@ -224,6 +256,7 @@ gate_score_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_const
             mbar_arrive(&acc_empty[buf]);
             const int64_t grow = t * kBM + row;
             if (grow < a.N) a.scores[grow] = acc + a.b2;
+            if (a.hist0) hist0_add(s_hist, a, grow, acc + a.b2);
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ row sums of squares
@@ -277,6 +310,7 @@ gate_score_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_const
         tc_fence_after();
         tmem_dealloc(tmem_base, C::kTmemCols);
     }
+    if (a.hist0) hist0_flush(s_hist, a.hist0);
 }
 
 // ---------------------------------------------------------------- CTA-pair kernel (d_g = 256)
@@ -308,7 +342,8 @@ struct PairCfg {
     // full, empty, a_full per stage; acc_full, acc_empty, ss_full, ss_empty per buffer; drain
     static constexpr int kNumBars = 3 * kStages + 9;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmem = kOffMisc + 16 + 1024;
+    static constexpr int kOffHist = kOffMisc + 16;
+    static constexpr int kSmem = kOffHist + kHistBins * 4 + 1024;
 };
 static_assert(PairCfg::kStageA % 1024 == 0 && PairCfg::kStage % 1024 == 0 && PairCfg::kOffBar % 8 == 0 &&
                   PairCfg::kSmem <= 232448,
@@ -335,9 +370,12 @@ gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_
     uint64_t* drain = acc_full + 8;             // [1] MMA completion on the abort path
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    unsigned int* s_hist = reinterpret_cast<unsigned int*>(smem + C::kOffHist);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank_in();   // 0: issues the MMAs
+    if (a.hist0)
+        for (int bb = threadIdx.x; bb < kHistBins; bb += kThreads) s_hist[bb] = 0u;
     const bool leader = rank == 0;
     const int64_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
     const int64_t num_tiles = (a.N + 2 * kBM - 1) / (2 * kBM);  // 256-row tiles of the pair
@@ -489,6 +527,7 @@ gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_
             mbar_arrive_cluster(acc_empty_leader[buf]);
             const int64_t grow = t * 2 * kBM + static_cast<int64_t>(rank) * kBM + row;
             if (grow < a.N) a.scores[grow] = acc + a.b2;
+            if (a.hist0) hist0_add(s_hist, a, grow, acc + a.b2);
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ row sums of squares (own rows)
@@ -541,6 +580,7 @@ gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, C::kTmemCols);
     }
+    if (a.hist0) hist0_flush(s_hist, a.hist0);
 }
 
 // W'_jc = bf16(gamma_c * W1_jc): the RMSNorm weight folded into the first layer.
@@ -614,10 +654,10 @@ static tg_status launch(const CUtensorMap& mh, const CUtensorMap& mw, const Args
 
 using namespace tg;
 
-extern "C" tg_status tg_gate_score(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h, const tg_bf16* rms_weight,
-                                   float eps, const tg_bf16* W1, const float* b1, const float* w2, float b2,
-                                   int32_t d_g, float* scores, void* workspace, size_t workspace_bytes,
-                                   void* stream) {
+static tg_status gate_impl(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h, const tg_bf16* rms_weight, float eps,
+                           const tg_bf16* W1, const float* b1, const float* w2, float b2, int32_t d_g, float* scores,
+                           void* workspace, size_t workspace_bytes, unsigned int* hist0, int64_t D0, int64_t D1,
+                           void* stream) {
     if (N < 0 || d <= 0 || d_g <= 0 || ld_h < d || !(eps >= 0.0f)) return TG_ERR_INVALID_ARG;
     if ((d % 64) != 0 || d > 16384) return TG_ERR_UNSUPPORTED;
     if (d_g != 64 && d_g != 128 && d_g != 256) return TG_ERR_UNSUPPORTED;
@@ -657,6 +697,9 @@ extern "C" tg_status tg_gate_score(const tg_bf16* h, int64_t N, int32_t d, int64
     a.b2 = b2;
     a.scores = scores;
     a.status = status_word(workspace);
+    a.hist0 = hist0;
+    a.D0 = D0;
+    a.D1 = D1;
     const int64_t num_tiles = (N + gate::kBM - 1) / gate::kBM;
     if (d_g == 256 && gate::pair_kernel_available()) {
         // W's half tile: 128 rows per CTA
@@ -670,4 +713,24 @@ extern "C" tg_status tg_gate_score(const tg_bf16* h, int64_t N, int32_t d, int64
         case 128: return gate::launch<128>(mh, mw, a, num_tiles, st);
         default: return gate::launch<256>(mh, mw, a, num_tiles, st);
     }
+}
+
+extern "C" tg_status tg_gate_score(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h, const tg_bf16* rms_weight,
+                                   float eps, const tg_bf16* W1, const float* b1, const float* w2, float b2,
+                                   int32_t d_g, float* scores, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+    return gate_impl(h, N, d, ld_h, rms_weight, eps, W1, b1, w2, b2, d_g, scores, workspace, workspace_bytes, nullptr,
+                     0, 0, stream);
+}
+
+extern "C" tg_status tg_gate_score_for_select(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
+                                              const tg_bf16* rms_weight, float eps, const tg_bf16* W1, const float* b1,
+                                              const float* w2, float b2, int32_t d_g, float* scores,
+                                              int64_t doc_begin, int64_t doc_end, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+    if (doc_begin < 0 || doc_end < doc_begin || doc_end > N) return TG_ERR_INVALID_ARG;
+    if (!workspace) return TG_ERR_INVALID_ARG;
+    SelectScratch* sc = reinterpret_cast<SelectScratch*>(static_cast<char*>(workspace) + kWsHeader);
+    return gate_impl(h, N, d, ld_h, rms_weight, eps, W1, b1, w2, b2, d_g, scores, workspace, workspace_bytes,
+                     &sc->hist[0][0], doc_begin, doc_end, stream);
 }

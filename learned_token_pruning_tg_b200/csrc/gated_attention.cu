@@ -81,7 +81,7 @@ struct Cfg {
     static constexpr int kOffAugA = kOffV + kStages * kKVTile;  // [NQ]      gamma_h parts, every row alike
     static constexpr int kOffAugB = kOffAugA + NQ * kAugTile;   // [kStages] s_c parts of a K tile's keys
     static constexpr int kOffBar = kOffAugB + kStages * kAugTile;
-    static constexpr int kNumBars = 1 + 5 * kStages + 3 * NQ + 1;
+    static constexpr int kNumBars = 2 + 5 * kStages + 4 * NQ + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmem = kOffMisc + 16 + 1024;
     static constexpr uint32_t kTmemCols = (NQ * kBN + NQ * D > 256) ? 512 : 256;
@@ -179,31 +179,45 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* q_full = bars;                        // TMA -> MMA
-    uint64_t* k_full = bars + 1;                    // [kStages] TMA -> MMA
+    uint64_t* q_full = bars;                        // TMA -> MMA (one phase per work item)
+    uint64_t* q_empty = bars + 1;                   // commit after an item's last S -> TMA (next Q), bias warp
+    uint64_t* k_full = bars + 2;                    // [kStages] TMA -> MMA
     uint64_t* k_empty = k_full + kStages;           // [kStages] commit after the last S of a K tile -> TMA
     uint64_t* v_full = k_empty + kStages;           // [kStages] TMA -> MMA
     uint64_t* v_empty = v_full + kStages;           // [kStages] commit after the last P V of a V tile -> TMA
     uint64_t* aug_full = v_empty + kStages;         // [kStages] converter (32 lanes) wrote B of a K tile -> MMA
     uint64_t* s_full = aug_full + kStages;          // [NQ] commit after S_h(j) (and P_h(j-1) V) -> softmax h
     uint64_t* p_full = s_full + NQ;                 // [NQ] 128 softmax threads wrote P_h(j) -> MMA
-    uint64_t* o_full = p_full + NQ;                 // [NQ] commit after the last P_h V -> epilogue h
-    uint64_t* drain = o_full + NQ;                  // abort path
+    uint64_t* o_full = p_full + NQ;                 // [NQ] commit after an item's last P_h V -> epilogue h
+    uint64_t* o_empty = o_full + NQ;                // [NQ] 128 epilogue threads read O_h -> MMA (next item)
+    uint64_t* drain = o_empty + NQ;                 // abort path
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-    (void)kStages;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Work items: (128-query tile, NQ query heads of one KV head), heaviest (most key tiles) first.
+    // Persistent CTAs take them in snake order -- round r hands item r G + b to CTA b on even
+    // rounds and r G + G - 1 - b on odd ones -- which evens out the triangular causal work.
     const int per_tile = a.Hkv * a.pairs_per_group;
-    const int m_tile = a.num_q_tiles - 1 - static_cast<int>(blockIdx.x / per_tile);  // heaviest first
-    const int rem = static_cast<int>(blockIdx.x % per_tile);
-    const int kvh = rem / a.pairs_per_group;
-    const int head0 = kvh * (a.Hq / a.Hkv) + (rem % a.pairs_per_group) * NQ;
-    // causal: key tiles 0..m_tile, the last one on the diagonal
-    const int n_kv = m_tile + 1;
+    const int n_items = a.num_q_tiles * per_tile;
+    const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+    auto item_of = [&](int r) -> int { return r * G + ((r & 1) ? (G - 1 - b) : b); };
+    struct Item {
+        int m_tile, kvh, head0, n_kv;
+    };
+    auto decode = [&](int idx) -> Item {
+        Item it;
+        it.m_tile = a.num_q_tiles - 1 - idx / per_tile;
+        const int rem = idx % per_tile;
+        it.kvh = rem / a.pairs_per_group;
+        it.head0 = it.kvh * (a.Hq / a.Hkv) + (rem % a.pairs_per_group) * NQ;
+        it.n_kv = it.m_tile + 1;  // causal: key tiles 0..m_tile, the last one on the diagonal
+        return it;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
@@ -215,6 +229,7 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             mbar_init(&s_full[h], 1);
             mbar_init(&p_full[h], 128);
             mbar_init(&o_full[h], 1);
+            mbar_init(&o_empty[h], 128);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -227,23 +242,6 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 2) {
-        // A_h: every row holds gamma_h's parts (i = col / 3 for col < 9, zeros after)
-        uint4* aug_a = reinterpret_cast<uint4*>(smem + C::kOffAugA);
-#pragma unroll
-        for (int h = 0; h < NQ; ++h) {
-            __nv_bfloat16 g[3];
-            split3_bf16(a.gain ? a.gain[head0 + h] * kLog2e / a.scale_log2 : 0.0f, g);
-            const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
-            const uint4 c0 = make_uint4(bf2(g[0], g[0]), bf2(g[0], g[1]), bf2(g[1], g[1]), bf2(g[2], g[2]));
-            const uint4 c1 = make_uint4(bf2(g[2], z), 0u, 0u, 0u);
-            for (int r = lane; r < kBM; r += 32) {
-                aug_a[h * (C::kAugTile / 16) + aug_slot(r, 0)] = c0;
-                aug_a[h * (C::kAugTile / 16) + aug_slot(r, 1)] = c1;
-            }
-        }
-        fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads (after the sync below)
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -254,35 +252,56 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         if (lane == 0) {
             int k_last[kStages], v_last[kStages];  // parity of the last phase loaded per stage, -1 if none
             for (int i = 0; i < kStages; ++i) k_last[i] = v_last[i] = -1;
-            mbar_arrive_expect_tx(q_full, NQ * C::kQTile);
-            for (int h = 0; h < NQ; ++h)
-#pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(smem + C::kOffQ + h * C::kQTile + c * (kBM * 128), &tmap_q, q_full, c * 64,
-                                head0 + h, m_tile * kBM, kEvictFirst);
-            auto load = [&](int j, uint64_t* empty, uint64_t* full, int off, const CUtensorMap* map,
-                            int* last) -> bool {
-                const int st = j % kStages;
-                const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
-                if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT))
+            int q_last = -1;
+            // K (is_k) or V tile j of an item whose first tile is number g0 of this CTA: wait for its ring
+            // slot, then one TMA box per 64-column chunk
+            auto load_kv = [&](int g0, int j, int kvh, bool is_k) -> bool {
+                const int g = g0 + j;
+                const int st = g % kStages;
+                const uint32_t ph = static_cast<uint32_t>(g / kStages) & 1;
+                uint64_t* full = is_k ? k_full : v_full;
+                if (!mbar_wait(is_k ? &k_empty[st] : &v_empty[st], ph ^ 1, abort_flag, a.status,
+                               TG_STATUS_ATTENTION_TIMEOUT))
                     return false;
-                uint8_t* dst = smem + off + st * C::kKVTile;
+                uint8_t* dst = smem + (is_k ? C::kOffK : C::kOffV) + st * C::kKVTile;
                 mbar_arrive_expect_tx(&full[st], C::kKVTile);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(dst + c * (kBN * 128), map, &full[st], c * 64, kvh, j * kBN, kEvictLast);
-                last[st] = static_cast<int>(ph);
+                    tma_load_3d(dst + c * (kBN * 128), is_k ? &tmap_k : &tmap_v, &full[st], c * 64, kvh, j * kBN,
+                                kEvictLast);
+                (is_k ? k_last : v_last)[st] = static_cast<int>(ph);
                 return true;
             };
-            // K runs one tile ahead of V: S(j+1) needs only K(j+1); P(j) V(j) waits for softmax j anyway.
-            bool ok = load(0, k_empty, k_full, C::kOffK, &tmap_k, k_last);
-            for (int j = 0; j < n_kv && ok; ++j) {
-                if (j + 1 < n_kv) ok = load(j + 1, k_empty, k_full, C::kOffK, &tmap_k, k_last);
-                if (ok) ok = load(j, v_empty, v_full, C::kOffV, &tmap_v, v_last);
+            bool ok = true;
+            int g0 = 0;
+            for (int r = 0, it = 0; ok && r * G < n_items; ++r) {
+                const int idx = item_of(r);
+                if (idx >= n_items) continue;
+                const Item w = decode(idx);
+                // Q of this item once the previous item's last S no longer reads the Q tiles
+                if (!(ok = mbar_wait(q_empty, (static_cast<uint32_t>(it) & 1) ^ 1, abort_flag, a.status,
+                                     TG_STATUS_ATTENTION_TIMEOUT)))
+                    break;
+                mbar_arrive_expect_tx(q_full, NQ * C::kQTile);
+                for (int h = 0; h < NQ; ++h)
+#pragma unroll
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(smem + C::kOffQ + h * C::kQTile + c * (kBM * 128), &tmap_q, q_full, c * 64,
+                                    w.head0 + h, w.m_tile * kBM, kEvictFirst);
+                q_last = it & 1;
+                // K runs one tile ahead of V: S(j+1) needs only K(j+1); P(j) V(j) waits for softmax j anyway.
+                ok = load_kv(g0, 0, w.kvh, true);
+                for (int j = 0; j < w.n_kv && ok; ++j) {
+                    if (j + 1 < w.n_kv) ok = load_kv(g0, j + 1, w.kvh, true);
+                    if (ok) ok = load_kv(g0, j, w.kvh, false);
+                }
+                g0 += w.n_kv;
+                ++it;
             }
             // Every issued copy must land before shared memory is released (matters on abort only).
             volatile int no_abort = 0;
-            mbar_wait(q_full, 0, &no_abort, a.status, TG_STATUS_ATTENTION_TIMEOUT);
+            if (q_last >= 0)
+                mbar_wait(q_full, static_cast<uint32_t>(q_last), &no_abort, a.status, TG_STATUS_ATTENTION_TIMEOUT);
             for (int i = 0; i < kStages; ++i) {
                 if (k_last[i] >= 0)
                     mbar_wait(&k_full[i], static_cast<uint32_t>(k_last[i]), &no_abort, a.status,
@@ -308,17 +327,17 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             const uint32_t aa_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffAugA), 128);
             const uint32_t ab_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffAugB), 128);
             const bool bias = a.gain != nullptr && a.s_kept != nullptr;
-            // K tile j and its bias operand B both in shared memory
-            auto wait_k = [&](int j) -> bool {
-                const uint32_t ph = static_cast<uint32_t>(j / kStages) & 1;
-                return mbar_wait(&k_full[j % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT) &&
-                       mbar_wait(&aug_full[j % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
+            // K tile g and its bias operand B both in shared memory
+            auto wait_k = [&](int g) -> bool {
+                const uint32_t ph = static_cast<uint32_t>(g / kStages) & 1;
+                return mbar_wait(&k_full[g % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT) &&
+                       mbar_wait(&aug_full[g % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
             };
-            // S_h = Q_h K_j^T into head h's S columns, then signal softmax h (the commit
-            // also covers every earlier MMA of this thread, P_h(j-1) V_{j-1} included)
-            auto issue_s = [&](int h, int j) {
+            // S_h = Q_h K_g^T into head h's S columns, then signal softmax h (the commit
+            // also covers every earlier MMA of this thread, P_h(g-1) V_{g-1} included)
+            auto issue_s = [&](int h, int g) {
                 const uint32_t q_lo = q_lo0 + static_cast<uint32_t>(h * (C::kQTile >> 4));
-                const uint32_t k_lo = k_lo0 + static_cast<uint32_t>((j % kStages) * (C::kKVTile >> 4));
+                const uint32_t k_lo = k_lo0 + static_cast<uint32_t>((g % kStages) * (C::kKVTile >> 4));
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     // K step k: 64-column chunk k / 4, 32-byte column offset k % 4 inside the swizzle atom
@@ -329,46 +348,62 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 // + A_h B^T: the key bias g_h s_c / c, one more K step (none without a bias)
                 if (bias)
                     mma_ss_lo(tmem + C::col_s(h), aa_lo0 + static_cast<uint32_t>(h * (C::kAugTile >> 4)),
-                              ab_lo0 + static_cast<uint32_t>((j % kStages) * (C::kAugTile >> 4)), ahi, idesc_s, 1u);
+                              ab_lo0 + static_cast<uint32_t>((g % kStages) * (C::kAugTile >> 4)), ahi, idesc_s, 1u);
                 mma_commit(&s_full[h]);
             };
-            bool ok = mbar_wait(q_full, 0, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
-            if (ok) ok = wait_k(0);
-            if (ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int h = 0; h < NQ; ++h) issue_s(h, 0);
-                mma_commit(&k_empty[0]);
-            }
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int st = j % kStages;
-                const bool more = j + 1 < n_kv;
-                if (!(ok = mbar_wait(&v_full[st], static_cast<uint32_t>(j / kStages) & 1, abort_flag, a.status,
+            bool ok = true;
+            int g0 = 0;
+            for (int r = 0, it = 0; ok && r * G < n_items; ++r) {
+                const int idx = item_of(r);
+                if (idx >= n_items) continue;
+                const int n_kv = decode(idx).n_kv;
+                if (!(ok = mbar_wait(q_full, static_cast<uint32_t>(it) & 1, abort_flag, a.status,
                                      TG_STATUS_ATTENTION_TIMEOUT)))
                     break;
-                if (more && !(ok = wait_k(j + 1))) break;
-                const uint32_t v_lo = v_lo0 + static_cast<uint32_t>(st * (C::kKVTile >> 4));
+                if (!(ok = wait_k(g0))) break;
+                tc_fence_after();
 #pragma unroll
-                for (int h = 0; h < NQ && ok; ++h) {
-                    // O_h += P_h(j) V_j once softmax h has written P_h(j) ...
-                    if (!(ok = mbar_wait(&p_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status,
-                                         TG_STATUS_ATTENTION_TIMEOUT)))
+                for (int h = 0; h < NQ; ++h) issue_s(h, g0);
+                mma_commit(&k_empty[g0 % kStages]);
+                if (n_kv == 1) mma_commit(q_empty);
+                for (int j = 0; j < n_kv && ok; ++j) {
+                    const int g = g0 + j;
+                    const int st = g % kStages;
+                    const bool more = j + 1 < n_kv;
+                    if (!(ok = mbar_wait(&v_full[st], static_cast<uint32_t>(g / kStages) & 1, abort_flag,
+                                         a.status, TG_STATUS_ATTENTION_TIMEOUT)))
                         break;
-                    tc_fence_after();
+                    if (more && !(ok = wait_k(g + 1))) break;
+                    const uint32_t v_lo = v_lo0 + static_cast<uint32_t>(st * (C::kKVTile >> 4));
 #pragma unroll
-                    for (int k = 0; k < kBN / 16; ++k)  // 16 keys per step: 16 rows of 128 bytes in each chunk
-                        mma_ts_lo(tmem + C::col_o(h), tmem + C::col_s(h) + static_cast<uint32_t>(k * 8),
-                                  v_lo + static_cast<uint32_t>(k * (2048 >> 4)), dhi, idesc_o,
-                                  (j > 0 || k > 0) ? 1u : 0u);
-                    // ... then, behind it in the same pipe, S_h(j+1) over the same columns
-                    if (more)
-                        issue_s(h, j + 1);
-                    else
-                        mma_commit(&o_full[h]);
+                    for (int h = 0; h < NQ && ok; ++h) {
+                        // O_h += P_h(j) V_j once softmax h has written P_h(j) (and, on the item's first
+                        // tile, once the previous item's epilogue has read O_h out) ...
+                        if (!(ok = mbar_wait(&p_full[h], static_cast<uint32_t>(g) & 1, abort_flag, a.status,
+                                             TG_STATUS_ATTENTION_TIMEOUT)))
+                            break;
+                        if (j == 0 && !(ok = mbar_wait(&o_empty[h], (static_cast<uint32_t>(it) & 1) ^ 1, abort_flag,
+                                                       a.status, TG_STATUS_ATTENTION_TIMEOUT)))
+                            break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int k = 0; k < kBN / 16; ++k)  // 16 keys per step: 16 rows of 128 bytes in each chunk
+                            mma_ts_lo(tmem + C::col_o(h), tmem + C::col_s(h) + static_cast<uint32_t>(k * 8),
+                                      v_lo + static_cast<uint32_t>(k * (2048 >> 4)), dhi, idesc_o,
+                                      (j > 0 || k > 0) ? 1u : 0u);
+                        // ... then, behind it in the same pipe, S_h(j+1) over the same columns
+                        if (more)
+                            issue_s(h, g + 1);
+                        else
+                            mma_commit(&o_full[h]);
+                    }
+                    if (!ok) break;
+                    mma_commit(&v_empty[st]);
+                    if (more) mma_commit(&k_empty[(g + 1) % kStages]);
+                    if (more && j + 2 == n_kv) mma_commit(q_empty);  // the item's last S is issued
                 }
-                if (!ok) break;
-                mma_commit(&v_empty[st]);
-                if (more) mma_commit(&k_empty[(j + 1) % kStages]);
+                g0 += n_kv;
+                ++it;
             }
             if (!ok) {
                 mma_commit(drain);
@@ -377,20 +412,41 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             }
         }
     } else if (warp == 2) {
-        // ------------------------------------------------------------ bias operand B
-        // B for K tile jb: row c holds s_c's parts (k = col mod 3 for col < 9, zeros after)
+        // ------------------------------------------------------------ bias operands A and B
+        uint4* aug_a = reinterpret_cast<uint4*>(smem + C::kOffAugA);
         uint4* aug_b = reinterpret_cast<uint4*>(smem + C::kOffAugB);
-        auto fill_aug = [&](int jb) -> bool {
-            const int st = jb % kStages;
-            // the slot is free once the S MMAs of tile jb - kStages are done (same release as K)
-            if (!mbar_wait(&k_empty[st], (static_cast<uint32_t>(jb / kStages) & 1) ^ 1, abort_flag, a.status,
+        // B for K tile g (key tile j of the item): row c holds s_c's parts (k = col mod 3 for col < 9)
+        auto fill_aug = [&](int g, int j, const Item& w, int it) -> bool {
+            const int st = g % kStages;
+            // the slot is free once the S MMAs of tile g - kStages are done (same release as K)
+            if (!mbar_wait(&k_empty[st], (static_cast<uint32_t>(g / kStages) & 1) ^ 1, abort_flag, a.status,
                            TG_STATUS_ATTENTION_TIMEOUT))
                 return false;
+            if (j == 0) {
+                // A_h of this item: every row holds gamma_h's parts (i = col / 3 for col < 9, zeros after),
+                // written once the previous item's S MMAs are done (q_empty)
+                if (!mbar_wait(q_empty, (static_cast<uint32_t>(it) & 1) ^ 1, abort_flag, a.status,
+                               TG_STATUS_ATTENTION_TIMEOUT))
+                    return false;
+#pragma unroll
+                for (int h = 0; h < NQ; ++h) {
+                    __nv_bfloat16 gp[3];
+                    split3_bf16(a.gain ? a.gain[w.head0 + h] * kLog2e / a.scale_log2 : 0.0f, gp);
+                    const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
+                    const uint4 c0 = make_uint4(bf2(gp[0], gp[0]), bf2(gp[0], gp[1]), bf2(gp[1], gp[1]),
+                                                bf2(gp[2], gp[2]));
+                    const uint4 c1 = make_uint4(bf2(gp[2], z), 0u, 0u, 0u);
+                    for (int rr = lane; rr < kBM; rr += 32) {
+                        aug_a[h * (C::kAugTile / 16) + aug_slot(rr, 0)] = c0;
+                        aug_a[h * (C::kAugTile / 16) + aug_slot(rr, 1)] = c1;
+                    }
+                }
+            }
             uint4* dst = aug_b + st * (C::kAugTile / 16);
 #pragma unroll
             for (int i = 0; i < kBN / 32; ++i) {
                 const int c = i * 32 + lane;
-                const int64_t key = static_cast<int64_t>(jb) * kBN + c;
+                const int64_t key = static_cast<int64_t>(j) * kBN + c;
                 __nv_bfloat16 p[3];
                 split3_bf16((a.s_kept && key < a.K) ? a.s_kept[key] : 0.0f, p);
                 const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
@@ -401,91 +457,110 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             mbar_arrive(&aug_full[st]);
             return true;
         };
-        for (int j = 0; j < n_kv; ++j)
-            if (!fill_aug(j)) break;
+        bool ok = true;
+        int g0 = 0;
+        for (int r = 0, it = 0; ok && r * G < n_items; ++r) {
+            const int idx = item_of(r);
+            if (idx >= n_items) continue;
+            const Item w = decode(idx);
+            for (int j = 0; j < w.n_kv && ok; ++j) ok = fill_aug(g0 + j, j, w, it);
+            g0 += w.n_kv;
+            ++it;
+        }
     } else {
         // ------------------------------------------------------------ softmax + epilogue of head h
         const int sw = warp - C::kSoftmaxWarp0;
         const int h = sw >> 2;
         const int q = warp & 3;         // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;  // query row inside the tile == TMEM lane
-        const int head = head0 + h;
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + C::col_s(h);
         const uint32_t o_addr = tmem + lane_off + C::col_o(h);
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-        float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
-        for (int j = 0; j < n_kv && ok; ++j) {
-            if (!(ok = warp_wait(&s_full[h], static_cast<uint32_t>(j) & 1, abort_flag, a.status))) break;
-            tc_fence_after();
-            // the row's 128 S values (bias included)
-            float x[kBN];
-            {
-                uint32_t* xv = reinterpret_cast<uint32_t*>(x);
+        int g0 = 0;
+        for (int r = 0, it = 0; ok && r * G < n_items; ++r) {
+            const int idx = item_of(r);
+            if (idx >= n_items) continue;
+            const int n_kv = a.num_q_tiles - idx / per_tile;  // the item's key tiles (its query tile + 1)
+            float m_run = -INFINITY, l_run = 0.0f;
+            for (int j = 0; j < n_kv && ok; ++j) {
+                if (!(ok = warp_wait(&s_full[h], static_cast<uint32_t>(g0 + j) & 1, abort_flag, a.status))) break;
+                tc_fence_after();
+                // the row's 128 S values (bias included)
+                float x[kBN];
+                {
+                    uint32_t* xv = reinterpret_cast<uint32_t*>(x);
 #pragma unroll
-                for (int c = 0; c < kBN; c += 32) tmem_ld32(s_addr + c, *reinterpret_cast<uint32_t(*)[32]>(xv + c));
-                tmem_ld_wait();
-            }
-            // on the diagonal tile, key c is in the future of query row r when c > r
-            if (j == n_kv - 1) {
-#pragma unroll
-                for (int c = 0; c < kBN; ++c)
-                    if (c > row) x[c] = -INFINITY;
-            }
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int c = 0; c < kBN; c += 2) mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], x[c], x[c + 1]);
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
-            // lazy rescaling: keep the stale max unless this row's max grew by more than 2^8
-            const bool need = mx > m_run + kRescaleThreshold;
-            float alpha = 1.0f;
-            if (need) {
-                alpha = ex2(m_run - mx);  // 0 on the first tile (m_run = -inf)
-                m_run = mx;
-                l_run *= alpha;
-            }
-            // S_h(j) complete implies P_h(j-1) V_{j-1} complete: O_h may be rescaled now
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(o_addr + c0, v);
+                    for (int c = 0; c < kBN; c += 32)
+                        tmem_ld32(s_addr + c, *reinterpret_cast<uint32_t(*)[32]>(xv + c));
                     tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                    tmem_st16(o_addr + c0, v);
                 }
-            }
-            // P = 2^(S c - m) as fp16 over the first kBN / 2 S columns (already read)
-            const float2 neg_m = make_float2(-m_run, -m_run);
-            float2 ls[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+                // on the diagonal tile, key c is in the future of query row r when c > r
+                if (j == n_kv - 1) {
 #pragma unroll
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
-                uint32_t p16[16];
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float2 y0 = ffma2(make_float2(x[c0 + i], x[c0 + i + 1]), sc2, neg_m);
-                    const float2 y1 = ffma2(make_float2(x[c0 + i + 2], x[c0 + i + 3]), sc2, neg_m);
-                    const float2 p0 = make_float2(ex2(y0.x), ex2(y0.y));
-                    const float2 p1 = make_float2(ex2(y1.x), ex2(y1.y));
-                    ls[0] = fadd2(ls[0], p0);
-                    ls[1] = fadd2(ls[1], p1);
-                    p16[i / 2] = f16x2(p0.x, p0.y);
-                    p16[i / 2 + 1] = f16x2(p1.x, p1.y);
+                    for (int c = 0; c < kBN; ++c)
+                        if (c > row) x[c] = -INFINITY;
                 }
-                tmem_st16(s_addr + (c0 >> 1), p16);
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int c = 0; c < kBN; c += 2) mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], x[c], x[c + 1]);
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
+                // lazy rescaling: keep the stale max unless this row's max grew by more than 2^8
+                const bool need = mx > m_run + kRescaleThreshold;
+                float alpha = 1.0f;
+                if (need) {
+                    alpha = ex2(m_run - mx);  // 0 on the first tile (m_run = -inf)
+                    m_run = mx;
+                    l_run *= alpha;
+                }
+                // S_h(j) complete implies P_h(j-1) V_{j-1} complete: O_h may be rescaled now
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld16(o_addr + c0, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                        tmem_st16(o_addr + c0, v);
+                    }
+                }
+                // P = 2^(S c - m) as fp16 over the first kBN / 2 S columns (already read)
+                const float2 neg_m = make_float2(-m_run, -m_run);
+                float2 ls[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll
+                for (int c0 = 0; c0 < kBN; c0 += 32) {
+                    uint32_t p16[16];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float2 y0 = ffma2(make_float2(x[c0 + i], x[c0 + i + 1]), sc2, neg_m);
+                        const float2 y1 = ffma2(make_float2(x[c0 + i + 2], x[c0 + i + 3]), sc2, neg_m);
+                        const float2 p0 = make_float2(ex2(y0.x), ex2(y0.y));
+                        const float2 p1 = make_float2(ex2(y1.x), ex2(y1.y));
+                        ls[0] = fadd2(ls[0], p0);
+                        ls[1] = fadd2(ls[1], p1);
+                        p16[i / 2] = f16x2(p0.x, p0.y);
+                        p16[i / 2 + 1] = f16x2(p1.x, p1.y);
+                    }
+                    tmem_st16(s_addr + (c0 >> 1), p16);
+                }
+                const float2 lsum = fadd2(ls[0], ls[1]);
+                tmem_st_wait();
+                l_run += lsum.x + lsum.y;
+                tc_fence_before();
+                mbar_arrive(&p_full[h]);
             }
-            const float2 lsum = fadd2(ls[0], ls[1]);
-            tmem_st_wait();
-            l_run += lsum.x + lsum.y;
-            tc_fence_before();
-            mbar_arrive(&p_full[h]);
-        }
-        if (ok && warp_wait(&o_full[h], 0, abort_flag, a.status)) {
-            // epilogue: normalise, store bf16 rows and the log-sum-exp
+            if (!ok || !warp_wait(&o_full[h], static_cast<uint32_t>(it) & 1, abort_flag, a.status)) {
+                ok = false;
+                break;
+            }
+            // epilogue: normalise, store bf16 rows and the log-sum-exp; O_h's columns are free for the
+            // next item once every row has been read out
             tc_fence_after();
-            const int64_t grow = static_cast<int64_t>(m_tile) * kBM + row;
+            const Item w = decode(idx);
+            const int head = w.head0 + h;
+            const int64_t grow = static_cast<int64_t>(w.m_tile) * kBM + row;
             const float inv_l = 1.0f / l_run;
             __nv_bfloat16* orow = a.out + (grow * a.Hq + head) * D;
 #pragma unroll
@@ -493,6 +568,10 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
                 uint32_t v[32];
                 tmem_ld32(o_addr + c0, v);
                 tmem_ld_wait();
+                if (c0 + 32 == D) {
+                    tc_fence_before();
+                    mbar_arrive(&o_empty[h]);
+                }
                 if (grow < a.K) {
                     uint32_t o[16];
 #pragma unroll
@@ -506,6 +585,8 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             }
             if (a.lse && grow < a.K)
                 a.lse[static_cast<int64_t>(head) * a.K + grow] = (m_run + log2f(l_run)) / kLog2e;
+            g0 += n_kv;
+            ++it;
         }
     }
 
@@ -549,8 +630,10 @@ static tg_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     if (!set_max_dynamic_smem(kern, C::kSmem, smem_set))
         return TG_ERR_CUDA;
     a.pairs_per_group = (a.Hq / a.Hkv) / NQ;
-    const int64_t grid = static_cast<int64_t>(a.num_q_tiles) * a.Hkv * a.pairs_per_group;
-    if (grid > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
+    const int64_t items = static_cast<int64_t>(a.num_q_tiles) * a.Hkv * a.pairs_per_group;
+    if (items > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
+    // persistent: one CTA per SM (TMEM and shared memory allow no more), each taking several items
+    const int grid = static_cast<int>(std::min<int64_t>(items, num_sms()));
     kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, st>>>(mq, mk, mv, a);
     return launch_status();
 }

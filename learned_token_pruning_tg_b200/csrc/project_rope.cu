@@ -13,7 +13,8 @@
 //              accumulator (one bf16 rounding instead of two)
 //   v heads:   bf16 into qkv and, when asked, fp16 into v16
 // Angles are formed in fp64 exactly as tg_rope_apply forms them (a small
-// kernel writes the cos / sin table of every kept row into the workspace).
+// kernel writes the cos / sin table of every kept row into the workspace, from
+// frequencies the host forms in fp64).
 //
 // Kernel (persistent, one CTA per SM, 8 warps): tiles of 128 rows x 256
 // output columns, row-tile-major so the CTAs working at one time share the
@@ -72,20 +73,24 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// cos / sin of pos[r] * base^(-2t / d_h), t < d_h / 2, in fp64, rounded to fp32.
-__global__ void __launch_bounds__(64) rope_table_kernel(const int32_t* __restrict__ pos, int64_t K, int D,
-                                                        double base, float* __restrict__ cos_t,
-                                                        float* __restrict__ sin_t) {
-    const int half = D >> 1;
-    for (int64_t r = blockIdx.x; r < K; r += gridDim.x) {
-        const double p = static_cast<double>(__ldg(pos + r));
-        for (int t = threadIdx.x; t < half; t += blockDim.x) {
-            const double inv_freq = pow(base, -2.0 * static_cast<double>(t) / static_cast<double>(D));
-            double s, c;
-            sincos(p * inv_freq, &s, &c);
-            cos_t[r * half + t] = static_cast<float>(c);
-            sin_t[r * half + t] = static_cast<float>(s);
-        }
+// The rotary frequencies base^(-2t / d_h), t < d_h / 2, formed on the host in fp64.
+struct InvFreq {
+    double v[64];
+};
+
+// cos / sin of pos[r] * inv_freq[t] in fp64, rounded to fp32; one (row, t) per thread.
+__global__ void __launch_bounds__(256) rope_table_kernel(const int32_t* __restrict__ pos, int64_t K, int half,
+                                                         const __grid_constant__ InvFreq f, float* __restrict__ cos_t,
+                                                         float* __restrict__ sin_t) {
+    const int64_t n = K * half;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * 256) {
+        const int64_t r = i / half;
+        const int t = static_cast<int>(i - r * half);
+        double s, c;
+        sincos(static_cast<double>(__ldg(pos + r)) * f.v[t], &s, &c);
+        cos_t[i] = static_cast<float>(c);
+        sin_t[i] = static_cast<float>(s);
     }
 }
 
@@ -544,8 +549,11 @@ extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int
     float* cos_t = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeader);
     float* sin_t = cos_t + K * (d_h / 2);
     {
-        const int64_t blocks = std::min<int64_t>(K, static_cast<int64_t>(num_sms()) * 16);
-        proj::rope_table_kernel<<<static_cast<unsigned>(blocks), 64, 0, st>>>(pos, K, d_h, base, cos_t, sin_t);
+        const int64_t blocks = std::min<int64_t>((K * (d_h / 2) + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
+        proj::InvFreq f;
+        for (int t = 0; t < d_h / 2; ++t)
+            f.v[t] = std::pow(base, -2.0 * static_cast<double>(t) / static_cast<double>(d_h));
+        proj::rope_table_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(pos, K, d_h / 2, f, cos_t, sin_t);
         if (launch_status() != TG_OK) return TG_ERR_CUDA;
     }
     CUtensorMap mx, mw;

@@ -29,6 +29,17 @@ struct SelectScratch {
     unsigned int blk_eq[kSelectMaxBlocks];
 };
 
+// Order-preserving 32-bit key of an fp32 score for the radix select: larger
+// score, larger key; -0 == +0; NaN ranks below every number.  The gate's
+// first-pass histogram and the select use the same key.
+__device__ __forceinline__ uint32_t radix_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN ranks lowest
+    if (u == 0x80000000u) u = 0u;                     // -0 == +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+constexpr int kSelectDigit0Shift = 21;  // the first radix pass ranks keys by their top 11 bits
+
 // Wait limit for every spin in the library (nanoseconds of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 

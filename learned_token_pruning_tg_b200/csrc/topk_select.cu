@@ -52,12 +52,6 @@ __device__ __forceinline__ uint32_t random_key(uint64_t seed, int64_t i) {
     return static_cast<uint32_t>((z ^ (z >> 31)) >> 32);
 }
 
-__device__ __forceinline__ uint32_t radix_key(float f) {
-    uint32_t u = __float_as_uint(f);
-    if ((u & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN ranks lowest
-    if (u == 0x80000000u) u = 0u;                     // -0 == +0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 // Time limit of the grid barrier's wait (ns of %globaltimer), per device.
 // tg_debug_set_select_wait_limit shrinks it so that tests can make the barrier
@@ -132,6 +126,7 @@ struct SelectArgs {
     SelectScratch* sc;
     unsigned int* status;
     int ept;           // keys per thread actually used (<= EPT)
+    int hist_given;    // the first pass's histogram is already in sc->hist[0] (written with the scores)
 };
 
 template <int EPT>
@@ -160,6 +155,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const Se
         const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
         const int nb = p == 2 ? 1024 : 2048;
         const uint32_t dmask = static_cast<uint32_t>(nb - 1);
+        if (!(p == 0 && a.hist_given)) {
         for (int b = tid; b < 2048; b += kSelectThreads) s_hist[b] = 0;
         __syncthreads();
 #pragma unroll
@@ -181,6 +177,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const Se
             if (c) atomicAdd(&a.sc->hist[p][b], c);
         }
         if (!grid_sync(a.sc, nblocks, a.status, &s_ok)) return;
+        }
 
         // Locate the bin holding the krem-th largest key: scan bins from the top digit down.
         const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
@@ -334,6 +331,27 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(
         const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
         const int nb = p == 2 ? 1024 : 2048;
         const uint32_t dmask = static_cast<uint32_t>(nb - 1);
+        if (p == 0 && a.hist_given) {
+            // the first pass's histogram was built with the scores: every CTA finds the bin from the
+            // 2048 global counts (two per thread, from the top digit down)
+            const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
+            const unsigned c0 = __ldcg(&a.sc->hist[0][d0]), c1 = __ldcg(&a.sc->hist[0][d1]);
+            unsigned tot;
+            const unsigned e = block_excl_scan(c0 + c1, s_warp, &tot);
+            if (e < krem && krem <= e + c0) {
+                s_pick[0] = static_cast<unsigned>(d0);
+                s_pick[1] = e;
+            } else if (e + c0 < krem && krem <= e + c0 + c1) {
+                s_pick[0] = static_cast<unsigned>(d1);
+                s_pick[1] = e + c0;
+            }
+            __syncthreads();
+            prefix |= s_pick[0] << shift;
+            pmask |= dmask << shift;
+            krem -= s_pick[1];
+            __syncthreads();
+            continue;
+        }
         for (int b = tid; b < nb; b += kSelectThreads) s_hist[b] = 0;
         __syncthreads();
 #pragma unroll
@@ -483,6 +501,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(
     for (int64_t i = a.D1 + static_cast<int64_t>(rank) * kSelectThreads + tid; i < a.N; i += gstride)
         a.out[a.D0 + a.kd + (i - a.D1)] = static_cast<int32_t>(i);
     cluster_barrier();  // this CTA's shared memory stays alive until every CTA has read it
+    // every CTA read the given first-pass histogram in pass 0: leave it zero for the next gate
+    if (a.hist_given && rank == 0)
+        for (int b = tid; b < 2048; b += kSelectThreads) a.sc->hist[0][b] = 0u;
 }
 
 // K_doc == 0 (only tokens outside the span) or K_doc >= N_doc (every token).
@@ -589,15 +610,21 @@ using namespace tg;
 // The select with keys from `scores`, or random keys from `seed` when scores is NULL.
 static tg_status select_impl(const float* scores, uint64_t seed, int64_t N, int64_t doc_begin, int64_t doc_end,
                              int64_t k_doc, int32_t* kept_idx, void* workspace, size_t workspace_bytes,
-                             void* stream) {
+                             void* stream, bool hist_given = false) {
     const int64_t K = tg_kept_count(N, doc_begin, doc_end, k_doc);
     if (K < 0) return TG_ERR_INVALID_ARG;
     if (N > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
-    if (K == 0) return TG_OK;
-    if (!kept_idx) return TG_ERR_INVALID_ARG;
     const int64_t n_doc = doc_end - doc_begin;
     const int64_t kd = k_doc < n_doc ? k_doc : n_doc;
     cudaStream_t st = as_stream(stream);
+    if (hist_given && (K == 0 || kd == 0 || kd == n_doc)) {
+        // no radix pass reads the gate's histogram: clear it here for the next gate
+        if (!workspace || workspace_bytes < tg_workspace_bytes(TG_OP_SELECT, N, 0, 0)) return TG_ERR_INVALID_ARG;
+        SelectScratch* sc = reinterpret_cast<SelectScratch*>(static_cast<char*>(workspace) + kWsHeader);
+        if (cudaMemsetAsync(&sc->hist[0][0], 0, sizeof(sc->hist[0]), st) != cudaSuccess) return TG_ERR_CUDA;
+    }
+    if (K == 0) return TG_OK;
+    if (!kept_idx) return TG_ERR_INVALID_ARG;
     if (kd == 0 || kd == n_doc) {
         const int64_t blocks = std::min<int64_t>((N + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
         select_trivial_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(N, doc_begin, doc_end,
@@ -617,6 +644,7 @@ static tg_status select_impl(const float* scores, uint64_t seed, int64_t N, int6
     a.out = kept_idx;
     a.sc = reinterpret_cast<SelectScratch*>(static_cast<char*>(workspace) + kWsHeader);
     a.status = status_word(workspace);
+    a.hist_given = hist_given ? 1 : 0;
     cudaError_t e;
     if (try_select_cluster(a, n_doc, st, &e)) return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;
 
@@ -647,6 +675,13 @@ extern "C" tg_status tg_topk_select(const float* scores, int64_t N, int64_t doc_
                                     void* stream) {
     if (!scores && tg_kept_count(N, doc_begin, doc_end, k_doc) > 0) return TG_ERR_INVALID_ARG;
     return select_impl(scores, 0, N, doc_begin, doc_end, k_doc, kept_idx, workspace, workspace_bytes, stream);
+}
+
+extern "C" tg_status tg_topk_select_after_gate(const float* scores, int64_t N, int64_t doc_begin, int64_t doc_end,
+                                               int64_t k_doc, int32_t* kept_idx, void* workspace,
+                                               size_t workspace_bytes, void* stream) {
+    if (!scores && tg_kept_count(N, doc_begin, doc_end, k_doc) > 0) return TG_ERR_INVALID_ARG;
+    return select_impl(scores, 0, N, doc_begin, doc_end, k_doc, kept_idx, workspace, workspace_bytes, stream, true);
 }
 
 extern "C" tg_status tg_debug_set_select_wait_limit(uint64_t ns) {
@@ -742,6 +777,7 @@ extern "C" tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int6
     a.sc = reinterpret_cast<SelectScratch*>(scratch + kWsHeader);
     a.status = reinterpret_cast<unsigned int*>(scratch);
     a.ept = static_cast<int>(ept);
+    a.hist_given = 0;
     cudaError_t e;
     if (ept <= 1)
         e = launch_select<1>(a, grid, st);

@@ -8,8 +8,9 @@ article, paragraph 事件详情; chathome.org article, sections TokenGate の学
 トークンプルーニングの仕組み and トークンゲート付きアテンションとは).
 
 Steps, in order, all on the caller's current CUDA stream:
-  gate     tg_gate_score            libtokengate (tcgen05 GEMM + fused epilogue)
-  select   tg_topk_select           libtokengate (radix select)
+  gate     tg_gate_score_for_select libtokengate (tcgen05 GEMM + fused epilogue, which also
+                                    counts the select's first radix pass)
+  select   tg_topk_select_after_gate libtokengate (radix select from that count)
   gather   tg_gather_compact        libtokengate (row copy)
   proj     tg_project_rope          libtokengate (tcgen05 GEMM of the kept rows with
                                     RoPE and V's fp16 copy in its epilogue)
@@ -92,36 +93,55 @@ class GatedPrefillLayer:
         self.v = self.qkv[:, (Hq + Hkv) * d_h:].view(K, Hkv, d_h)
         self.out = torch.empty(K, Hq, d_h, dtype=torch.bfloat16, device=dev)
 
+    def stage_calls(self, h: torch.Tensor):
+        """{step name: a call running that step alone on the layer's buffers}, in path order.  Each
+        step reads only what the steps before it wrote, so after one full pass any step may be run
+        again by itself (the benchmark times each step this way)."""
+        K = self.K
+
+        def gate():
+            # also counts the select's first radix pass in the workspace (the select below starts from it)
+            tg.tg_gate_score_for_select(h, self.W1, self.w2, self.scores, self.ws, self.doc_begin, self.doc_end,
+                                        b1=self.b1, b2=self.b2, rms_weight=self.rms_weight, eps=self.eps)
+
+        def select():
+            tg.tg_topk_select_after_gate(self.scores, self.doc_begin, self.doc_end, self.k_doc, self.kept[:K], self.ws)
+
+        def gather():
+            tg.tg_gather_compact(h, self.kept[:K], self.h_kept, self.pos[:K], scores=self.scores,
+                                 s_out=self.s_kept[:K])
+
+        def proj():
+            tg.tg_project_rope(self.h_kept, self.Wqkv, self.pos[:K], self.qkv, self.ws_proj, self.Hq, self.Hkv,
+                               self.d_h, base=self.rope_base, v16=self.v16)
+
+        def qkv():
+            torch.matmul(self.h_kept, self.WqkvT, out=self.qkv)
+
+        def rope():
+            tg.tg_rope_apply(self.q, self.k, self.pos[:K], self.rope_base)
+
+        def attn():
+            if self.fused:
+                tg.tg_gated_attention_f16v(self.q, self.k, self.v16, self.out, self.ws_attn,
+                                           s_kept=self.s_kept[:K], gain=self.gain, tau=self.tau)
+            else:
+                tg.tg_gated_attention(self.q, self.k, self.v, self.out, self.ws_attn, s_kept=self.s_kept[:K],
+                                      gain=self.gain, tau=self.tau)
+
+        calls = {"gate": gate, "select": select, "gather": gather, "proj": proj, "qkv": qkv, "rope": rope,
+                 "attn": attn}
+        return {name: calls[name] for name in self.stages}
+
     def run(self, h: torch.Tensor, mark: Optional[Callable[[str], None]] = None):
         """Runs the steps on device-resident h [N, d]; returns (out [K, Hq, d_h], kept [K]).
         `mark(name)` is called before each step (self.stages) and with "end" after the last."""
         m = mark or (lambda _n: None)
-        K = self.K
-        m("gate")
-        tg.tg_gate_score(h, self.W1, self.w2, self.scores, self.ws, b1=self.b1, b2=self.b2,
-                         rms_weight=self.rms_weight, eps=self.eps)
-        m("select")
-        tg.tg_topk_select(self.scores, self.doc_begin, self.doc_end, self.k_doc, self.kept[:K], self.ws)
-        m("gather")
-        tg.tg_gather_compact(h, self.kept[:K], self.h_kept, self.pos[:K], scores=self.scores,
-                             s_out=self.s_kept[:K])
-        if self.fused:
-            m("proj")
-            tg.tg_project_rope(self.h_kept, self.Wqkv, self.pos[:K], self.qkv, self.ws_proj, self.Hq, self.Hkv,
-                               self.d_h, base=self.rope_base, v16=self.v16)
-            m("attn")
-            tg.tg_gated_attention_f16v(self.q, self.k, self.v16, self.out, self.ws_attn, s_kept=self.s_kept[:K],
-                                       gain=self.gain, tau=self.tau)
-        else:
-            m("qkv")
-            torch.matmul(self.h_kept, self.WqkvT, out=self.qkv)
-            m("rope")
-            tg.tg_rope_apply(self.q, self.k, self.pos[:K], self.rope_base)
-            m("attn")
-            tg.tg_gated_attention(self.q, self.k, self.v, self.out, self.ws_attn, s_kept=self.s_kept[:K],
-                                  gain=self.gain, tau=self.tau)
+        for name, call in self.stage_calls(h).items():
+            m(name)
+            call()
         m("end")
-        return self.out, self.kept[:K]
+        return self.out, self.kept[:self.K]
 
     def run_host(self, h_host: torch.Tensor, h_dev: torch.Tensor, out_host: torch.Tensor,
                  kept_host: torch.Tensor):

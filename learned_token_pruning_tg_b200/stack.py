@@ -184,9 +184,10 @@ class PrunedPrefillStack:
             if prune and li == c.gate_layer:
                 # the gate on layer L's post-attention residual, then top-K and the gather
                 self.scores = torch.empty(c.N, dtype=torch.float32, device=self.dev)
-                tg.tg_gate_score(x, self.wts.W1, self.wts.w2, self.scores, self.ws_gate, eps=c.eps)
+                tg.tg_gate_score_for_select(x, self.wts.W1, self.wts.w2, self.scores, self.ws_gate, c.doc_begin,
+                                            c.doc_end, eps=c.eps)
                 self.kept = torch.empty(c.K, dtype=torch.int32, device=self.dev)
-                tg.tg_topk_select(self.scores, c.doc_begin, c.doc_end, c.k_doc, self.kept, self.ws_gate)
+                tg.tg_topk_select_after_gate(self.scores, c.doc_begin, c.doc_end, c.k_doc, self.kept, self.ws_gate)
                 xk = torch.empty(c.K, c.d, dtype=torch.bfloat16, device=self.dev)
                 pk = torch.empty(c.K, dtype=torch.int32, device=self.dev)
                 s_kept = torch.empty(c.K, dtype=torch.float32, device=self.dev)

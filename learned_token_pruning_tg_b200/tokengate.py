@@ -49,6 +49,9 @@ def lib() -> ctypes.CDLL:
         L.tg_workspace_bytes.restype = sz
         L.tg_gate_score.argtypes = [vp, i64, i32, i64, vp, f32, vp, vp, vp, f32, i32, vp, vp, sz, vp]
         L.tg_topk_select.argtypes = [vp, i64, i64, i64, i64, vp, vp, sz, vp]
+        L.tg_gate_score_for_select.argtypes = [vp, i64, i32, i64, vp, f32, vp, vp, vp, f32, i32, vp, i64, i64, vp, sz,
+                                               vp]
+        L.tg_topk_select_after_gate.argtypes = [vp, i64, i64, i64, i64, vp, vp, sz, vp]
         L.tg_topk_select_noalloc.argtypes = [vp, i64, i64, i64, i64, vp, vp]
         L.tg_topk_select_noalloc_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
         L.tg_random_select.argtypes = [i64, i64, i64, i64, ctypes.c_uint64, vp, vp, sz, vp]
@@ -64,7 +67,7 @@ def lib() -> ctypes.CDLL:
                                                   vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.tg_debug_set_select_wait_limit.argtypes = [ctypes.c_uint64]
         L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
-        for fn in ("tg_gate_score", "tg_topk_select", "tg_topk_select_noalloc", "tg_random_select", "tg_gather_compact",
+        for fn in ("tg_gate_score", "tg_gate_score_for_select", "tg_topk_select", "tg_topk_select_after_gate", "tg_topk_select_noalloc", "tg_random_select", "tg_gather_compact",
                    "tg_rope_apply",
                    "tg_gated_attention", "tg_gated_attention_f16v", "tg_project_rope",
                    "tg_gated_attention_backward", "tg_gated_decode", "tg_debug_set_select_wait_limit", "tg_device_status"):
@@ -149,6 +152,49 @@ def tg_gate_score(h, W1, w2, scores, workspace, b1=None, b2: float = 0.0, rms_we
         _ptr(h), N, d, ld_h, _ptr(rms_weight), eps, _ptr(W1), _ptr(b1), _ptr(w2), b2, d_g,
         _ptr(scores), _ptr(workspace), workspace.numel(), _stream(stream)))
     return scores
+
+
+def _gate_args(h, W1, w2, scores, b1, rms_weight):
+    _req(h, "h", torch.bfloat16, 2)
+    _req(W1, "W1", torch.bfloat16, 2)
+    _req(w2, "w2", torch.float32, 1)
+    _req(scores, "scores", torch.float32, 1)
+    _req(b1, "b1", torch.float32, 1)
+    _req(rms_weight, "rms_weight", torch.bfloat16, 1)
+    N, d = h.shape
+    d_g = W1.shape[0]
+    if h.stride(1) != 1 or not W1.is_contiguous() or not w2.is_contiguous() or not scores.is_contiguous():
+        raise ValueError("h rows, W1, w2 and scores must be dense")
+    if W1.shape[1] != d or w2.shape[0] != d_g or scores.shape[0] != N:
+        raise ValueError("shape mismatch")
+    return N, d, (h.stride(0) if N > 1 else d), d_g
+
+
+def tg_gate_score_for_select(h, W1, w2, scores, workspace, doc_begin: int, doc_end: int, b1=None, b2: float = 0.0,
+                             rms_weight=None, eps: float = 1e-6, stream=None):
+    """tg_gate_score that also leaves the select's first radix pass over [doc_begin, doc_end) in the
+    workspace, for a tg_topk_select_after_gate on the same workspace right after it."""
+    N, d, ld_h, d_g = _gate_args(h, W1, w2, scores, b1, rms_weight)
+    _check("tg_gate_score_for_select", lib().tg_gate_score_for_select(
+        _ptr(h), N, d, ld_h, _ptr(rms_weight), eps, _ptr(W1), _ptr(b1), _ptr(w2), b2, d_g,
+        _ptr(scores), doc_begin, doc_end, _ptr(workspace), workspace.numel(), _stream(stream)))
+    return scores
+
+
+def tg_topk_select_after_gate(scores, doc_begin: int, doc_end: int, k_doc: int, kept_idx, workspace, stream=None):
+    """tg_topk_select starting from the first radix pass tg_gate_score_for_select left in the workspace."""
+    _req(scores, "scores", torch.float32, 1)
+    _req(kept_idx, "kept_idx", torch.int32, 1)
+    N = scores.shape[0]
+    K = tg_kept_count(N, doc_begin, doc_end, k_doc)
+    if K < 0:
+        raise TokenGateError("tg_topk_select_after_gate", TG_ERR_INVALID_ARG)
+    if kept_idx.numel() < K or not scores.is_contiguous() or not kept_idx.is_contiguous():
+        raise ValueError("kept_idx too small or not contiguous")
+    _check("tg_topk_select_after_gate", lib().tg_topk_select_after_gate(
+        _ptr(scores), N, doc_begin, doc_end, k_doc, _ptr(kept_idx), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return kept_idx
 
 
 def tg_topk_select(scores, doc_begin: int, doc_end: int, k_doc: int, kept_idx, workspace, stream=None):

@@ -128,3 +128,39 @@ def test_gate_repeatable_bit_exact():
     for _ in range(7):
         assert np.array_equal(_gpu_scores(gi), first)
     _check(first, _oracle_scores(gi))
+
+
+@pytest.mark.parametrize("N,d,d_g,db,de,k", [
+    (1024, 256, 64, 0, 960, 192),              # tiny workload's shape
+    (16384, 2048, 256, 0, 16000, 1024),        # 16k (CTA-pair gate, one-cluster select)
+    (131072, 2048, 256, 0, 130560, 4096),      # 128k
+    (70001, 512, 128, 333, 69000, 12345),      # ragged span inside the prompt
+    (300000, 64, 256, 1000, 299000, 50000),    # a span beyond one cluster: the cooperative select
+    (5000, 128, 64, 0, 5000, 0),               # budget 0: nothing selected, the count still cleared
+    (5000, 128, 64, 100, 4900, 10000),         # budget above the span: every token kept
+])
+def test_gate_and_select_pair(N, d, d_g, db, de, k):
+    # tg_gate_score_for_select gives tg_gate_score's scores bit for bit and leaves the select's first
+    # radix pass in the workspace; tg_topk_select_after_gate then gives the oracle's selection on those
+    # scores and leaves the count at zero (three pairs in a row on one workspace).
+    w = synth.scaled(synth.L16K, N=N, doc_begin=db, doc_end=de, d=d, d_g=d_g, k_doc=k, n_scaled=min(8, de - db),
+                     seed=N + d_g)
+    gi = synth.gate_inputs(w)
+    h, W1, w2 = gi.h.to(torch.bfloat16).cuda(), gi.W1.to(torch.bfloat16).cuda(), gi.w2.cuda()
+    ws = tg.new_workspace(N, d, d_g)
+    plain = torch.empty(N, device="cuda")
+    tg.tg_gate_score(h, W1, w2, plain, ws)
+    K = tg.tg_kept_count(N, db, de, k)
+    for _ in range(3):
+        scores = torch.full((N,), float("nan"), device="cuda")
+        kept = torch.full((max(K, 1),), -1, dtype=torch.int32, device="cuda")
+        tg.tg_gate_score_for_select(h, W1, w2, scores, ws, db, de)
+        tg.tg_topk_select_after_gate(scores, db, de, k, kept[:K], ws)
+        torch.cuda.synchronize()
+        assert tg.tg_device_status(ws) == 0
+        assert torch.equal(scores.view(torch.int32), plain.view(torch.int32))
+        s_np = scores.cpu().numpy()
+        assert np.array_equal(kept[:K].cpu().numpy(), oracle.topk_select(s_np, db, de, k))
+        # the first-pass count (2048 words after the status header and the barrier words) is zero again
+        hist0 = ws[256 + 256: 256 + 256 + 2048 * 4].view(torch.int32)
+        assert int(hist0.abs().sum().item()) == 0
