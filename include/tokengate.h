@@ -351,19 +351,22 @@ tg_status tg_gated_attention_backward(const tg_bf16* q, int64_t ld_q, const tg_b
  * the GEMM epilogue (layers above the gate see only the kept tokens, rotated
  * at their original positions; aiproducthub.cn article, paragraph 事件详情):
  *   qkv[r, :] = x[r, :] W^T, then for every query and key head the
- *   rotate-half pairs (t, t + d_h/2) turned by pos[r] * base^(-2t/d_h)
- *   (angles in fp64, as tg_rope_apply), from the fp32 accumulators;
+ *   rotate-half pairs (t, t + d_h/2) turned by pos[r] * base^(-2t/d_h),
+ *   from the fp32 accumulators (the angle formed and reduced modulo 2 pi in
+ *   fp64, its cos / sin in fp32: within 6e-7 of tg_rope_apply's);
  *   value heads are stored as they are, and also in fp16 into v16.
  * x: [K, d] bf16, row stride ld_x (multiple of 8).  W: [(Hq + 2 Hkv) d_h, d]
  * bf16 (query heads, then key heads, then value heads, as an nn.Linear
  * weight).  pos: [K] int32.  qkv: [K, (Hq + 2 Hkv) d_h] bf16, row stride
  * ld_qkv (multiple of 8).  v16: [K, Hkv d_h] fp16 (uint16 bit patterns)
  * dense, or NULL.  workspace: tg_workspace_bytes(TG_OP_PROJECT, K, d_h, 0)
- * bytes (the cos / sin table of the K rows).
+ * bytes (the status word).
  * Supported: d a multiple of 64; (Hq + 2 Hkv) d_h a multiple of 256; d_h in
- * {64, 128}; x, W, qkv, v16 16-byte aligned.  Two launches: the cos / sin
- * table, then a persistent tcgen05 GEMM (128 x 256 tiles, TMA-staged
- * operands, TMEM accumulators double-buffered against the epilogue).
+ * {64, 128}; x, W, qkv, v16 16-byte aligned.  One launch: a persistent
+ * tcgen05 GEMM over CTA pairs (256 x 256 tiles, each CTA of a pair loading
+ * its own rows and half of W's tile by TMA, TMEM accumulators double-buffered
+ * against the epilogue), or over single CTAs (128 x 256 tiles) where a pair
+ * cannot be resident.
  * Waits are bounded (TG_STATUS_PROJECT_TIMEOUT).  A value head element above
  * fp16's range (|v| > 65504) written into v16 sets TG_STATUS_V_RANGE. */
 tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int64_t ld_x, const tg_bf16* W, int32_t Hq,

@@ -12,9 +12,11 @@
 //   q/k heads: rotate-half pairs (t, t + d_h/2) at pos[r], from the fp32
 //              accumulator (one bf16 rounding instead of two)
 //   v heads:   bf16 into qkv and, when asked, fp16 into v16
-// Angles are formed in fp64 exactly as tg_rope_apply forms them (a small
-// kernel writes the cos / sin table of every kept row into the workspace, from
-// frequencies the host forms in fp64).
+// Angles in the epilogue: pos[r] * base^(-2t / d_h) in fp64 (the frequencies
+// formed on the host in fp64), reduced modulo 2 pi in fp64, then cos and sin of
+// the reduced angle (|x| <= pi) in fp32 -- within 6e-7 of the fp64 values (the fast
+// sine and cosine, 2^-21.4 on [-pi, pi], and the fp32 rounding of the angle), far
+// below the bf16 rounding of the result.
 //
 // Kernel (persistent, one CTA per SM, 8 warps): tiles of 128 rows x 256
 // output columns, row-tile-major so the CTAs working at one time share the
@@ -55,13 +57,13 @@ static_assert(kStageA % 1024 == 0 && kStage % 1024 == 0 && kOffBar % 8 == 0 && k
               "projection shared-memory layout");
 
 struct Args {
+    double inv_freq[64];  // base^(-2t / d_h), t < d_h / 2, formed on the host in fp64
     int64_t K;
     int d;
     int Hq, Hkv, D;
     int num_col_tiles;
     int64_t num_tiles;
-    const float* cos_t;   // [K, D/2]
-    const float* sin_t;   // [K, D/2]
+    const int32_t* pos;   // [K] original positions
     __nv_bfloat16* qkv;
     int64_t ld_qkv;
     __half* v16;          // [K, Hkv D] or null
@@ -73,25 +75,14 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// The rotary frequencies base^(-2t / d_h), t < d_h / 2, formed on the host in fp64.
-struct InvFreq {
-    double v[64];
-};
-
-// cos / sin of pos[r] * inv_freq[t] in fp64, rounded to fp32; one (row, t) per thread.
-__global__ void __launch_bounds__(256) rope_table_kernel(const int32_t* __restrict__ pos, int64_t K, int half,
-                                                         const __grid_constant__ InvFreq f, float* __restrict__ cos_t,
-                                                         float* __restrict__ sin_t) {
-    const int64_t n = K * half;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * 256) {
-        const int64_t r = i / half;
-        const int t = static_cast<int>(i - r * half);
-        double s, c;
-        sincos(static_cast<double>(__ldg(pos + r)) * f.v[t], &s, &c);
-        cos_t[i] = static_cast<float>(c);
-        sin_t[i] = static_cast<float>(s);
-    }
+// cos / sin of pos * inv_freq: the angle and its reduction modulo 2 pi in fp64, the cos and sin of
+// the reduced angle in fp32 (|angle| <= pi there).
+__device__ __forceinline__ void rope_cos_sin(double p, double inv_freq, float* c, float* s) {
+    constexpr double kTwoPi = 6.283185307179586;
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    const double ang = p * inv_freq;
+    const double r = fma(-rint(ang * kInvTwoPi), kTwoPi, ang);
+    __sincosf(static_cast<float>(r), s, c);
 }
 
 // One output tile's epilogue for the thread that owns TMEM lane `row` (row
@@ -112,13 +103,13 @@ __device__ __forceinline__ void epilogue_tile(const Args& a, uint32_t taddr, int
                 tmem_ld32(taddr + c_head + half + t0, x2);
                 tmem_ld_wait();
                 if (live) {
-                    const float4* cp = reinterpret_cast<const float4*>(a.cos_t + grow * half + t0);
-                    const float4* sp = reinterpret_cast<const float4*>(a.sin_t + grow * half + t0);
+                    const double p = static_cast<double>(__ldg(a.pos + grow));
                     uint32_t o1[16], o2[16];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float4 c4 = cp[i], s4 = sp[i];
-                        const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+                        float cc[4], ss[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) rope_cos_sin(p, a.inv_freq[t0 + 4 * i + e], &cc[e], &ss[e]);
                         float r1[4], r2[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -523,7 +514,7 @@ static bool pair_kernel_available() {
 
 size_t ws_project_bytes(int64_t K, int32_t d_h) {
     if (K < 0 || (d_h != 64 && d_h != 128)) return 0;
-    return kWsHeader + ((static_cast<size_t>(K) * d_h * 4 + 255) / 256) * 256;  // cos and sin, K x d_h/2 each
+    return kWsHeader;  // the status word
 }
 
 }  // namespace tg
@@ -546,16 +537,6 @@ extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int
         return TG_ERR_INVALID_ARG;
     if (workspace_bytes < ws_project_bytes(K, d_h)) return TG_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
-    float* cos_t = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeader);
-    float* sin_t = cos_t + K * (d_h / 2);
-    {
-        const int64_t blocks = std::min<int64_t>((K * (d_h / 2) + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
-        proj::InvFreq f;
-        for (int t = 0; t < d_h / 2; ++t)
-            f.v[t] = std::pow(base, -2.0 * static_cast<double>(t) / static_cast<double>(d_h));
-        proj::rope_table_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(pos, K, d_h / 2, f, cos_t, sin_t);
-        if (launch_status() != TG_OK) return TG_ERR_CUDA;
-    }
     CUtensorMap mx, mw;
     const uint64_t xd[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(K)};
     const uint64_t xs[1] = {static_cast<uint64_t>(ld_x) * 2};
@@ -573,8 +554,9 @@ extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int
     a.D = d_h;
     a.num_col_tiles = static_cast<int>(cols / proj::kBN);
     a.num_tiles = ((K + proj::kBM - 1) / proj::kBM) * a.num_col_tiles;
-    a.cos_t = cos_t;
-    a.sin_t = sin_t;
+    a.pos = pos;
+    for (int t = 0; t < d_h / 2; ++t)
+        a.inv_freq[t] = std::pow(base, -2.0 * static_cast<double>(t) / static_cast<double>(d_h));
     a.qkv = reinterpret_cast<__nv_bfloat16*>(qkv);
     a.ld_qkv = ld_qkv;
     a.v16 = reinterpret_cast<__half*>(v16);

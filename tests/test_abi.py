@@ -174,7 +174,7 @@ def test_project_rope_workspace_and_argument_errors(lib):
     vp = ctypes.c_void_p
     INV, UNS = tg.TG_ERR_INVALID_ARG, tg.TG_ERR_UNSUPPORTED
     ws = tg.tg_workspace_bytes(tg.TG_OP_PROJECT, 4608, 128)
-    assert ws >= 256 + 4608 * 128 * 4 and ws % 256 == 0       # cos and sin of K rows x d_h / 2
+    assert ws >= 256 and ws % 256 == 0                        # the status word
     assert tg.tg_workspace_bytes(tg.TG_OP_PROJECT, 4608, 96) == 0
 
     def proj(x=16, K=300, d=2048, ldx=2048, Hq=16, Hkv=8, d_h=128, base=1e6, ldo=4096, v16=None, ws_bytes=ws):
@@ -189,5 +189,5 @@ def test_project_rope_workspace_and_argument_errors(lib):
     assert proj(ldo=4092) == INV                    # output stride not a multiple of 8
     assert proj(ldo=2048) == INV                    # output stride shorter than a row
     assert proj(v16=40) == INV                      # misaligned fp16 copy
-    assert proj(ws_bytes=1024) == INV
+    assert proj(ws_bytes=128) == INV                 # shorter than the status word
     assert proj(K=0) == tg.TG_OK

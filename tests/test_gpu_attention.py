@@ -125,6 +125,16 @@ def test_attention_128k_workload_sampled_rows():
     check(d, rows=rows)
 
 
+def test_attention_dense_64k_layer_sampled_rows():
+    # The stack's dense layers run the kernel over all 65,536 tokens with no bias and tau = 1 (plain
+    # causal attention); sampled rows across the whole range, the last ones included.
+    d = synth.qkv(65536, 16, 8, 128, seed=65536)
+    d.gain.zero_()
+    d.tau = 1.0
+    rows = np.unique(np.concatenate([np.arange(0, 65536, 1021), np.arange(65536 - 24, 65536)]))
+    check(d, rows=rows, use_bias=False)
+
+
 def test_attention_large_k_sampled_rows():
     d = synth.qkv(16896, 16, 8, 128, seed=3204, n_pos=32768)
     rows = np.unique(np.concatenate([np.arange(0, 16896, 131), np.arange(16896 - 40, 16896)]))
