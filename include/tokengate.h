@@ -87,6 +87,9 @@ typedef enum {
  * into an fp16 copy of V (tg_gated_attention, tg_project_rope); the outputs
  * that read it are not the specified values. */
 #define TG_STATUS_V_RANGE 0x40u
+/* Not a timeout: a row index outside [0, N) was given to
+ * tg_project_rope_gather; that row was read from row 0 instead. */
+#define TG_STATUS_INDEX_RANGE 0x80u
 #define TG_STATUS_TIMEOUT_BITS 0x3fu
 
 /* Static description of a status code.  Never NULL. */
@@ -175,6 +178,16 @@ tg_status tg_gate_score_for_select(const tg_bf16* h, int64_t N, int32_t d, int64
 tg_status tg_topk_select_after_gate(const float* scores, int64_t N, int64_t doc_begin,
                                     int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* tg_topk_select_after_gate that also writes the kept tokens' scores:
+ * s_kept[i] = scores[kept_idx[i]] ([tg_kept_count(...)] fp32, in the order of
+ * kept_idx) -- the compacted scores the attention's key bias reads, so no
+ * separate compaction pass is needed for them.  Same call order, workspace
+ * and errors as tg_topk_select_after_gate; s_kept must not be NULL when the
+ * kept count is positive. */
+tg_status tg_topk_select_after_gate_kept_scores(const float* scores, int64_t N, int64_t doc_begin, int64_t doc_end,
+                                                int64_t k_doc, int32_t* kept_idx, float* s_kept, void* workspace,
+                                                size_t workspace_bytes, void* stream);
 
 /* Top-K selection that allocates nothing and takes no workspace.
  * There is no counterpart on the TokenGate pages: this is a calling-convention
@@ -373,6 +386,23 @@ tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int64_t ld_x, 
                           int32_t Hkv, int32_t d_h, const int32_t* pos, double base, tg_bf16* qkv, int64_t ld_qkv,
                           uint16_t* v16, void* workspace, size_t workspace_bytes, void* stream);
 
+/* tg_project_rope whose rows are gathered from h on the way into the GEMM
+ * (the compaction of the kept rows fused into the projection's operand
+ * loads): x[r, :] = h[rows[r], :], fetched by TMA gather4 copies (four rows
+ * of 128 bytes per copy) straight into the tensor-core operand tiles, so the
+ * compacted rows are never written out.
+ * h: [N, d] bf16, row stride ld_h (multiple of 8), 16-byte aligned.
+ * rows: [K] int32 indices into h (the kept indices from the select).  An
+ * index outside [0, N) is not followed: row 0 is read in its place and
+ * TG_STATUS_INDEX_RANGE is set in the workspace's status word.
+ * Every other argument, the outputs, the workspace and the limits are those
+ * of tg_project_rope (pos: the rows' original positions; pass `rows` itself
+ * when the positions are the indices). */
+tg_status tg_project_rope_gather(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h, const int32_t* rows, int64_t K,
+                                 const tg_bf16* W, int32_t Hq, int32_t Hkv, int32_t d_h, const int32_t* pos,
+                                 double base, tg_bf16* qkv, int64_t ld_qkv, uint16_t* v16, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 /* Test hook (fault injection without a fault): sets the time limit of the
  * grid barrier inside tg_topk_select, tg_topk_select_noalloc and
  * tg_random_select on the current device to `ns` nanoseconds of %globaltimer
@@ -387,7 +417,7 @@ tg_status tg_debug_set_select_wait_limit(uint64_t ns);
 /* Reads the workspace's status word after synchronizing `stream`.
  * *status_word receives the raw TG_STATUS_* bits (may be NULL).
  * Returns TG_ERR_TIMEOUT if a timeout bit is set, else TG_ERR_RANGE if
- * TG_STATUS_V_RANGE is set, TG_OK otherwise. */
+ * TG_STATUS_V_RANGE or TG_STATUS_INDEX_RANGE is set, TG_OK otherwise. */
 tg_status tg_device_status(const void* workspace, uint32_t* status_word, void* stream);
 
 #ifdef __cplusplus

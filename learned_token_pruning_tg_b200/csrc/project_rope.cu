@@ -64,11 +64,31 @@ struct Args {
     int num_col_tiles;
     int64_t num_tiles;
     const int32_t* pos;   // [K] original positions
+    const int32_t* rows;  // [K] rows of h to gather (tg_project_rope_gather), or null: x is dense
+    int64_t n_rows;       // rows of h (the valid range of `rows`)
     __nv_bfloat16* qkv;
     int64_t ld_qkv;
     __half* v16;          // [K, Hkv D] or null
     unsigned int* status;
 };
+
+// The 4 rows of h that lane `lane` of the producer warp gathers for tile rows [r0, r0 + 4): indices
+// outside [0, n_rows) are replaced by row 0 and flagged; rows past K (the last tile's tail, whose
+// outputs are not stored) read row 0.
+__device__ __forceinline__ void gather_rows4(const Args& a, int64_t r0, int (&g)[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int v = 0;
+        if (r0 + i < a.K) {
+            v = __ldg(a.rows + r0 + i);
+            if (v < 0 || static_cast<int64_t>(v) >= a.n_rows) {
+                atomicOr(a.status, TG_STATUS_INDEX_RANGE);
+                v = 0;
+            }
+        }
+        g[i] = v;
+    }
+}
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
@@ -205,7 +225,48 @@ project_rope_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == 0 && a.rows) {
+        // ------------------------------------------------------------ TMA producer, rows gathered from h
+        // lane l fetches tile rows 4l .. 4l + 3 with one gather4 copy per 64-column step
+        int s = 0;
+        uint32_t ph = 0;
+        int last_ph[kStages];
+        for (int i = 0; i < kStages; ++i) last_ph[i] = -1;
+        for (int64_t t = blockIdx.x; t < a.num_tiles; t += gridDim.x) {
+            if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+            const int rt = static_cast<int>(t / a.num_col_tiles);
+            const int ct = static_cast<int>(t % a.num_col_tiles);
+            int g[4];
+            gather_rows4(a, static_cast<int64_t>(rt) * kBM + lane * 4, g);
+            bool ok = true;
+            for (int kb = 0; kb < kb_per_tile; ++kb) {
+                if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT);
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sa = smem + s * kStage;
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], kStage);
+                __syncwarp();
+                tma_gather4(sa + lane * 512, &tmap_x, &full[s], kb * kBK, g[0], g[1], g[2], g[3], kEvictLast);
+                if (lane == 0) tma_load_2d(sa + kStageA, &tmap_w, &full[s], kb * kBK, ct * kBN, kEvictLast);
+                last_ph[s] = static_cast<int>(ph);
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+            if (!ok) break;
+        }
+        // every issued copy lands before shared memory is released (matters on abort only)
+        if (lane == 0) {
+            volatile int no_abort = 0;
+            for (int i = 0; i < kStages; ++i)
+                if (last_ph[i] >= 0)
+                    mbar_wait(&full[i], static_cast<uint32_t>(last_ph[i]), &no_abort, a.status,
+                              TG_STATUS_PROJECT_TIMEOUT);
+        }
+    } else if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int s = 0;
@@ -373,7 +434,50 @@ project_rope_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __gri
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == 0 && a.rows) {
+        // ------------------------------------------------------------ TMA producer (both CTAs), rows gathered
+        // lane l fetches this CTA's tile rows 4l .. 4l + 3 with one gather4 copy per 64-column step
+        int s = 0;
+        uint32_t ph = 0;
+        int last_ph[kPairStages];
+        for (int i = 0; i < kPairStages; ++i) last_ph[i] = -1;
+        for (int64_t t = pair; t < a.num_tiles; t += num_pairs) {
+            if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+            const int rt = static_cast<int>(t / a.num_col_tiles);
+            const int ct = static_cast<int>(t % a.num_col_tiles);
+            int g[4];
+            gather_rows4(a, static_cast<int64_t>(rt) * 2 * kBM + static_cast<int64_t>(rank) * kBM + lane * 4, g);
+            bool ok = true;
+            for (int kb = 0; kb < kb_per_tile; ++kb) {
+                if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, TG_STATUS_PROJECT_TIMEOUT);
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sa = smem + s * kPairStage;
+                if (leader && lane == 0) mbar_arrive_expect_tx(&full[s], 2 * kPairStage);
+                __syncwarp();
+                const uint32_t fb = cluster_addr(&full[s], 0);
+                tma_gather4_pair(sa + lane * 512, &tmap_x, fb, kb * kBK, g[0], g[1], g[2], g[3], kEvictLast);
+                if (lane == 0)
+                    tma_load_2d_pair(sa + kPairStageA, &tmap_w, fb, kb * kBK,
+                                     ct * kBN + static_cast<int>(rank) * (kBN / 2), kEvictLast);
+                last_ph[s] = static_cast<int>(ph);
+                if (++s == kPairStages) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+            if (!ok) break;
+        }
+        if (lane == 0 && *abort_flag && leader) {
+            volatile int no_abort = 0;
+            for (int i = 0; i < kPairStages; ++i)
+                if (last_ph[i] >= 0)
+                    mbar_wait_cluster(&full[i], static_cast<uint32_t>(last_ph[i]), &no_abort, a.status,
+                                      TG_STATUS_PROJECT_TIMEOUT);
+        }
+    } else if (warp == 0) {
         // ------------------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             int s = 0;
@@ -521,10 +625,11 @@ size_t ws_project_bytes(int64_t K, int32_t d_h) {
 
 using namespace tg;
 
-extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int64_t ld_x, const tg_bf16* W,
-                                     int32_t Hq, int32_t Hkv, int32_t d_h, const int32_t* pos, double base,
-                                     tg_bf16* qkv, int64_t ld_qkv, uint16_t* v16, void* workspace,
-                                     size_t workspace_bytes, void* stream) {
+// x: [K, d] dense rows (rows == null), or h: [n_rows, d] with x[r] = h[rows[r]].
+static tg_status project_impl(const tg_bf16* x, int64_t n_rows, const int32_t* rows, int64_t K, int32_t d,
+                              int64_t ld_x, const tg_bf16* W, int32_t Hq, int32_t Hkv, int32_t d_h,
+                              const int32_t* pos, double base, tg_bf16* qkv, int64_t ld_qkv, uint16_t* v16,
+                              void* workspace, size_t workspace_bytes, void* stream) {
     if (K < 0 || d <= 0 || Hq <= 0 || Hkv <= 0 || ld_x < d || !(base > 0.0)) return TG_ERR_INVALID_ARG;
     if (d_h != 64 && d_h != 128) return TG_ERR_UNSUPPORTED;
     const int64_t cols = static_cast<int64_t>(Hq + 2 * Hkv) * d_h;
@@ -538,9 +643,9 @@ extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int
     if (workspace_bytes < ws_project_bytes(K, d_h)) return TG_ERR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     CUtensorMap mx, mw;
-    const uint64_t xd[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(K)};
+    const uint64_t xd[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows ? n_rows : K)};
     const uint64_t xs[1] = {static_cast<uint64_t>(ld_x) * 2};
-    const uint32_t xb[2] = {proj::kBK, proj::kBM};
+    const uint32_t xb[2] = {proj::kBK, rows ? 1u : static_cast<uint32_t>(proj::kBM)};  // gather4: one-row boxes
     const uint64_t wd[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(cols)};
     const uint64_t wsd[1] = {static_cast<uint64_t>(d) * 2};
     const uint32_t wb[2] = {proj::kBK, proj::kBN};
@@ -555,6 +660,8 @@ extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int
     a.num_col_tiles = static_cast<int>(cols / proj::kBN);
     a.num_tiles = ((K + proj::kBM - 1) / proj::kBM) * a.num_col_tiles;
     a.pos = pos;
+    a.rows = rows;
+    a.n_rows = n_rows;
     for (int t = 0; t < d_h / 2; ++t)
         a.inv_freq[t] = std::pow(base, -2.0 * static_cast<double>(t) / static_cast<double>(d_h));
     a.qkv = reinterpret_cast<__nv_bfloat16*>(qkv);
@@ -589,4 +696,23 @@ extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int
     const int grid = static_cast<int>(std::min<int64_t>(a.num_tiles, num_sms()));
     kern<<<grid, proj::kThreads, proj::kSmem, st>>>(mx, mw, a);
     return launch_status();
+}
+
+extern "C" tg_status tg_project_rope(const tg_bf16* x, int64_t K, int32_t d, int64_t ld_x, const tg_bf16* W,
+                                     int32_t Hq, int32_t Hkv, int32_t d_h, const int32_t* pos, double base,
+                                     tg_bf16* qkv, int64_t ld_qkv, uint16_t* v16, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    return project_impl(x, K, nullptr, K, d, ld_x, W, Hq, Hkv, d_h, pos, base, qkv, ld_qkv, v16, workspace,
+                        workspace_bytes, stream);
+}
+
+extern "C" tg_status tg_project_rope_gather(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
+                                            const int32_t* rows, int64_t K, const tg_bf16* W, int32_t Hq,
+                                            int32_t Hkv, int32_t d_h, const int32_t* pos, double base,
+                                            tg_bf16* qkv, int64_t ld_qkv, uint16_t* v16, void* workspace,
+                                            size_t workspace_bytes, void* stream) {
+    if (N < 0 || N > 0x7fffffffLL) return N < 0 ? TG_ERR_INVALID_ARG : TG_ERR_UNSUPPORTED;
+    if (K > 0 && (N == 0 || !rows)) return TG_ERR_INVALID_ARG;
+    return project_impl(h, N, rows, K, d, ld_h, W, Hq, Hkv, d_h, pos, base, qkv, ld_qkv, v16, workspace,
+                        workspace_bytes, stream);
 }

@@ -29,7 +29,7 @@ extern "C" const char* tg_status_string(tg_status s) {
         case TG_ERR_UNSUPPORTED: return "unsupported shape";
         case TG_ERR_CUDA: return "CUDA launch or runtime error";
         case TG_ERR_TIMEOUT: return "device wait timed out";
-        case TG_ERR_RANGE: return "a value of V beyond fp16's range (|v| > 65504)";
+        case TG_ERR_RANGE: return "a value out of range (V beyond fp16's range, or a row index outside [0, N))";
     }
     return "unknown status";
 }
@@ -66,5 +66,5 @@ extern "C" tg_status tg_device_status(const void* workspace, uint32_t* status_wo
     if (cudaStreamSynchronize(st) != cudaSuccess) return TG_ERR_CUDA;
     if (status_word_out) *status_word_out = w;
     if (w & TG_STATUS_TIMEOUT_BITS) return TG_ERR_TIMEOUT;
-    return (w & TG_STATUS_V_RANGE) ? TG_ERR_RANGE : TG_OK;
+    return (w & (TG_STATUS_V_RANGE | TG_STATUS_INDEX_RANGE)) ? TG_ERR_RANGE : TG_OK;
 }

@@ -355,6 +355,26 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap, ui
         "l"(tmap), "r"(c0), "r"(c1), "r"(bar_cluster_addr), "l"(cache_hint)
         : "memory");
 }
+// Four rows r0..r3 of a 2D tensor (a box one row high and 64 bf16 wide; x a
+// multiple of 64) into 4 consecutive 128-byte rows of shared memory, swizzled
+// by their shared-memory address as a tiled load would place them.
+__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, uint64_t* bar, int x, int r0, int r1, int r2,
+                                            int r3, uint64_t cache_hint) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar)), "l"(cache_hint)
+        : "memory");
+}
+// The same for a CTA of a pair, completing on the even CTA's barrier (cluster address).
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const void* tmap, uint32_t bar_cluster_addr, int x, int r0,
+                                                 int r1, int r2, int r3, uint64_t cache_hint) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar_cluster_addr), "l"(cache_hint)
+        : "memory");
+}
 // TMEM allocation for a CTA pair: one warp of EACH CTA executes it; both get the same columns.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),

@@ -123,11 +123,18 @@ struct SelectArgs {
     int64_t N, D0, D1;
     unsigned int kd;   // document tokens kept, 0 < kd < n_doc
     int32_t* out;
+    float* s_out;      // when non-null: the kept tokens' scores, in the order of `out`
     SelectScratch* sc;
     unsigned int* status;
     int ept;           // keys per thread actually used (<= EPT)
     int hist_given;    // the first pass's histogram is already in sc->hist[0] (written with the scores)
 };
+
+// Token i goes to slot p of the kept list (and its score beside it when asked).
+__device__ __forceinline__ void keep_at(const SelectArgs& a, int64_t p, int64_t i) {
+    a.out[p] = static_cast<int32_t>(i);
+    if (a.s_out) a.s_out[p] = __ldg(a.scores + i);
+}
 
 template <int EPT>
 __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const SelectArgs a) {
@@ -245,9 +252,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const Se
             const unsigned g_before = run_g + (ex & 0xffffu);
             const unsigned e_before = run_e + (ex >> 16);
             if (fg)
-                a.out[a.D0 + g_before + min(e_before, krem)] = static_cast<int32_t>(i);
+                keep_at(a, a.D0 + g_before + min(e_before, krem), i);
             else if (fe && e_before < krem)
-                a.out[a.D0 + g_before + e_before] = static_cast<int32_t>(i);
+                keep_at(a, a.D0 + g_before + e_before, i);
             run_g += t2 & 0xffffu;
             run_e += t2 >> 16;
         }
@@ -256,9 +263,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const Se
     // Tokens outside the span are always kept: [0, D0) first, [D1, N) after the kept document tokens.
     const int64_t gstride = static_cast<int64_t>(nblocks) * kSelectThreads;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kSelectThreads + tid; i < a.D0; i += gstride)
-        a.out[i] = static_cast<int32_t>(i);
+        keep_at(a, i, i);
     for (int64_t i = a.D1 + static_cast<int64_t>(blockIdx.x) * kSelectThreads + tid; i < a.N; i += gstride)
-        a.out[a.D0 + a.kd + (i - a.D1)] = static_cast<int32_t>(i);
+        keep_at(a, a.D0 + a.kd + (i - a.D1), i);
 
     // Every block has read the global histograms; block 0 clears them for the next call.
     if (blockIdx.x == 0)
@@ -486,10 +493,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(
         if (j < a.ept && tb + j < end) {
             const int32_t i = static_cast<int32_t>(tb + j);
             if (key[j] > T) {
-                a.out[a.D0 + g_before + min(e_before, krem)] = i;
+                keep_at(a, a.D0 + g_before + min(e_before, krem), i);
                 ++g_before;
             } else if (key[j] == T) {
-                if (e_before < krem) a.out[a.D0 + g_before + e_before] = i;
+                if (e_before < krem) keep_at(a, a.D0 + g_before + e_before, i);
                 ++e_before;
             }
         }
@@ -497,9 +504,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(
     // Tokens outside the span are always kept: [0, D0) first, [D1, N) after the kept document tokens.
     const int64_t gstride = static_cast<int64_t>(ncta) * kSelectThreads;
     for (int64_t i = static_cast<int64_t>(rank) * kSelectThreads + tid; i < a.D0; i += gstride)
-        a.out[i] = static_cast<int32_t>(i);
+        keep_at(a, i, i);
     for (int64_t i = a.D1 + static_cast<int64_t>(rank) * kSelectThreads + tid; i < a.N; i += gstride)
-        a.out[a.D0 + a.kd + (i - a.D1)] = static_cast<int32_t>(i);
+        keep_at(a, a.D0 + a.kd + (i - a.D1), i);
     cluster_barrier();  // this CTA's shared memory stays alive until every CTA has read it
     // every CTA read the given first-pass histogram in pass 0: leave it zero for the next gate
     if (a.hist_given && rank == 0)
@@ -507,15 +514,19 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(
 }
 
 // K_doc == 0 (only tokens outside the span) or K_doc >= N_doc (every token).
-__global__ void select_trivial_kernel(int64_t N, int64_t D0, int64_t D1, int keep_doc, int32_t* out) {
+__global__ void select_trivial_kernel(int64_t N, int64_t D0, int64_t D1, int keep_doc, int32_t* out,
+                                      const float* scores, float* s_out) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N; i += stride) {
-        if (keep_doc)
-            out[i] = static_cast<int32_t>(i);
-        else if (i < D0)
-            out[i] = static_cast<int32_t>(i);
+        int64_t p = -1;
+        if (keep_doc || i < D0)
+            p = i;
         else if (i >= D1)
-            out[D0 + (i - D1)] = static_cast<int32_t>(i);
+            p = D0 + (i - D1);
+        if (p >= 0) {
+            out[p] = static_cast<int32_t>(i);
+            if (s_out) s_out[p] = __ldg(scores + i);
+        }
     }
 }
 
@@ -610,7 +621,7 @@ using namespace tg;
 // The select with keys from `scores`, or random keys from `seed` when scores is NULL.
 static tg_status select_impl(const float* scores, uint64_t seed, int64_t N, int64_t doc_begin, int64_t doc_end,
                              int64_t k_doc, int32_t* kept_idx, void* workspace, size_t workspace_bytes,
-                             void* stream, bool hist_given = false) {
+                             void* stream, bool hist_given = false, float* s_kept = nullptr) {
     const int64_t K = tg_kept_count(N, doc_begin, doc_end, k_doc);
     if (K < 0) return TG_ERR_INVALID_ARG;
     if (N > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
@@ -624,11 +635,12 @@ static tg_status select_impl(const float* scores, uint64_t seed, int64_t N, int6
         if (cudaMemsetAsync(&sc->hist[0][0], 0, sizeof(sc->hist[0]), st) != cudaSuccess) return TG_ERR_CUDA;
     }
     if (K == 0) return TG_OK;
-    if (!kept_idx) return TG_ERR_INVALID_ARG;
+    if (!kept_idx || (s_kept && !scores)) return TG_ERR_INVALID_ARG;
     if (kd == 0 || kd == n_doc) {
         const int64_t blocks = std::min<int64_t>((N + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
         select_trivial_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(N, doc_begin, doc_end,
-                                                                             kd == n_doc ? 1 : 0, kept_idx);
+                                                                             kd == n_doc ? 1 : 0, kept_idx,
+                                                                             scores, s_kept);
         return launch_status();
     }
     if (!workspace || workspace_bytes < tg_workspace_bytes(TG_OP_SELECT, N, 0, 0)) return TG_ERR_INVALID_ARG;
@@ -642,6 +654,7 @@ static tg_status select_impl(const float* scores, uint64_t seed, int64_t N, int6
     a.D1 = doc_end;
     a.kd = static_cast<unsigned int>(kd);
     a.out = kept_idx;
+    a.s_out = s_kept;
     a.sc = reinterpret_cast<SelectScratch*>(static_cast<char*>(workspace) + kWsHeader);
     a.status = status_word(workspace);
     a.hist_given = hist_given ? 1 : 0;
@@ -682,6 +695,16 @@ extern "C" tg_status tg_topk_select_after_gate(const float* scores, int64_t N, i
                                                size_t workspace_bytes, void* stream) {
     if (!scores && tg_kept_count(N, doc_begin, doc_end, k_doc) > 0) return TG_ERR_INVALID_ARG;
     return select_impl(scores, 0, N, doc_begin, doc_end, k_doc, kept_idx, workspace, workspace_bytes, stream, true);
+}
+
+extern "C" tg_status tg_topk_select_after_gate_kept_scores(const float* scores, int64_t N, int64_t doc_begin,
+                                                           int64_t doc_end, int64_t k_doc, int32_t* kept_idx,
+                                                           float* s_kept, void* workspace, size_t workspace_bytes,
+                                                           void* stream) {
+    const int64_t K = tg_kept_count(N, doc_begin, doc_end, k_doc);
+    if (K > 0 && (!scores || !s_kept)) return TG_ERR_INVALID_ARG;
+    return select_impl(scores, 0, N, doc_begin, doc_end, k_doc, kept_idx, workspace, workspace_bytes, stream, true,
+                       s_kept);
 }
 
 extern "C" tg_status tg_debug_set_select_wait_limit(uint64_t ns) {
@@ -748,7 +771,7 @@ extern "C" tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int6
     if (kd == 0 || kd == n_doc) {
         const int64_t blocks = std::min<int64_t>((N + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
         select_trivial_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(N, doc_begin, doc_end,
-                                                                             kd == n_doc ? 1 : 0, kept_idx);
+                                                                             kd == n_doc ? 1 : 0, kept_idx, nullptr, nullptr);
         return launch_status();
     }
     // the same launch shape as tg_topk_select; spans beyond its largest grid are rejected
@@ -774,6 +797,7 @@ extern "C" tg_status tg_topk_select_noalloc(const float* scores, int64_t N, int6
     a.D1 = doc_end;
     a.kd = static_cast<unsigned int>(kd);
     a.out = kept_idx;
+    a.s_out = nullptr;
     a.sc = reinterpret_cast<SelectScratch*>(scratch + kWsHeader);
     a.status = reinterpret_cast<unsigned int*>(scratch);
     a.ept = static_cast<int>(ept);

@@ -11,13 +11,23 @@ Steps, in order, all on the caller's current CUDA stream:
   gate     tg_gate_score_for_select libtokengate (tcgen05 GEMM + fused epilogue, which also
                                     counts the select's first radix pass)
   select   tg_topk_select_after_gate libtokengate (radix select from that count)
-  gather   tg_gather_compact        libtokengate (row copy)
+  gather   tg_gather_compact        libtokengate (bulk row copy; also the kept rows'
+                                    positions and scores)
   proj     tg_project_rope          libtokengate (tcgen05 GEMM of the kept rows with
                                     RoPE and V's fp16 copy in its epilogue)
   attn     tg_gated_attention_f16v  libtokengate (tcgen05 flash attention)
-With fused_projection=False the projection is instead a library GEMM
-(torch.matmul, cuBLAS) followed by tg_rope_apply, and the attention converts V
-itself (tg_gated_attention); stages "qkv", "rope", "attn".
+With gather_into_projection=True the compaction instead happens on the way into
+the projection: the select also writes the kept scores
+(tg_topk_select_after_gate_kept_scores) and the projection's operand tiles are
+the kept rows of h fetched by TMA gather4 copies (tg_project_rope_gather), so
+no compacted copy is written (stages "gate", "select", "proj", "attn").  It is
+not the default: on a B200 the gathered projection took 181 us at the 128k
+workload against 9 + 72 us for the copy and the dense projection (four rows of
+128 bytes per copy instruction, issued again for every one of the 16 column
+tiles).  With fused_projection=False the projection is a library GEMM
+(torch.matmul, cuBLAS) over the compacted rows followed by tg_rope_apply, and
+the attention converts V itself (tg_gated_attention); stages "gather", "qkv",
+"rope", "attn".
 torch allocates every buffer once (plumbing); the kept count K is known on the
 host, so nothing synchronizes inside a step.
 """
@@ -29,6 +39,7 @@ import torch
 
 from . import tokengate as tg
 
+STAGES_GATHER_FUSED = ("gate", "select", "proj", "attn")
 STAGES_FUSED = ("gate", "select", "gather", "proj", "attn")
 STAGES_UNFUSED = ("gate", "select", "gather", "qkv", "rope", "attn")
 STAGES = STAGES_FUSED
@@ -53,7 +64,8 @@ class GatedPrefillLayer:
     def __init__(self, N: int, doc_begin: int, doc_end: int, k_doc: int, W1: torch.Tensor, w2: torch.Tensor,
                  Wqkv: torch.Tensor, Hq: int, Hkv: int, d_h: int, gain: torch.Tensor, tau: float,
                  b1: Optional[torch.Tensor] = None, b2: float = 0.0, rms_weight: Optional[torch.Tensor] = None,
-                 eps: float = 1e-6, rope_base: float = 1e6, device="cuda", fused_projection: bool = True):
+                 eps: float = 1e-6, rope_base: float = 1e6, device="cuda", fused_projection: bool = True,
+                 gather_into_projection: bool = False):
         self.N, self.doc_begin, self.doc_end, self.k_doc = N, doc_begin, doc_end, k_doc
         self.K = tg.tg_kept_count(N, doc_begin, doc_end, k_doc)
         if self.K < 0:
@@ -68,7 +80,8 @@ class GatedPrefillLayer:
         self.rms_weight = None if rms_weight is None else rms_weight.to(dev, torch.bfloat16).contiguous()
         self.eps, self.rope_base, self.tau = eps, rope_base, float(tau)
         self.fused = fused_projection
-        self.stages = STAGES_FUSED if fused_projection else STAGES_UNFUSED
+        self.gather_fused = fused_projection and gather_into_projection
+        self.stages = (STAGES_GATHER_FUSED if self.gather_fused else STAGES_FUSED) if fused_projection else STAGES_UNFUSED
         self.Wqkv = Wqkv.to(dev, torch.bfloat16).contiguous()             # [(Hq + 2 Hkv) d_h, d]
         self.WqkvT = None if fused_projection else self.Wqkv.t().contiguous()
         self.gain = gain.to(dev, torch.float32).contiguous()
@@ -84,7 +97,8 @@ class GatedPrefillLayer:
             self.v16 = None
         self.scores = torch.empty(N, dtype=torch.float32, device=dev)
         self.kept = torch.empty(max(K, 1), dtype=torch.int32, device=dev)
-        self.h_kept = torch.empty(K, d, dtype=torch.bfloat16, device=dev)
+        # the compacted rows exist only when a separate step writes them
+        self.h_kept = None if self.gather_fused else torch.empty(K, d, dtype=torch.bfloat16, device=dev)
         self.pos = torch.empty(max(K, 1), dtype=torch.int32, device=dev)
         self.s_kept = torch.empty(max(K, 1), dtype=torch.float32, device=dev)
         self.qkv = torch.empty(K, (Hq + 2 * Hkv) * d_h, dtype=torch.bfloat16, device=dev)
@@ -105,15 +119,25 @@ class GatedPrefillLayer:
                                         b1=self.b1, b2=self.b2, rms_weight=self.rms_weight, eps=self.eps)
 
         def select():
-            tg.tg_topk_select_after_gate(self.scores, self.doc_begin, self.doc_end, self.k_doc, self.kept[:K], self.ws)
+            if self.gather_fused:
+                tg.tg_topk_select_after_gate_kept_scores(self.scores, self.doc_begin, self.doc_end, self.k_doc,
+                                                         self.kept[:K], self.s_kept[:K], self.ws)
+            else:
+                tg.tg_topk_select_after_gate(self.scores, self.doc_begin, self.doc_end, self.k_doc, self.kept[:K],
+                                             self.ws)
 
         def gather():
             tg.tg_gather_compact(h, self.kept[:K], self.h_kept, self.pos[:K], scores=self.scores,
                                  s_out=self.s_kept[:K])
 
         def proj():
-            tg.tg_project_rope(self.h_kept, self.Wqkv, self.pos[:K], self.qkv, self.ws_proj, self.Hq, self.Hkv,
-                               self.d_h, base=self.rope_base, v16=self.v16)
+            if self.gather_fused:
+                # the positions are the kept indices themselves
+                tg.tg_project_rope_gather(h, self.kept[:K], self.Wqkv, self.kept[:K], self.qkv, self.ws_proj,
+                                          self.Hq, self.Hkv, self.d_h, base=self.rope_base, v16=self.v16)
+            else:
+                tg.tg_project_rope(self.h_kept, self.Wqkv, self.pos[:K], self.qkv, self.ws_proj, self.Hq, self.Hkv,
+                                   self.d_h, base=self.rope_base, v16=self.v16)
 
         def qkv():
             torch.matmul(self.h_kept, self.WqkvT, out=self.qkv)
@@ -153,11 +177,16 @@ class GatedPrefillLayer:
         kept_host.copy_(kept, non_blocking=True)
         return out_host, kept_host
 
+    def positions(self) -> torch.Tensor:
+        """[K] int32 original positions of the kept rows (the kept indices when the gather is fused)."""
+        return self.kept[:self.K] if self.gather_fused else self.pos[:self.K]
+
     def launches_per_step(self) -> int:
-        """libtokengate kernels per run(): gate (+ the RMSNorm-weight fold), select, gather, then either the
-        projection's two (cos / sin table, GEMM) and the attention, or RoPE and the attention's two (V to
-        fp16, attention) after the library GEMM."""
-        return 6 + (1 if self.rms_weight is not None else 0)
+        """libtokengate kernels per run(): gate (+ the RMSNorm-weight fold), select, then the projection with
+        its gather and the attention; or a separate gather, the projection and the attention; or a gather,
+        RoPE and the attention's two (V to fp16, attention) after the library GEMM."""
+        n = 4 if self.gather_fused else (5 if self.fused else 6)
+        return n + (1 if self.rms_weight is not None else 0)
 
     def device_status(self) -> int:
         """OR of the status words of the layer's workspaces (synchronizes the stream); 0 = no timeout

@@ -21,6 +21,7 @@ TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_CUDA, TG_ERR_TIMEOUT, TG_E
 TG_OP_GATE, TG_OP_SELECT, TG_OP_ATTENTION, TG_OP_ALL, TG_OP_DECODE, TG_OP_ATTENTION_BACKWARD, TG_OP_PROJECT = range(7)
 TG_STATUS_SELECT_TIMEOUT, TG_STATUS_GATE_TIMEOUT, TG_STATUS_ATTENTION_TIMEOUT, TG_STATUS_DECODE_TIMEOUT = 1, 2, 4, 8
 TG_STATUS_BACKWARD_TIMEOUT, TG_STATUS_PROJECT_TIMEOUT, TG_STATUS_V_RANGE = 16, 32, 64
+TG_STATUS_INDEX_RANGE = 128
 
 _lib = None
 
@@ -52,6 +53,7 @@ def lib() -> ctypes.CDLL:
         L.tg_gate_score_for_select.argtypes = [vp, i64, i32, i64, vp, f32, vp, vp, vp, f32, i32, vp, i64, i64, vp, sz,
                                                vp]
         L.tg_topk_select_after_gate.argtypes = [vp, i64, i64, i64, i64, vp, vp, sz, vp]
+        L.tg_topk_select_after_gate_kept_scores.argtypes = [vp, i64, i64, i64, i64, vp, vp, vp, sz, vp]
         L.tg_topk_select_noalloc.argtypes = [vp, i64, i64, i64, i64, vp, vp]
         L.tg_topk_select_noalloc_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
         L.tg_random_select.argtypes = [i64, i64, i64, i64, ctypes.c_uint64, vp, vp, sz, vp]
@@ -63,6 +65,8 @@ def lib() -> ctypes.CDLL:
                                               vp]
         L.tg_gated_decode.argtypes = [vp, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp, vp, vp, sz, vp]
         L.tg_project_rope.argtypes = [vp, i64, i32, i64, vp, i32, i32, i32, vp, f64, vp, i64, vp, vp, sz, vp]
+        L.tg_project_rope_gather.argtypes = [vp, i64, i32, i64, vp, i64, vp, i32, i32, i32, vp, f64, vp, i64, vp, vp,
+                                             sz, vp]
         L.tg_gated_attention_backward.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp,
                                                   vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.tg_debug_set_select_wait_limit.argtypes = [ctypes.c_uint64]
@@ -195,6 +199,25 @@ def tg_topk_select_after_gate(scores, doc_begin: int, doc_end: int, k_doc: int, 
         _ptr(scores), N, doc_begin, doc_end, k_doc, _ptr(kept_idx), _ptr(workspace), workspace.numel(),
         _stream(stream)))
     return kept_idx
+
+
+def tg_topk_select_after_gate_kept_scores(scores, doc_begin: int, doc_end: int, k_doc: int, kept_idx, s_kept,
+                                          workspace, stream=None):
+    """tg_topk_select_after_gate that also writes s_kept[i] = scores[kept_idx[i]]."""
+    _req(scores, "scores", torch.float32, 1)
+    _req(kept_idx, "kept_idx", torch.int32, 1)
+    _req(s_kept, "s_kept", torch.float32, 1)
+    N = scores.shape[0]
+    K = tg_kept_count(N, doc_begin, doc_end, k_doc)
+    if K < 0:
+        raise TokenGateError("tg_topk_select_after_gate_kept_scores", TG_ERR_INVALID_ARG)
+    if (kept_idx.numel() < K or s_kept.numel() < K or not scores.is_contiguous() or not kept_idx.is_contiguous()
+            or not s_kept.is_contiguous()):
+        raise ValueError("kept_idx or s_kept too small or not contiguous")
+    _check("tg_topk_select_after_gate_kept_scores", lib().tg_topk_select_after_gate_kept_scores(
+        _ptr(scores), N, doc_begin, doc_end, k_doc, _ptr(kept_idx), _ptr(s_kept), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return kept_idx, s_kept
 
 
 def tg_topk_select(scores, doc_begin: int, doc_end: int, k_doc: int, kept_idx, workspace, stream=None):
@@ -375,6 +398,31 @@ def tg_project_rope(x, W, pos, qkv, workspace, Hq: int, Hkv: int, d_h: int, base
     _check("tg_project_rope", lib().tg_project_rope(
         _ptr(x), K, d, x.stride(0), _ptr(W), Hq, Hkv, d_h, _ptr(pos), float(base), _ptr(qkv), qkv.stride(0),
         _ptr(v16), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return qkv
+
+
+def tg_project_rope_gather(h, rows, W, pos, qkv, workspace, Hq: int, Hkv: int, d_h: int, base: float = 1e6,
+                           v16=None, stream=None):
+    """tg_project_rope over the rows h[rows[r]] (rows [K] int32), gathered into the GEMM's operand tiles."""
+    _req(h, "h", torch.bfloat16, 2)
+    _req(rows, "rows", torch.int32, 1)
+    _req(W, "W", torch.bfloat16, 2)
+    _req(pos, "pos", torch.int32, 1)
+    _req(qkv, "qkv", torch.bfloat16, 2)
+    _req(v16, "v16", torch.float16, 2)
+    N, d = h.shape
+    K = qkv.shape[0]
+    cols = (Hq + 2 * Hkv) * d_h
+    if tuple(W.shape) != (cols, d) or not W.is_contiguous():
+        raise ValueError("W must be a contiguous [(Hq + 2 Hkv) d_h, d] tensor")
+    if (qkv.shape[1] != cols or qkv.stride(1) != 1 or pos.shape[0] < K or rows.shape[0] < K
+            or not rows.is_contiguous()):
+        raise ValueError("shape mismatch")
+    if v16 is not None and (tuple(v16.shape) != (K, Hkv * d_h) or not v16.is_contiguous()):
+        raise ValueError("v16 must be a contiguous [K, Hkv d_h] tensor")
+    _check("tg_project_rope_gather", lib().tg_project_rope_gather(
+        _ptr(h), N, d, h.stride(0), _ptr(rows), K, _ptr(W), Hq, Hkv, d_h, _ptr(pos), float(base), _ptr(qkv),
+        qkv.stride(0), _ptr(v16), _ptr(workspace), workspace.numel(), _stream(stream)))
     return qkv
 
 

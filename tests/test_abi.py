@@ -191,3 +191,23 @@ def test_project_rope_workspace_and_argument_errors(lib):
     assert proj(v16=40) == INV                      # misaligned fp16 copy
     assert proj(ws_bytes=128) == INV                 # shorter than the status word
     assert proj(K=0) == tg.TG_OK
+
+
+def test_gathered_projection_and_kept_scores_argument_errors(lib):
+    # host-side rejections, before any device work
+    vp = ctypes.c_void_p
+    INV = tg.TG_ERR_INVALID_ARG
+    ws = tg.tg_workspace_bytes(tg.TG_OP_PROJECT, 300, 128)
+
+    def projg(N=1000, rows=64, K=300, h=16):
+        return lib.tg_project_rope_gather(vp(h), N, 256, 256, vp(rows) if rows else None, K, vp(4096), 4, 2, 128,
+                                          vp(64), 1e6, vp(8192), 1024, None, vp(256), ws, None)
+
+    assert projg(N=-1) == INV
+    assert projg(rows=0) == INV                      # no index array
+    assert projg(N=0) == INV                         # rows to gather from an empty h
+    assert projg(K=0) == tg.TG_OK                    # nothing to do
+    assert projg(h=24) == INV                        # misaligned h
+    sel = lib.tg_topk_select_after_gate_kept_scores
+    assert sel(vp(16), 1000, 0, 960, 256, vp(64), None, vp(256), 1 << 20, None) == INV  # no s_kept
+    assert sel(None, 1000, 0, 960, 256, vp(64), vp(128), vp(256), 1 << 20, None) == INV  # no scores

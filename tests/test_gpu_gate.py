@@ -151,16 +151,23 @@ def test_gate_and_select_pair(N, d, d_g, db, de, k):
     plain = torch.empty(N, device="cuda")
     tg.tg_gate_score(h, W1, w2, plain, ws)
     K = tg.tg_kept_count(N, db, de, k)
-    for _ in range(3):
+    for it in range(3):
         scores = torch.full((N,), float("nan"), device="cuda")
         kept = torch.full((max(K, 1),), -1, dtype=torch.int32, device="cuda")
+        s_kept = torch.full((max(K, 1),), float("nan"), device="cuda")
         tg.tg_gate_score_for_select(h, W1, w2, scores, ws, db, de)
-        tg.tg_topk_select_after_gate(scores, db, de, k, kept[:K], ws)
+        if it == 1:  # the variant that also writes the kept tokens' scores
+            tg.tg_topk_select_after_gate_kept_scores(scores, db, de, k, kept[:K], s_kept[:K], ws)
+        else:
+            tg.tg_topk_select_after_gate(scores, db, de, k, kept[:K], ws)
         torch.cuda.synchronize()
         assert tg.tg_device_status(ws) == 0
         assert torch.equal(scores.view(torch.int32), plain.view(torch.int32))
         s_np = scores.cpu().numpy()
-        assert np.array_equal(kept[:K].cpu().numpy(), oracle.topk_select(s_np, db, de, k))
+        kept_np = kept[:K].cpu().numpy()
+        assert np.array_equal(kept_np, oracle.topk_select(s_np, db, de, k))
+        if it == 1:
+            assert np.array_equal(s_kept[:K].cpu().numpy().view(np.int32), s_np[kept_np].view(np.int32))
         # the first-pass count (2048 words after the status header and the barrier words) is zero again
         hist0 = ws[256 + 256: 256 + 256 + 2048 * 4].view(torch.int32)
         assert int(hist0.abs().sum().item()) == 0

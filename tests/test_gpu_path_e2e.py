@@ -65,14 +65,20 @@ def sample_rows(K, kept, heavy_rows, n=48):
     return np.unique(np.concatenate(rows))
 
 
-@pytest.mark.parametrize("name", WORKLOADS)
-def test_path_matches_oracle_pipeline(name):
+CASES = [(name, False) for name in WORKLOADS] + [(name, True) for name in ("tiny-1k", "qwen3-1.7b-16k",
+                                                                             "qwen3-1.7b-128k")]
+
+
+@pytest.mark.parametrize("name,gather_into_projection", CASES,
+                         ids=[f"{n}{'-gathered-projection' if g else ''}" for n, g in CASES])
+def test_path_matches_oracle_pipeline(name, gather_into_projection):
+    # gather_into_projection: the layer whose projection gathers the kept rows from h itself
     w = synth.WORKLOADS[name]
     gi = synth.gate_inputs(w)
     ap = synth.attn_params(w)
     dev = torch.device("cuda", 0)
     h = gi.h.to(torch.bfloat16)
-    layer = bench.make_layer(w, gi, ap, dev)
+    layer = bench.make_layer(w, gi, ap, dev, gather_into_projection=gather_into_projection)
     out, kept = layer.run(h.to(dev))
     torch.cuda.synchronize()
     assert layer.device_status() == 0
@@ -103,10 +109,13 @@ def test_path_matches_oracle_pipeline(name):
                                        w.Hkv, w.d_h, ap.gain.numpy(), ap.tau, rows, eps=w.eps,
                                        rope_base=w.rope_base, kept_override=kept_gpu, scores=o.scores)
 
-    # gather: bit-exact against the oracle's gather of the same kept set with the GPU's scores
+    # compaction: bit-exact against the oracle's gather of the same kept set with the GPU's scores (the
+    # path gathers the rows inside the projection's operand loads, which the Q/K/V checks below cover;
+    # the kept scores come from the select, the positions are the kept indices)
     want_h, want_pos, want_s = oracle.gather_compact(h_bits, kept_gpu, scores=s_gpu)
-    assert np.array_equal(layer.h_kept.cpu().view(torch.int16).numpy().view(np.uint16), want_h)
-    assert np.array_equal(layer.pos[:K].cpu().numpy(), want_pos)
+    if layer.h_kept is not None:
+        assert np.array_equal(layer.h_kept.cpu().view(torch.int16).numpy().view(np.uint16), want_h)
+    assert np.array_equal(layer.positions().cpu().numpy(), want_pos)
     assert np.array_equal(layer.s_kept[:K].cpu().numpy(), want_s)
 
     # Q, K, V on the sampled rows

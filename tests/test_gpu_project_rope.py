@@ -63,3 +63,45 @@ def test_project_rope_matches_oracle(K, d, Hq, Hkv, d_h):
     vcols = slice((Hq + Hkv) * d_h, None)
     wv = want[:, vcols]
     assert np.all(np.abs(v16 - wv) <= 2.0 ** -11 * np.abs(wv) + 2.0 ** -20 * 2 * absum[:, vcols] + 1e-6)
+
+
+@pytest.mark.parametrize("N,K,d,Hq,Hkv,d_h,bad", [
+    (1000, 300, 256, 4, 2, 128, None),        # ragged K, repeated rows
+    (5000, 129, 512, 4, 2, 64, None),         # d_h = 64, K not a multiple of 4
+    (131072, 4608, 2048, 16, 8, 128, None),   # the 128k workload's kept set
+    (1000, 300, 256, 4, 2, 128, 77),          # one index outside [0, N)
+])
+def test_project_rope_gather_matches_dense(N, K, d, Hq, Hkv, d_h, bad):
+    # tg_project_rope_gather (rows gathered from h by TMA gather4 copies into the operand tiles) gives
+    # tg_project_rope on the compacted rows bit for bit; that one is checked against the oracle above.
+    # An index outside [0, N) is not followed: row 0 is read in its place and the status flags it.
+    g = torch.Generator().manual_seed(N + K)
+    h = torch.randn(N, d, generator=g).to(torch.bfloat16)
+    W = (torch.randn((Hq + 2 * Hkv) * d_h, d, generator=g) / d ** 0.5).to(torch.bfloat16)
+    rows = torch.randint(0, N, (K,), generator=g).to(torch.int32)
+    if bad is not None:
+        rows[bad] = N
+    cols = (Hq + 2 * Hkv) * d_h
+    x = h[torch.where(rows < N, rows, torch.zeros_like(rows)).long()].contiguous()
+    outs = []
+    for gather in (True, False):
+        qkv, cq = guarded((K, cols), torch.bfloat16)
+        v16, cv = guarded((K, Hkv * d_h), torch.float16)
+        qkv.fill_(float("nan"))
+        v16.fill_(float("nan"))
+        ws = tg.new_workspace(K, d_h, op=tg.TG_OP_PROJECT)
+        if gather:
+            tg.tg_project_rope_gather(h.cuda(), rows.cuda(), W.cuda(), rows.cuda(), qkv, ws, Hq, Hkv, d_h, base=1e6,
+                                      v16=v16)
+        else:
+            tg.tg_project_rope(x.cuda(), W.cuda(), rows.cuda(), qkv, ws, Hq, Hkv, d_h, base=1e6, v16=v16)
+        torch.cuda.synchronize()
+        cq(), cv()
+        status = tg.tg_device_status(ws)
+        if gather and bad is not None:
+            assert status == tg.TG_STATUS_INDEX_RANGE
+        else:
+            assert status == 0
+        outs.append((qkv.cpu(), v16.cpu()))
+    assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16))
+    assert torch.equal(outs[0][1].view(torch.int16), outs[1][1].view(torch.int16))
