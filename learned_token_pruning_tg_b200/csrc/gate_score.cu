@@ -399,10 +399,6 @@ gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_
         tma_prefetch_desc(&tmap_h);
         tma_prefetch_desc(&tmap_w);
     }
-    for (int j = threadIdx.x; j < DG; j += kThreads) {
-        w2_s[j] = a.w2[j];
-        b1_s[j] = a.b1 ? a.b1[j] : 0.0f;
-    }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, C::kTmemCols);
         tmem_relinquish_pair();
@@ -411,6 +407,14 @@ gate_score_pair_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_
     cluster_sync_all();  // both CTAs' barriers are initialised before either touches the other's
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // set-up done: from here on global memory is shared with the kernels before this one
+    pdl_trigger();
+    pdl_wait();
+    for (int j = threadIdx.x; j < DG; j += kThreads) {
+        w2_s[j] = a.w2[j];
+        b1_s[j] = a.b1 ? a.b1[j] : 0.0f;
+    }
+    __syncthreads();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -626,13 +630,14 @@ static tg_status launch_pair(const CUtensorMap& mh, const CUtensorMap& mw, const
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = PairCfg::kSmem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, gate_score_pair_kernel, mh, mw, a) == cudaSuccess ? TG_OK : TG_ERR_CUDA;
 }
 

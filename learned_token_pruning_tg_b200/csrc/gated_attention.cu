@@ -246,6 +246,8 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_trigger();
+    pdl_wait();  // global memory is shared with the kernels before this one from here on
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -634,8 +636,15 @@ static tg_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     if (items > 0x7fffffffLL) return TG_ERR_UNSUPPORTED;
     // persistent: one CTA per SM (TMEM and shared memory allow no more), each taking several items
     const int grid = static_cast<int>(std::min<int64_t>(items, num_sms()));
-    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, st>>>(mq, mk, mv, a);
-    return launch_status();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, a) == cudaSuccess ? TG_OK : TG_ERR_CUDA;
 }
 
 }  // namespace attn

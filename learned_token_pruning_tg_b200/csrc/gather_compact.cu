@@ -35,6 +35,8 @@ gather_rows_bulk_kernel(const uint8_t* __restrict__ h, int64_t ld_bytes, uint32_
     if (lane < rows_per_block) mbar_init(bar, 1);
     fence_mbar_init();
     __syncwarp();
+    pdl_trigger();
+    pdl_wait();  // global memory is shared with the kernels before this one from here on
     uint8_t* slot = g_smem + static_cast<size_t>(lane) * row_bytes;
     uint32_t ph = 0;
     for (int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_block; r0 < K;
@@ -144,10 +146,19 @@ extern "C" tg_status tg_gather_compact(const tg_bf16* h, int64_t N, int32_t d, i
         static std::atomic<int> smem_set[64];
         if (!set_max_dynamic_smem(gather_rows_bulk_kernel, smem, smem_set)) return TG_ERR_CUDA;
         const int64_t blocks = std::min<int64_t>((K + rows_per_block - 1) / rows_per_block, static_cast<int64_t>(sms));
-        gather_rows_bulk_kernel<<<static_cast<unsigned>(blocks), 32, smem, st>>>(
-            reinterpret_cast<const uint8_t*>(h), ld_h * 2, row_bytes, kept_idx, K, N, rows_per_block, pos_in, scores,
-            reinterpret_cast<uint8_t*>(h_out), pos_out, s_out);
-        return launch_status();
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+        cfg.blockDim = dim3(32);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1] = {pdl_attr()};
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, gather_rows_bulk_kernel, reinterpret_cast<const uint8_t*>(h), ld_h * 2,
+                                  row_bytes, kept_idx, K, N, rows_per_block, pos_in, scores,
+                                  reinterpret_cast<uint8_t*>(h_out), pos_out, s_out) == cudaSuccess
+                   ? TG_OK
+                   : TG_ERR_CUDA;
     }
     int64_t blocks = (K + kGatherWarps - 1) / kGatherWarps;
     const int64_t max_blocks = static_cast<int64_t>(sms) * 8;  // 8 resident blocks of 256 threads per SM

@@ -433,6 +433,8 @@ project_rope_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __gri
     cluster_sync_all();  // both CTAs' barriers are initialised before either touches the other's
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger();
+    pdl_wait();  // global memory is shared with the kernels before this one from here on
 
     if (warp == 0 && a.rows) {
         // ------------------------------------------------------------ TMA producer (both CTAs), rows gathered
@@ -680,13 +682,14 @@ static tg_status project_impl(const tg_bf16* x, int64_t n_rows, const int32_t* r
         cfg.blockDim = dim3(proj::kThreads);
         cfg.dynamicSmemBytes = proj::kPairSmem;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1] = pdl_attr();
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         return cudaLaunchKernelEx(&cfg, proj::project_rope_pair_kernel, mx, mw2, a) == cudaSuccess ? TG_OK
                                                                                                   : TG_ERR_CUDA;
     }

@@ -106,6 +106,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with the programmatic-serialization attribute (pdl_attr) may be scheduled while
+// the kernel before it on the stream is still finishing.  pdl_wait() blocks the calling thread until
+// that kernel has completed and its memory operations are visible (every thread that touches global
+// memory the kernels before it write or read calls it first); without the attribute it returns at
+// once.  pdl_trigger() lets the next such kernel be scheduled once every CTA of this one has called
+// it or exited (the next kernel still waits for this one's completion in its own pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

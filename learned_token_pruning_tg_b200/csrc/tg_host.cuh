@@ -132,6 +132,15 @@ inline bool set_max_dynamic_smem(Kernel* kern, int bytes, std::atomic<int>* done
     return true;
 }
 
+// Launch attribute letting a kernel start while the previous kernel on the stream finishes (the
+// kernel itself calls pdl_wait() before touching memory the previous kernels use).
+inline cudaLaunchAttribute pdl_attr() {
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at.val.programmaticStreamSerializationAllowed = 1;
+    return at;
+}
+
 inline tg_status launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;

@@ -323,6 +323,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_cluster_kernel(
     const int64_t base = a.D0 + static_cast<int64_t>(rank) * chunk;
     const int64_t end = min(base + chunk, a.D1);
     const int64_t tb = base + static_cast<int64_t>(tid) * a.ept;
+    // global memory is shared with the kernels before this one from here on
+    pdl_trigger();
+    pdl_wait();
 
     uint32_t key[EPT];
 #pragma unroll
@@ -582,13 +585,14 @@ static cudaError_t launch_select_cluster(const SelectArgs& a, int cl, cudaStream
     cfg.blockDim = dim3(kSelectThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cl;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
