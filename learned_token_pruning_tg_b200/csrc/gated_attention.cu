@@ -81,7 +81,7 @@ struct Cfg {
     static constexpr int kOffAugA = kOffV + kStages * kKVTile;  // [NQ]      gamma_h parts, every row alike
     static constexpr int kOffAugB = kOffAugA + NQ * kAugTile;   // [kStages] s_c parts of a K tile's keys
     static constexpr int kOffBar = kOffAugB + kStages * kAugTile;
-    static constexpr int kNumBars = 2 + 5 * kStages + 4 * NQ + 1;
+    static constexpr int kNumBars = 2 + 4 * kStages + 4 * NQ + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmem = kOffMisc + 16 + 1024;
     static constexpr uint32_t kTmemCols = (NQ * kBN + NQ * D > 256) ? 512 : 256;
@@ -181,12 +181,11 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* q_full = bars;                        // TMA -> MMA (one phase per work item)
     uint64_t* q_empty = bars + 1;                   // commit after an item's last S -> TMA (next Q), bias warp
-    uint64_t* k_full = bars + 2;                    // [kStages] TMA -> MMA
+    uint64_t* k_full = bars + 2;                    // [kStages] TMA bytes of K + the bias warp's 32 lanes -> MMA
     uint64_t* k_empty = k_full + kStages;           // [kStages] commit after the last S of a K tile -> TMA
     uint64_t* v_full = k_empty + kStages;           // [kStages] TMA -> MMA
     uint64_t* v_empty = v_full + kStages;           // [kStages] commit after the last P V of a V tile -> TMA
-    uint64_t* aug_full = v_empty + kStages;         // [kStages] converter (32 lanes) wrote B of a K tile -> MMA
-    uint64_t* s_full = aug_full + kStages;          // [NQ] commit after S_h(j) (and P_h(j-1) V) -> softmax h
+    uint64_t* s_full = v_empty + kStages;           // [NQ] commit after S_h(j) (and P_h(j-1) V) -> softmax h
     uint64_t* p_full = s_full + NQ;                 // [NQ] 128 softmax threads wrote P_h(j) -> MMA
     uint64_t* o_full = p_full + NQ;                 // [NQ] commit after an item's last P_h V -> epilogue h
     uint64_t* o_empty = o_full + NQ;                // [NQ] 128 epilogue threads read O_h -> MMA (next item)
@@ -219,11 +218,10 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&k_full[s], 1);
+            mbar_init(&k_full[s], 1 + 32);  // the TMA bytes of K, and the 32 lanes writing its bias operand B
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
-            mbar_init(&aug_full[s], 32);
         }
         for (int h = 0; h < NQ; ++h) {
             mbar_init(&s_full[h], 1);
@@ -329,11 +327,10 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
             const uint32_t aa_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffAugA), 128);
             const uint32_t ab_lo0 = sw128_desc_lo(smem_u32(smem + C::kOffAugB), 128);
             const bool bias = a.gain != nullptr && a.s_kept != nullptr;
-            // K tile g and its bias operand B both in shared memory
+            // K tile g and its bias operand B both in shared memory (one barrier counts both)
             auto wait_k = [&](int g) -> bool {
                 const uint32_t ph = static_cast<uint32_t>(g / kStages) & 1;
-                return mbar_wait(&k_full[g % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT) &&
-                       mbar_wait(&aug_full[g % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
+                return mbar_wait(&k_full[g % kStages], ph, abort_flag, a.status, TG_STATUS_ATTENTION_TIMEOUT);
             };
             // S_h = Q_h K_g^T into head h's S columns, then signal softmax h (the commit
             // also covers every earlier MMA of this thread, P_h(g-1) V_{g-1} included)
@@ -420,6 +417,13 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
         // B for K tile g (key tile j of the item): row c holds s_c's parts (k = col mod 3 for col < 9)
         auto fill_aug = [&](int g, int j, const Item& w, int it) -> bool {
             const int st = g % kStages;
+            // the tile's key scores are loaded first, so their latency overlaps the wait for the slot
+            float sv[kBN / 32];
+#pragma unroll
+            for (int i = 0; i < kBN / 32; ++i) {
+                const int64_t key = static_cast<int64_t>(j) * kBN + i * 32 + lane;
+                sv[i] = (a.s_kept && key < a.K) ? __ldg(a.s_kept + key) : 0.0f;
+            }
             // the slot is free once the S MMAs of tile g - kStages are done (same release as K)
             if (!mbar_wait(&k_empty[st], (static_cast<uint32_t>(g / kStages) & 1) ^ 1, abort_flag, a.status,
                            TG_STATUS_ATTENTION_TIMEOUT))
@@ -448,15 +452,14 @@ gated_attention_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
 #pragma unroll
             for (int i = 0; i < kBN / 32; ++i) {
                 const int c = i * 32 + lane;
-                const int64_t key = static_cast<int64_t>(j) * kBN + c;
                 __nv_bfloat16 p[3];
-                split3_bf16((a.s_kept && key < a.K) ? a.s_kept[key] : 0.0f, p);
+                split3_bf16(sv[i], p);
                 const __nv_bfloat16 z = __float2bfloat16_rn(0.0f);
                 dst[aug_slot(c, 0)] = make_uint4(bf2(p[0], p[1]), bf2(p[2], p[0]), bf2(p[1], p[2]), bf2(p[0], p[1]));
                 dst[aug_slot(c, 1)] = make_uint4(bf2(p[2], z), 0u, 0u, 0u);
             }
             fence_proxy_async_smem();  // generic-proxy writes -> tensor-core (async proxy) reads
-            mbar_arrive(&aug_full[st]);
+            mbar_arrive(&k_full[st]);  // B written: with K's bytes this completes the tile's k_full phase
             return true;
         };
         bool ok = true;
