@@ -617,7 +617,7 @@ def run_tokengate(args, rank, world, local_rank):
     roof["peak_source"] = peaks["source"] + (" (burst bf16)" if roof["bound"] == "tensor" else " (HBM copy)")
     if roof["bound"] == "tensor":
         roof["frac_of_sustained_peak"] = roof["achieved"] / peaks["bf16_tflops_sustained"]
-    # the benchmark spec path (gate, select, gather, attention) and the whole step (plus the projection)
+    # the specification's path (gate, select, gather, attention) and the whole step (plus the projection)
     # the spec steps that run as stages of their own (a layer that gathers inside the projection's
     # operand loads has no gather stage: that work is inside "proj", which the step fractions cover)
     path = [s for s in ("gate", "select", "gather", "attn") if s in stages]
