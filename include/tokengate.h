@@ -414,6 +414,13 @@ tg_status tg_project_rope_gather(const tg_bf16* h, int64_t N, int32_t d, int64_t
  * Synchronous; not for use while a select may be running. */
 tg_status tg_debug_set_select_wait_limit(uint64_t ns);
 
+/* Test hook: with enabled = 0 the gate (d_g = 256) and the projection
+ * (tg_project_rope, tg_project_rope_gather) run their one-CTA kernels instead
+ * of the CTA-pair kernels they use where the device offers clusters of 2, so
+ * that tests can check both shapes on one device; 1 restores the default.
+ * Process-wide; not for use while another thread launches those calls. */
+tg_status tg_debug_set_cta_pairs(int enabled);
+
 /* Reads the workspace's status word after synchronizing `stream`.
  * *status_word receives the raw TG_STATUS_* bits (may be NULL).
  * Returns TG_ERR_TIMEOUT if a timeout bit is set, else TG_ERR_RANGE if

@@ -706,7 +706,7 @@ static tg_status gate_impl(const tg_bf16* h, int64_t N, int32_t d, int64_t ld_h,
     a.D0 = D0;
     a.D1 = D1;
     const int64_t num_tiles = (N + gate::kBM - 1) / gate::kBM;
-    if (d_g == 256 && gate::pair_kernel_available()) {
+    if (d_g == 256 && cta_pairs_enabled().load() && gate::pair_kernel_available()) {
         // W's half tile: 128 rows per CTA
         CUtensorMap mw2;
         const uint32_t wb2[2] = {gate::kBK, static_cast<uint32_t>(gate::kPairBN)};

@@ -670,7 +670,7 @@ static tg_status project_impl(const tg_bf16* x, int64_t n_rows, const int32_t* r
     a.ld_qkv = ld_qkv;
     a.v16 = reinterpret_cast<__half*>(v16);
     a.status = status_word(workspace);
-    if (proj::pair_kernel_available()) {
+    if (cta_pairs_enabled().load() && proj::pair_kernel_available()) {
         // 256 x 256 tiles over CTA pairs; W's box is half a tile (128 rows)
         CUtensorMap mw2;
         const uint32_t wb2[2] = {proj::kBK, proj::kBN / 2};

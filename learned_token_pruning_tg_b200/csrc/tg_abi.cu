@@ -68,3 +68,8 @@ extern "C" tg_status tg_device_status(const void* workspace, uint32_t* status_wo
     if (w & TG_STATUS_TIMEOUT_BITS) return TG_ERR_TIMEOUT;
     return (w & (TG_STATUS_V_RANGE | TG_STATUS_INDEX_RANGE)) ? TG_ERR_RANGE : TG_OK;
 }
+
+extern "C" tg_status tg_debug_set_cta_pairs(int enabled) {
+    tg::cta_pairs_enabled().store(enabled ? 1 : 0);
+    return TG_OK;
+}

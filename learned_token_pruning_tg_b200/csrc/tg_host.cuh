@@ -28,6 +28,13 @@ inline int current_device() {
     return (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) ? dev : -1;
 }
 
+// Whether the gate (d_g = 256) and the projection may use their CTA-pair kernels (the default);
+// tg_debug_set_cta_pairs(0) makes them take their one-CTA kernels, so tests can run both.
+inline std::atomic<int>& cta_pairs_enabled() {
+    static std::atomic<int> enabled{1};
+    return enabled;
+}
+
 // Number of SMs of the current device (queried once per device).
 inline int num_sms() {
     static int cache[64] = {0};

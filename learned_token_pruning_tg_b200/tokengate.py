@@ -70,11 +70,14 @@ def lib() -> ctypes.CDLL:
         L.tg_gated_attention_backward.argtypes = [vp, i64, vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, f32, vp,
                                                   vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.tg_debug_set_select_wait_limit.argtypes = [ctypes.c_uint64]
+        L.tg_debug_set_cta_pairs.argtypes = [ctypes.c_int]
         L.tg_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
         for fn in ("tg_gate_score", "tg_gate_score_for_select", "tg_topk_select", "tg_topk_select_after_gate", "tg_topk_select_noalloc", "tg_random_select", "tg_gather_compact",
                    "tg_rope_apply",
                    "tg_gated_attention", "tg_gated_attention_f16v", "tg_project_rope",
-                   "tg_gated_attention_backward", "tg_gated_decode", "tg_debug_set_select_wait_limit", "tg_device_status"):
+                   "tg_gated_attention_backward", "tg_gated_decode", "tg_debug_set_select_wait_limit", "tg_device_status",
+                   "tg_project_rope_gather", "tg_topk_select_after_gate_kept_scores", "tg_topk_select_noalloc_status",
+                   "tg_debug_set_cta_pairs"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -453,6 +456,11 @@ def tg_gated_decode(q, k_cache, v_cache, out, workspace, s_cache=None, gain=None
 def tg_debug_set_select_wait_limit(ns: int) -> None:
     """Test hook: the select's grid-barrier time limit on the current device (0 = the default)."""
     _check("tg_debug_set_select_wait_limit", lib().tg_debug_set_select_wait_limit(ctypes.c_uint64(ns)))
+
+
+def tg_debug_set_cta_pairs(enabled: bool) -> None:
+    """Test hook: False makes the gate (d_g = 256) and the projection run their one-CTA kernels."""
+    _check("tg_debug_set_cta_pairs", lib().tg_debug_set_cta_pairs(1 if enabled else 0))
 
 
 def tg_device_status(workspace, stream=None) -> int:

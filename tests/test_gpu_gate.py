@@ -171,3 +171,15 @@ def test_gate_and_select_pair(N, d, d_g, db, de, k):
         # the first-pass count (2048 words after the status header and the barrier words) is zero again
         hist0 = ws[256 + 256: 256 + 256 + 2048 * 4].view(torch.int32)
         assert int(hist0.abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("N,d,bias,gamma", [(129, 128, True, False), (4099, 2048, False, True), (300, 8192, True, True)])
+def test_gate_one_cta_kernel_d_g_256(N, d, bias, gamma):
+    # d_g = 256 on the one-CTA kernel (taken where a device offers no clusters of 2)
+    tg.tg_debug_set_cta_pairs(False)
+    try:
+        w = synth.scaled(synth.L16K, N=N, doc_end=N, d=d, d_g=256, n_scaled=min(8, N), seed=N + d + 7)
+        gi = synth.gate_inputs(w, with_bias=bias, with_gamma=gamma)
+        _check(_gpu_scores(gi), _oracle_scores(gi))
+    finally:
+        tg.tg_debug_set_cta_pairs(True)

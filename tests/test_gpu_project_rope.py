@@ -105,3 +105,26 @@ def test_project_rope_gather_matches_dense(N, K, d, Hq, Hkv, d_h, bad):
         outs.append((qkv.cpu(), v16.cpu()))
     assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16))
     assert torch.equal(outs[0][1].view(torch.int16), outs[1][1].view(torch.int16))
+
+
+@pytest.fixture
+def one_cta_kernels():
+    # the one-CTA projection kernel (taken where a device offers no clusters of 2)
+    tg.tg_debug_set_cta_pairs(False)
+    yield
+    tg.tg_debug_set_cta_pairs(True)
+
+
+@pytest.mark.parametrize("K,d,Hq,Hkv,d_h", [(300, 256, 4, 2, 128), (4608, 2048, 16, 8, 128)])
+def test_project_rope_one_cta_kernel(one_cta_kernels, K, d, Hq, Hkv, d_h):
+    rows = None if K <= 1000 else np.unique(np.concatenate([np.arange(0, K, 37), np.arange(K - 40, K)]))
+    got, want, absum, v16, Hq, Hkv, d_h = run(K, d, Hq, Hkv, d_h, seed=K + d + 1, rows=rows)
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - want) <= half_ulp_bf16(want) + 2.0 ** -20 * 2 * absum + 1e-6)
+    wv = want[:, (Hq + Hkv) * d_h:]
+    assert np.all(np.abs(v16 - wv) <= 2.0 ** -11 * np.abs(wv) + 2.0 ** -20 * 2 * absum[:, (Hq + Hkv) * d_h:] + 1e-6)
+
+
+@pytest.mark.parametrize("N,K,d,Hq,Hkv,d_h,bad", [(1000, 300, 256, 4, 2, 128, None), (5000, 129, 512, 4, 2, 64, 5)])
+def test_project_rope_gather_one_cta_kernel(one_cta_kernels, N, K, d, Hq, Hkv, d_h, bad):
+    test_project_rope_gather_matches_dense(N, K, d, Hq, Hkv, d_h, bad)
