@@ -470,13 +470,12 @@ def run_tokengate(args, rank, world, local_rank):
 
     gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     # (3) per-step kernel times in the step's own context and without host launch gaps: one CUDA graph
-    # per prefix of the step (gate; gate + select; ...), each replayed R times between its own events,
-    # the prefixes taken in turn (round r replays every prefix once, so a drift of the clock over the
-    # run affects them alike); a step's time is the difference between the median times of the prefix
-    # that ends with it and the prefix before it.  Every replay follows a 256 MB L2 flush, so each
-    # prefix's gate starts from the same L2 state (a gate right after a gate runs ~10% slower than after
-    # other work, which would shift time from the gate's prefix into the select's difference).
-    R = max(20, min(K, 60))
+    # per prefix of the step (gate; gate + select; ...), each replayed R times between its own events;
+    # a step's time is the difference between the mean times of the prefix that ends with it and the
+    # prefix before it.  Every replay follows a 256 MB L2 flush, so each prefix's gate starts from the
+    # same L2 state (a gate right after a gate runs ~10% slower than after other work, which would
+    # shift time from the gate's prefix into the select's difference).
+    R = max(10, min(K, 40))
     flush_each = flush if flush is not None else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     prefix_graphs, staged_err = [], None
     try:
@@ -520,9 +519,8 @@ def run_tokengate(args, rank, world, local_rank):
                 torch.distributed.barrier()
         # (3) the step's prefixes
         if not staged_failed:
-            for r in range(R):
-                for gs, evs in zip(prefix_graphs, pev):
-                    e0, e1 = evs[r]
+            for gs, evs in zip(prefix_graphs, pev):
+                for e0, e1 in evs:
                     flush_each.fill_(1)
                     e0.record()
                     gs.replay()
@@ -534,11 +532,11 @@ def run_tokengate(args, rank, world, local_rank):
     stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / K for j, s in enumerate(stages)}
     stage_timing = "kernel-by-kernel launches of the timed steps (host launch gaps included)"
     if not staged_failed:
-        prefix_ms = [reduce_max(statistics.median(e0.elapsed_time(e1) for e0, e1 in evs), dev) for evs in pev]
+        prefix_ms = [reduce_max(sum(e0.elapsed_time(e1) for e0, e1 in evs) / R, dev) for evs in pev]
         stage_ms = {s: prefix_ms[j] - (prefix_ms[j - 1] if j else 0.0) for j, s in enumerate(stages)}
         stage_timing = (f"step prefixes (gate; gate + select; ...) each captured in a CUDA graph and replayed {R} "
-                        f"times between events, the prefixes in turn, each replay after a 256 MB L2 flush; a "
-                        f"step's time is the difference of consecutive prefix medians")
+                        f"times between events, each replay after a 256 MB L2 flush; a step's time is the "
+                        f"difference of consecutive prefix means")
     del prefix_graphs
     status = layer.device_status()
     ungraphed = {"ms_per_step": ms_launched, "value": job_throughput(w.N, world, ms_launched), "unit": "tokens/s"}
