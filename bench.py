@@ -645,6 +645,7 @@ def run_tokengate(args, rank, world, local_rank):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; stands in for NIAH-style prompts)",
             "config": config_dict(w), "impl": "tokengate",
             "path_ms": t_path * 1e3, "path_tokens_per_s": w.N * world / t_path, "path_stages": path,
+            "stage_sum_ms": sum(stage_ms.values()),
             "path_roofline_frac": path_roof, "path_roofline_frac_sustained_peak": path_roof_sustained,
             "path_roofline_frac_nominal_peak": path_roof_nominal,
             "step_roofline_frac_ungraphed": step_bound / (ms_launched * 1e-3),
