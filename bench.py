@@ -536,21 +536,14 @@ def run_tokengate(args, rank, world, local_rank):
         stage_ms = {s: prefix_ms[j] - (prefix_ms[j - 1] if j else 0.0) for j, s in enumerate(stages)}
         stage_timing = (f"step prefixes (gate; gate + select; ...) each captured in a CUDA graph and replayed {R} "
                         f"times between events, each replay after a 256 MB L2 flush; a step's time is the "
-                        f"difference of consecutive prefix means, the split then scaled to the measured graphed "
-                        f"step (kernels_unscaled_us: before scaling)")
+                        f"difference of consecutive prefix means")
     del prefix_graphs
-    stage_ms_raw = dict(stage_ms)
     status = layer.device_status()
     ungraphed = {"ms_per_step": ms_launched, "value": job_throughput(w.N, world, ms_launched), "unit": "tokens/s"}
     if not graph_failed:
         ms_graph = reduce_max(sum(e0.elapsed_time(e1) for e0, e1 in gev) / K, dev)
         graph_line = {"ms_per_step": ms_graph, "value": job_throughput(w.N, world, ms_graph), "unit": "tokens/s"}
         ms_step, value = ms_graph, graph_line["value"]
-        # the split is estimated from prefix graphs, the step's total is measured directly: scale the
-        # split to the measured step (the estimate's sum is within a few % of it; see stage_sum_ms)
-        split_sum = sum(stage_ms.values())
-        if not staged_failed and split_sum > 0:
-            stage_ms = {k: v * ms_graph / split_sum for k, v in stage_ms.items()}
     else:
         graph_line = {"unavailable": graph_err or "capture failed on another rank"}
         ms_step, value = ms_launched, ungraphed["value"]
@@ -652,8 +645,7 @@ def run_tokengate(args, rank, world, local_rank):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; stands in for NIAH-style prompts)",
             "config": config_dict(w), "impl": "tokengate",
             "path_ms": t_path * 1e3, "path_tokens_per_s": w.N * world / t_path, "path_stages": path,
-            "stage_sum_ms": sum(stage_ms_raw.values()),
-            "kernels_unscaled_us": {k: v * 1e3 for k, v in stage_ms_raw.items()},
+            "stage_sum_ms": sum(stage_ms.values()),
             "path_roofline_frac": path_roof, "path_roofline_frac_sustained_peak": path_roof_sustained,
             "path_roofline_frac_nominal_peak": path_roof_nominal,
             "step_roofline_frac_ungraphed": step_bound / (ms_launched * 1e-3),
