@@ -472,11 +472,19 @@ def run_tokengate(args, rank, world, local_rank):
     # (3) per-step kernel times in the step's own context and without host launch gaps: one CUDA graph
     # per prefix of the step (gate; gate + select; ...), each replayed R times between its own events;
     # a step's time is the difference between the mean times of the prefix that ends with it and the
-    # prefix before it.  Every replay follows a 256 MB L2 flush, so each prefix's gate starts from the
-    # same L2 state (a gate right after a gate runs ~10% slower than after other work, which would
-    # shift time from the gate's prefix into the select's difference).
+    # prefix before it.  Every replay follows a 256 MB pass over L2, so each prefix's gate starts from
+    # the same L2 state (a gate right after a gate runs ~10% slower than after other work, which would
+    # shift time from the gate's prefix into the select's difference): the same write flush the timed
+    # steps have where they have one, else a read of 256 MB, which evicts L2 without leaving dirty
+    # lines whose write-back the next gate would pay and the timed steps do not.
     R = max(10, min(K, 40))
-    flush_each = flush if flush is not None else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evict = None if flush is not None else torch.empty(256 << 20, dtype=torch.uint8, device=dev).view(torch.int32)
+
+    def before_prefix():
+        if flush is not None:
+            flush.fill_(1)
+        else:
+            evict.max()
     prefix_graphs, staged_err = [], None
     try:
         calls = list(layer.stage_calls(h).values())
@@ -521,7 +529,7 @@ def run_tokengate(args, rank, world, local_rank):
         if not staged_failed:
             for gs, evs in zip(prefix_graphs, pev):
                 for e0, e1 in evs:
-                    flush_each.fill_(1)
+                    before_prefix()
                     e0.record()
                     gs.replay()
                     e1.record()
@@ -535,8 +543,8 @@ def run_tokengate(args, rank, world, local_rank):
         prefix_ms = [reduce_max(sum(e0.elapsed_time(e1) for e0, e1 in evs) / R, dev) for evs in pev]
         stage_ms = {s: prefix_ms[j] - (prefix_ms[j - 1] if j else 0.0) for j, s in enumerate(stages)}
         stage_timing = (f"step prefixes (gate; gate + select; ...) each captured in a CUDA graph and replayed {R} "
-                        f"times between events, each replay after a 256 MB L2 flush; a step's time is the "
-                        f"difference of consecutive prefix means")
+                        f"times between events, each replay after a 256 MB pass over L2 ({'write' if flush is not None else 'read'}); "
+                        f"a step's time is the difference of consecutive prefix means")
     del prefix_graphs
     status = layer.device_status()
     ungraphed = {"ms_per_step": ms_launched, "value": job_throughput(w.N, world, ms_launched), "unit": "tokens/s"}
@@ -615,11 +623,21 @@ def run_tokengate(args, rank, world, local_rank):
     roof["peak_source"] = peaks["source"] + (" (burst bf16)" if roof["bound"] == "tensor" else " (HBM copy)")
     if roof["bound"] == "tensor":
         roof["frac_of_sustained_peak"] = roof["achieved"] / peaks["bf16_tflops_sustained"]
-    # the specification's path (gate, select, gather, attention) and the whole step (plus the projection)
-    # the spec steps that run as stages of their own (a layer that gathers inside the projection's
-    # operand loads has no gather stage: that work is inside "proj", which the step fractions cover)
+    # the specification's path (gate, select, gather, attention) and the whole step (plus the projection):
+    # the path's steps that run as stages of their own (a layer that gathers inside the projection's
+    # operand loads has no gather stage: that work is inside "proj", which the step fractions cover).
+    # The path's time is the measured graphed step minus the estimated time of the stages off the path
+    # (one estimate instead of the sum of four, each a difference of two prefix means); the sum of the
+    # path's own stage estimates is reported beside it.
     path = [s for s in ("gate", "select", "gather", "attn") if s in stages]
-    t_path = sum(stage_ms[s] for s in path) * 1e-3
+    off_path = [s for s in stages if s not in path]
+    t_split = sum(stage_ms[s] for s in path) * 1e-3
+    t_path, path_method = t_split, "sum of the path's stage times"
+    if not graph_failed and not staged_failed:
+        t_rest = ms_step * 1e-3 - sum(stage_ms[s] for s in off_path) * 1e-3
+        if t_rest > 0:
+            t_path = t_rest
+            path_method = f"graphed step minus the stage times off the path ({', '.join(off_path)})"
     path_roof = sum(lower_bound(s) for s in path) / t_path
     path_roof_sustained = sum(lower_bound(s, peaks["bf16_tflops_sustained"]) for s in path) / t_path
     path_roof_nominal = sum(max(work[s]["flops"] / 2.25e15, work[s]["bytes"] / 8.0e12) for s in path) / t_path
@@ -645,6 +663,8 @@ def run_tokengate(args, rank, world, local_rank):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; stands in for NIAH-style prompts)",
             "config": config_dict(w), "impl": "tokengate",
             "path_ms": t_path * 1e3, "path_tokens_per_s": w.N * world / t_path, "path_stages": path,
+            "path_method": path_method, "path_ms_from_split": t_split * 1e3,
+            "path_roofline_frac_from_split": sum(lower_bound(s) for s in path) / t_split,
             "stage_sum_ms": sum(stage_ms.values()),
             "path_roofline_frac": path_roof, "path_roofline_frac_sustained_peak": path_roof_sustained,
             "path_roofline_frac_nominal_peak": path_roof_nominal,
