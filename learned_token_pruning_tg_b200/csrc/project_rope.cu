@@ -29,8 +29,11 @@
 //               tile's main loop
 // Every wait is bounded (TG_STATUS_PROJECT_TIMEOUT).
 // Where the device offers clusters of 2, the same roles run on CTA pairs with
-// 256 x 256 tiles (project_rope_pair_kernel below), which halves the W bytes
-// each SM moves per stage.
+// 256 x 256 tiles and a 6-deep ring (project_rope_pair_kernel below), which
+// halves the W bytes each SM moves per stage.
+// With a row index array (tg_project_rope_gather) the producer warp fetches the
+// x tiles as rows of h instead: lane l issues one TMA gather4 copy of tile rows
+// 4l .. 4l + 3 per 64-column step, and each lane checks its indices.
 #include <cuda_fp16.h>
 
 #include <cmath>
